@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the TriAttention KV-cache compression pass on B200.
+
+Workload: the Qwen3-32B-shape long-reasoning decode cache (64 layers, 64 query
+/ 8 KV heads, head_dim 128, 32768 cached tokens, budget 2048, window 256,
+NEOX pairing, theta 1e4), seeded synthetic bf16 K/V.  One step = one full
+compression pass (coefficients, scoring + normalize-then-max + selection,
+in-place compaction of K, V and positions) through the C ABI.
+
+Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
+on the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "keys scored+selected/s (Qwen3-32B-shape 32K pass)"
+UNIT = "keys/s"
+
+
+def _env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("tria_kernels.cu", "tria_internal.h"):
+        with open(os.path.join(ROOT, "key_retention_scoring_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if it
+    was taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch_full_size")
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons with NVML while the
+    timed region runs (reads only)."""
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.index, self.period = index, period_s
+        self.samples = []
+        self._stop = threading.Event()
+        self._t = None
+        self.max_mhz = None
+        self.error = None
+
+    def __enter__(self):
+        try:
+            import pynvml as N
+
+            N.nvmlInit()
+            self._N = N
+            self._h = N.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(self._h, N.NVML_CLOCK_SM)
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        except Exception as e:  # NVML missing: report it, do not fail the bench
+            self.error = repr(e)
+        return self
+
+    def _run(self):
+        N = self._N
+        while not self._stop.is_set():
+            try:
+                mhz = N.nvmlDeviceGetClockInfo(self._h, N.NVML_CLOCK_SM)
+                reasons = N.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                pw = N.nvmlDeviceGetPowerUsage(self._h) / 1000.0
+                self.samples.append((mhz, reasons, pw))
+            except Exception as e:
+                self.error = repr(e)
+                return
+            time.sleep(self.period)
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        names = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+                 0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+                 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+                 0x100: "display_clock_setting"}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0, "error": self.error}
+        mhz = [s[0] for s in self.samples]
+        seen = set()
+        for _, r, _ in self.samples:
+            for bit, n in names.items():
+                if r & bit:
+                    seen.add(n)
+        seen.discard("gpu_idle")
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(seen), "samples": len(mhz),
+                "power_w_median": round(statistics.median(s[2] for s in self.samples), 1)}
+
+
+# ---------------------------------------------------------------------------
+# oracle (CPU baseline and reference arm)
+# ---------------------------------------------------------------------------
+def oracle_unit_keys_per_s(cfg, seconds: float, max_units: int = 64):
+    """Time the fp64 oracle (folded form, normalize-then-max, selection) on
+    units of the workload generated on the host with the same recipe."""
+    import synth
+    from oracle import tria_oracle as O
+
+    re, im, am = synth.make_stats(cfg)
+    centers = synth.make_centers(cfg)
+    omega = O.band_frequencies(cfg.head_dim, cfg.theta)
+    G = cfg.group
+    N = int(synth.seq_lengths(cfg)[0])
+    spent, keys, units = 0.0, 0, 0
+    rng = np.random.default_rng(0)
+    while spent < seconds and units < max_units:
+        l, h = int(rng.integers(cfg.n_layers)), int(rng.integers(cfg.n_kv_heads))
+        bits = synth.host_key_rows(cfg, centers, 0, l, h, np.arange(N))
+        k = O.bf16_bits_to_f64(bits)
+        qc = re[l, h * G:(h + 1) * G].astype(np.float64) + 1j * im[l, h * G:(h + 1) * G]
+        qa = am[l, h * G:(h + 1) * G].astype(np.float64)
+        t0 = time.perf_counter()
+        O.compress_unit(k, np.arange(N), N - 1, qc, qa, omega, cfg.pairing, cfg.budget,
+                        cfg.window, cfg.sinks, cfg.offset_log2_max)
+        spent += time.perf_counter() - t0
+        keys += N
+        units += 1
+    return keys / spent, units, spent
+
+
+def run_reference(args, rank, world):
+    import synth
+
+    if rank != 0:
+        return 0
+    cfg = synth.CONFIGS[args.config]
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        v, units, spent = oracle_unit_keys_per_s(cfg, 0.0, max_units=1)
+        if i >= args.warmup:
+            per_step.append(spent)
+    N = int(synth.seq_lengths(cfg)[0])
+    t = sum(per_step)
+    value = args.steps * N / t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_desc(cfg, "one unit (1 layer x 1 KV head) per step"),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{args.steps} units of {N} keys (G={cfg.group}), fp64 numpy, "
+                                   "folded form + z-norm + selection"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_desc(cfg, extra=None):
+    d = {"workload": cfg.name, "layers": cfg.n_layers, "q_heads": cfg.n_q_heads,
+         "kv_heads": cfg.n_kv_heads, "head_dim": cfg.head_dim, "seq_len": cfg.seq_len,
+         "n_seq": cfg.n_seq, "budget": cfg.budget, "window": cfg.window, "sinks": cfg.sinks,
+         "pairing": "neox" if cfg.pairing == 0 else "interleaved", "theta": cfg.theta,
+         "offsets": f"2^0..2^{cfg.offset_log2_max}",
+         "l2": "inputs (4.3 GB of K) larger than L2, plus a 256 MB L2 flush before each pass",
+         "restore": "rows overwritten by compaction restored between passes, outside the "
+                    "per-pass CUDA events"}
+    if extra:
+        d["sample"] = extra
+    return d
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="tria", choices=["tria", "reference"])
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-extras", action="store_true", help="skip e2e, run16 and CPU baseline")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = _env_int("RANK", 0)
+    world = _env_int("WORLD_SIZE", 1)
+    local = _env_int("LOCAL_RANK", 0)
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+
+    import key_retention_scoring_b200 as T
+    import synth
+    from key_retention_scoring_b200 import build as tria_build
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    tria_build.build()
+    synth.build()
+
+    base = synth.CONFIGS[args.config]
+    cfg = base.scaled(seed=base.seed + 1000 * rank)   # each rank: its own sequence (weak scaling)
+    w = synth.Workload(cfg)
+    re, im, am = w.stats
+    st = T.tria_load_stats(T.model_desc(cfg.n_layers, cfg.n_q_heads, cfg.n_kv_heads, cfg.pairing,
+                                        cfg.theta, cfg.offset_log2_max), re, im, am)
+    cache = T.Cache.from_workload(w)
+    prm = T.params(cfg.budget, cfg.window, cfg.sinks)
+    ws = T.alloc_workspace(T.tria_workspace_size(st, cache, prm))
+    T.tria_read_device_status(ws)
+    B = cfg.budget
+    kept = torch.empty((cfg.n_seq, cfg.n_layers, cfg.n_kv_heads, B), dtype=torch.int32,
+                       device="cuda")
+    # backups of what compaction overwrites
+    kb = [t[:, :, :B].clone() for t in w.k]
+    vb = [t[:, :, :B].clone() for t in w.v]
+    pb = w.positions[..., :B].clone()
+    lens0 = w.seq_lens.clone()
+    qpos0 = w.query_pos.clone()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+
+    def restore():
+        for l in range(cfg.n_layers):
+            w.k[l][:, :, :B].copy_(kb[l])
+            w.v[l][:, :, :B].copy_(vb[l])
+        w.positions[..., :B].copy_(pb)
+        w.seq_lens.copy_(lens0)
+        w.query_pos.copy_(qpos0)
+        flush.zero_()
+
+    stream = torch.cuda.current_stream()
+
+    def timed_pass():
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        T.tria_set_pass_events(evs)
+        T.tria_compress_pass(st, cache, prm, kept, ws, stream=stream)
+        T.tria_set_pass_events(None)
+        return evs
+
+    for _ in range(args.warmup):
+        restore()
+        timed_pass()
+    torch.cuda.synchronize()
+    if T.tria_read_device_status(ws) != 0:
+        raise RuntimeError("device status flags set")
+    # moved rows of one pass (for the compaction bytes)
+    kh = kept.cpu().numpy()
+    moved = int(np.sum(kh != np.arange(B)[None, None, None, :]))
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    all_evs = []
+    with ClockSampler(local) as clk:
+        br0 = torch.cuda.Event(enable_timing=True)
+        br1 = torch.cuda.Event(enable_timing=True)
+        br0.record()
+        for _ in range(args.steps):
+            restore()
+            all_evs.append(timed_pass())
+        br1.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    pass_ms = [e[0].elapsed_time(e[3]) for e in all_evs]
+    coef_ms = [e[0].elapsed_time(e[1]) for e in all_evs]
+    score_ms = [e[1].elapsed_time(e[2]) for e in all_evs]
+    compact_ms = [e[2].elapsed_time(e[3]) for e in all_evs]
+    ms = statistics.mean(pass_ms)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    N = cfg.seq_len
+    units = cfg.n_seq * cfg.n_layers * cfg.n_kv_heads
+    keys = units * N
+    C = N - cfg.window - cfg.sinks
+    score_bytes = units * C * 256
+    compact_bytes = moved * 1024
+    hbm, peak_kind = peaks()
+    score_avg = statistics.mean(score_ms)
+    compact_avg = statistics.mean(compact_ms)
+    achieved = score_bytes / (score_avg * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": keys * world / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": config_desc(cfg),
+        "us_per_pass": ms * 1e3,
+        "pass_gbs": (score_bytes + compact_bytes) / (ms * 1e-3) / 1e9,
+        "keys_per_s_per_query_head": keys * world * cfg.group / (ms * 1e-3),
+        "kernels_us": {"coef": 1e3 * statistics.mean(coef_ms), "score_select": 1e3 * score_avg,
+                       "compact": 1e3 * compact_avg},
+        "roofline": {"bound": "hbm", "kernel": "score_kernel (score + normalize-then-max + select)",
+                     "achieved": achieved, "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": recorded_traffic("score_kernel"),
+                     "algorithmic_bytes": score_bytes},
+        "compact_roofline": {"achieved": compact_bytes / (compact_avg * 1e-3) / 1e9, "peak": hbm,
+                             "unit": "GB/s",
+                             "frac": compact_bytes / (compact_avg * 1e-3) / 1e9 / hbm,
+                             "algorithmic_bytes": compact_bytes, "moved_rows": moved},
+        "bracket_ms_per_step": br0.elapsed_time(br1) / args.steps,
+        "clocks": clk.summary(),
+        "gpu_launches": 3 * args.steps,
+    }
+
+    if not args.no_extras:
+        line["run16"] = run16(T, w, st, cache, prm, ws, kept, restore)
+        line["e2e"] = e2e(T, torch, w, st, cache, prm, ws, kept, restore, args.e2e_steps, keys, world)
+        if rank == 0 and world == 1:
+            v, n_units, spent = oracle_unit_keys_per_s(cfg, args.cpu_seconds)
+            line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                    "sample": f"{n_units} units of {N} keys (G={cfg.group}), "
+                                              f"{spent:.1f} s, fp64 numpy (single thread), "
+                                              "folded form + z-norm + selection"}
+    T.tria_set_pass_events(None)
+    st.free()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def run16(T, w, st, cache, prm, ws, kept, restore):
+    """The decode run: a first pass at 32K, then 15 passes each after 128
+    appended tokens (append excluded from the pass times)."""
+    import torch
+
+    restore()
+    torch.cuda.synchronize()
+    pass_us, append_ms = [], []
+    for i in range(16):
+        if i:
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record()
+            w.append(128)
+            a1.record()
+            torch.cuda.synchronize()
+            append_ms.append(a0.elapsed_time(a1))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        T.tria_compress_pass(st, cache, prm, kept, ws)
+        e1.record()
+        torch.cuda.synchronize()
+        pass_us.append(1e3 * e0.elapsed_time(e1))
+    w.next_pos = w.lens.astype(np.int64).copy()
+    restore()
+    return {"first_pass_us": pass_us[0], "steady_pass_us_mean": statistics.mean(pass_us[1:]),
+            "steady_keys_per_pass": int(w.cfg.n_layers * w.cfg.n_kv_heads * (w.cfg.budget + 128)),
+            "total_pass_ms": sum(pass_us) / 1e3, "append_ms_mean": statistics.mean(append_ms)}
+
+
+def e2e(T, torch, w, st, cache, prm, ws, kept, restore, steps, keys, world):
+    """Same metric through the C ABI with host buffers: every step copies the
+    K, V and positions of the cache from pinned host memory, runs the pass and
+    reads the kept lists back."""
+    restore()
+    torch.cuda.synchronize()
+    hk = [t.cpu().pin_memory() for t in w.k]
+    hv = [t.cpu().pin_memory() for t in w.v]
+    hp = w.positions.cpu().pin_memory()
+    hl = w.seq_lens.cpu().pin_memory()
+    hq = w.query_pos.cpu().pin_memory()
+    hkept = torch.empty(kept.shape, dtype=kept.dtype).pin_memory()
+    h2d = sum(t.numel() * 2 for t in hk) + sum(t.numel() * 2 for t in hv) + hp.numel() * 4 \
+        + hl.numel() * 4 + hq.numel() * 8
+    d2h = hkept.numel() * 4
+    times = []
+    for i in range(steps + 1):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for l in range(len(hk)):
+            w.k[l].copy_(hk[l], non_blocking=True)
+            w.v[l].copy_(hv[l], non_blocking=True)
+        w.positions.copy_(hp, non_blocking=True)
+        w.seq_lens.copy_(hl, non_blocking=True)
+        w.query_pos.copy_(hq, non_blocking=True)
+        T.tria_compress_pass(st, cache, prm, kept, ws)
+        hkept.copy_(kept, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        if i:
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.mean(times)
+    del hk, hv, hp
+    return {"value": keys * world / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": steps}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

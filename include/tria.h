@@ -1,0 +1,270 @@
+/*
+ * tria.h - C ABI of the B200 (sm_100a) TriAttention KV-cache compression pass.
+ *
+ * The pass, for every cached key of every layer and KV head ("unit" =
+ * (sequence, layer, KV head)):
+ *   1. splits the 128-wide head into 64 RoPE bands (NEOX half split or
+ *      interleaved pairs) and scores the key against calibrated query
+ *      statistics:  S~(k) = S~_trig(k) + S_norm(k)
+ *      - S~_trig is the trigonometric term of Eq. (2) of the academ.us article
+ *        2607.13051 ("a small improvement to one step of TriAttention"),
+ *        averaged over the future offsets D = {1, 2, 4, ..., 2^m} (Eq. 4),
+ *        evaluated through the folded centers mu'_f = E[q_f] W_f of Eq. (7);
+ *      - S_norm(k) = sum_f (E|q_f| - |E q_f|) |k_f|, the distance-independent
+ *        term that weighs a key's own band magnitudes by (1 - R_f)
+ *        (ghidav.me, "TriAttention, or: what a rotating query already knows",
+ *        section "The Method");
+ *   2. z-normalises the score of each query head over the unit's candidates
+ *      and takes the max over the query heads sharing the KV head
+ *      (article 2607.13051, sec. 4, "normalize-then-max");
+ *   3. keeps the top-K candidates, always keeping the first `sinks` and the
+ *      last `window` slots, `budget` rows in all (ghidav.me, "The Method":
+ *      sort, keep the top B, drop the rest; GitHub issue #10 of the llama.cpp
+ *      TurboQuant HIP fork, runtime log: window 256, interval 128, sink 0);
+ *   4. gathers the kept K/V rows to the front of each unit, in place, in
+ *      ascending slot order ("per-layer compaction path", triattention README).
+ *
+ * Conventions for every entry point:
+ *   - Pointers documented "device" are CUDA device pointers owned by the
+ *     caller; "host" pointers are read during the call only.
+ *   - All work is enqueued on `stream` (NULL = legacy default stream) and is
+ *     asynchronous; no entry point synchronises except tria_load_stats,
+ *     tria_free_stats and tria_read_device_status.
+ *   - Arguments are validated on the host before anything is enqueued; a
+ *     validation failure returns an error and enqueues nothing.
+ *   - Launch failures return TRIA_ERR_CUDA.
+ *   - The library allocates device memory only in tria_load_stats (the stats
+ *     object); scoring, selection and compaction never allocate.
+ *   - bf16 K/V rows are 128 elements (256 bytes); row starts must be 16-byte
+ *     aligned (strides multiples of 8 elements, 16-byte aligned bases).
+ *   - A unit whose length N is at most the budget is left unchanged.
+ *   - Floating point decides the kept set only through the fp32 aggregated
+ *     score agg (below); exactly equal agg go to the lower slot; -0.0 equals
+ *     +0.0; NaN ranks below every number.
+ */
+#ifndef TRIA_H
+#define TRIA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *tria_stream_t;
+
+typedef enum {
+  TRIA_OK = 0,
+  TRIA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or range */
+  TRIA_ERR_UNSUPPORTED = 2, /* valid but not built: head_dim != 128, G > 16 */
+  TRIA_ERR_WORKSPACE = 3,   /* workspace null or smaller than required */
+  TRIA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+  TRIA_ERR_OOM = 5          /* device allocation failed (tria_load_stats) */
+} tria_status;
+
+typedef enum {
+  TRIA_PAIR_NEOX = 0,        /* band f = x[f] + i x[f + d/2]   (Qwen, NEOX)   */
+  TRIA_PAIR_INTERLEAVED = 1  /* band f = x[2f] + i x[2f + 1]   (Llama, NORM)  */
+} tria_pairing;
+
+typedef enum {
+  TRIA_LAYOUT_CONTIGUOUS = 0, /* row = k_layers[l] + s*stride_seq + h*stride_head + t*stride_token */
+  TRIA_LAYOUT_PAGED = 1       /* row = k_layers[l] + block_table[s][t / block_size]*stride_block
+                                       + (t % block_size)*stride_token + h*stride_head */
+} tria_layout;
+
+#define TRIA_HEAD_DIM 128
+#define TRIA_MAX_LAYERS 256
+#define TRIA_MAX_GROUP 16
+#define TRIA_MAX_SEQS 1024
+
+/* Model shape and RoPE convention. */
+typedef struct {
+  int n_layers;        /* 1 .. TRIA_MAX_LAYERS                                  */
+  int n_q_heads;       /* Hq; a multiple of n_kv_heads                          */
+  int n_kv_heads;      /* Hkv; G = Hq / Hkv in 1 .. TRIA_MAX_GROUP              */
+  int head_dim;        /* d; only 128 is built                                  */
+  int pairing;         /* tria_pairing                                          */
+  double rope_theta;   /* theta of omega_f = theta^(-2f/d) (article 2607.13051,
+                          sec. 2, list under Eq. 2); > 1                        */
+  int offset_log2_max; /* m of D = {2^0 .. 2^m}; the published method uses 16
+                          (article 2607.13051, Eq. 4); 0 .. 30                  */
+} tria_model_desc;
+
+/* Opaque, library-owned device copy of the folded statistics. */
+typedef struct tria_stats tria_stats;
+
+/* The caller's KV cache.  Every pointer stays owned by the caller. */
+typedef struct {
+  int layout;                /* tria_layout                                          */
+  int n_seq;                 /* 1 .. TRIA_MAX_SEQS                                   */
+  int max_seq_len;           /* host: upper bound of every seq_lens[s]; sizes the
+                                candidate axis C_max = max_seq_len - window - sinks  */
+  void *const *k_layers;     /* host array [n_layers] of device pointers, bf16 K     */
+  void *const *v_layers;     /* host array [n_layers] of device pointers, bf16 V;
+                                needed by compaction only                            */
+  int64_t stride_seq;        /* elements between sequences (contiguous layout)       */
+  int64_t stride_head;       /* elements between KV heads                            */
+  int64_t stride_token;      /* elements between slots (contiguous) or between the
+                                rows of one block (paged)                            */
+  int64_t stride_block;      /* elements between blocks (paged)                      */
+  const int32_t *block_table;/* device [n_seq][max_blocks_per_seq] (paged)           */
+  int max_blocks_per_seq;    /* paged                                                */
+  int block_size;            /* rows per block (paged), 1 .. 1024                    */
+  int32_t *seq_lens;         /* device [n_seq] cached tokens N per sequence; set to
+                                min(N, budget) by tria_compact when it covers the last
+                                layer                                                */
+  const int64_t *query_pos;  /* device [n_seq] position p_q of the current query: the
+                                position of the newest cached token (offsets
+                                delta in D are added to it)                          */
+  int32_t *positions;        /* optional device [n_seq][n_layers][n_kv_heads][max_seq_len]
+                                token position of every slot; compacted with the
+                                rows when non-null.  Scoring never reads it: the
+                                post-RoPE key already carries its position.          */
+} tria_cache_view;
+
+/* Retention parameters (one set for all units of a call). */
+typedef struct {
+  int budget;  /* B: rows kept per unit, window and sinks included; >= window + sinks */
+  int window;  /* W: the newest W slots are always kept                               */
+  int sinks;   /* S: the oldest S slots are always kept                               */
+} tria_params;
+
+/* Human-readable name of a status code (static string). */
+const char *tria_status_string(tria_status status);
+
+/* Library version string (static). */
+const char *tria_version(void);
+
+/*
+ * tria_load_stats - fold calibrated query statistics into a device object.
+ *
+ * Inputs (host, fp32, [n_layers][n_q_heads][head_dim/2], band f innermost):
+ *   q_mean_re, q_mean_im : E[Re q_f], E[Im q_f] of the pre-RoPE query bands;
+ *   q_abs_mean           : E|q_f|
+ *   (the three statistics of the calibration tool in GitHub issue #10 of the
+ *   llama.cpp TurboQuant HIP fork, paired as desc->pairing says);
+ *   band_mask            : optional host [head_dim/2] per-band multiplier of
+ *                          |mu'_f| (the high-frequency mask of article
+ *                          2607.13051, sec. 7); NULL = all ones.
+ * On the host, in fp64: W_f = (1/|D|) sum_{delta in D} e^{i omega_f delta}
+ * (Eq. 6), mu'_f = E[q_f] W_f mask_f (Eq. 7), w_f = E|q_f| - |E q_f|.
+ * The result is copied to the device (stream-ordered, then synchronised).
+ * *out receives a new object; free it with tria_free_stats.
+ * Errors: INVALID_ARG (null pointer, non-finite input, bad desc),
+ * UNSUPPORTED (head_dim != 128, G > TRIA_MAX_GROUP), OOM, CUDA.
+ */
+tria_status tria_load_stats(const tria_model_desc *desc, const float *q_mean_re,
+                            const float *q_mean_im, const float *q_abs_mean,
+                            const float *band_mask, tria_stream_t stream,
+                            tria_stats **out);
+
+/* Free a stats object (synchronises the device first).  NULL is allowed. */
+tria_status tria_free_stats(tria_stats *stats);
+
+/* Copy of the model description a stats object was built with. */
+tria_status tria_stats_desc(const tria_stats *stats, tria_model_desc *desc_out);
+
+/*
+ * tria_workspace_size - device workspace bytes that tria_score, tria_select
+ * and tria_compress_pass need for this cache view, these parameters and the
+ * layer range [layer0, layer1).  The workspace is scratch: no state is kept
+ * between calls, and concurrent calls need separate workspaces.
+ * Errors: INVALID_ARG.
+ */
+tria_status tria_workspace_size(const tria_stats *stats, const tria_cache_view *cache,
+                                const tria_params *params, int layer0, int layer1,
+                                size_t *bytes);
+
+/*
+ * tria_score - averaged scores and the aggregated (normalize-then-max) score
+ * of every candidate slot of layers [layer0, layer1).
+ *
+ * Candidates of a unit with N cached rows are slots [sinks, N - window);
+ * C = N - window - sinks of them.  Outputs (device, fp32):
+ *   agg_out    [n_seq][layer1 - layer0][n_kv_heads][C_max]:
+ *              agg[c] = max_g (S~_g[c] - mean_g) / (std_g + 1e-6), mean and
+ *              population std of head g over the unit's C candidates;
+ *   scores_out optional [n_seq][layer1 - layer0][n_kv_heads][C_max][G]:
+ *              S~_g of candidate c for the G query heads of the KV head.
+ * Entries c >= C, and units with N <= budget, are not written.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+tria_status tria_score(const tria_stats *stats, const tria_cache_view *cache,
+                       const tria_params *params, int layer0, int layer1,
+                       float *agg_out, float *scores_out,
+                       void *workspace, size_t workspace_bytes, tria_stream_t stream);
+
+/*
+ * tria_select - kept slots of every unit of layers [layer0, layer1) from
+ * agg (layout of tria_score's agg_out).
+ *   kept_idx (device int32 [n_seq][layer1 - layer0][n_kv_heads][budget]):
+ *   ascending slots: 0 .. sinks-1, then the top K = budget - window - sinks
+ *   candidates by agg (ties: lower slot), then N-window .. N-1.  A unit with
+ *   N <= budget gets 0 .. N-1 followed by -1.
+ * Errors: INVALID_ARG, WORKSPACE, CUDA.
+ */
+tria_status tria_select(const tria_stats *stats, const tria_cache_view *cache,
+                        const tria_params *params, const float *agg, int layer0,
+                        int layer1, int32_t *kept_idx, void *workspace,
+                        size_t workspace_bytes, tria_stream_t stream);
+
+/*
+ * tria_compact - in-place gather of the kept K and V rows (and positions, if
+ * the view has them) of layers [layer0, layer1): row j of each unit becomes
+ * the old row kept_idx[j] (kept_idx as tria_select writes it; -1 entries and
+ * entries equal to j move nothing).  kept_idx must be strictly ascending
+ * with kept_idx[j] >= j (tria_select guarantees it); rows are byte-copied.
+ * When layer1 == n_layers, seq_lens[s] becomes min(N_s, budget) and, for the
+ * paged layout, the blocks of each sequence past ceil(budget / block_size)
+ * that held rows are listed in freed_blocks (device int32 [n_seq][max_blocks_per_seq],
+ * nullable) with their count in n_freed (device int32 [n_seq], nullable); the
+ * block table itself is not modified.
+ * Errors: INVALID_ARG, CUDA.
+ */
+tria_status tria_compact(const tria_stats *stats, const tria_cache_view *cache,
+                         const tria_params *params, const int32_t *kept_idx,
+                         int layer0, int layer1, int32_t *freed_blocks,
+                         int32_t *n_freed, tria_stream_t stream);
+
+/*
+ * tria_compress_pass - the whole pass over every layer: score, select and
+ * compact, with scores and agg kept in the workspace.  kept_idx: optional
+ * device [n_seq][n_layers][n_kv_heads][budget] copy of the kept slots (NULL:
+ * kept in the workspace only).  freed_blocks / n_freed as in tria_compact.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ */
+tria_status tria_compress_pass(const tria_stats *stats, const tria_cache_view *cache,
+                               const tria_params *params, int32_t *kept_idx,
+                               int32_t *freed_blocks, int32_t *n_freed,
+                               void *workspace, size_t workspace_bytes,
+                               tria_stream_t stream);
+
+/*
+ * tria_read_device_status - errors the kernels found in device-resident
+ * inputs during the calls that used this workspace (bit 0: a seq_lens entry
+ * outside [0, max_seq_len]; such a unit is skipped and its kept row is all
+ * -1), then clears them.  Synchronises `stream`.  *flags_out = 0 means none.
+ * The flags start undefined in a fresh workspace: read (and so clear) them
+ * once before the first call.
+ */
+tria_status tria_read_device_status(void *workspace, tria_stream_t stream,
+                                    int32_t *flags_out);
+
+/*
+ * tria_set_pass_events - kernel timing hook for tria_compress_pass (tracing).
+ * events: NULL to disable, or a host array of 4 cudaEvent_t created by the
+ * caller; the next tria_compress_pass calls made from this host thread record
+ * events[0] before the coefficient kernel, events[1] before the scoring
+ * kernel, events[2] before the compaction kernel and events[3] after it, on
+ * the pass's stream.  The array is copied; the events stay owned by the caller.
+ */
+tria_status tria_set_pass_events(void *const *events);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRIA_H */

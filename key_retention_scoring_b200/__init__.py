@@ -1,0 +1,262 @@
+"""Python binding of libtria.so, the sm_100a TriAttention KV-cache
+compression pass (C ABI in include/tria.h).
+
+Argument marshalling only: every step of the pass runs in the CUDA library.
+There is no CPU fallback; loading fails loudly when the library is missing.
+The entry points keep the C names: tria_load_stats, tria_workspace_size,
+tria_score, tria_select, tria_compact, tria_compress_pass, ...
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtria.so")
+
+TRIA_OK = 0
+STATUS_NAMES = {0: "TRIA_OK", 1: "TRIA_ERR_INVALID_ARG", 2: "TRIA_ERR_UNSUPPORTED",
+                3: "TRIA_ERR_WORKSPACE", 4: "TRIA_ERR_CUDA", 5: "TRIA_ERR_OOM"}
+PAIR_NEOX = 0
+PAIR_INTERLEAVED = 1
+LAYOUT_CONTIGUOUS = 0
+LAYOUT_PAGED = 1
+MAX_LAYERS = 256
+
+EXPORTS = ["tria_status_string", "tria_version", "tria_load_stats", "tria_free_stats",
+           "tria_stats_desc", "tria_workspace_size", "tria_score", "tria_select", "tria_compact",
+           "tria_compress_pass", "tria_read_device_status", "tria_set_pass_events"]
+
+
+class TriaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+class ModelDesc(ctypes.Structure):
+    _fields_ = [("n_layers", ctypes.c_int), ("n_q_heads", ctypes.c_int),
+                ("n_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("pairing", ctypes.c_int), ("rope_theta", ctypes.c_double),
+                ("offset_log2_max", ctypes.c_int)]
+
+
+class CacheView(ctypes.Structure):
+    _fields_ = [("layout", ctypes.c_int), ("n_seq", ctypes.c_int), ("max_seq_len", ctypes.c_int),
+                ("k_layers", ctypes.POINTER(ctypes.c_void_p)),
+                ("v_layers", ctypes.POINTER(ctypes.c_void_p)),
+                ("stride_seq", ctypes.c_int64), ("stride_head", ctypes.c_int64),
+                ("stride_token", ctypes.c_int64), ("stride_block", ctypes.c_int64),
+                ("block_table", ctypes.c_void_p), ("max_blocks_per_seq", ctypes.c_int),
+                ("block_size", ctypes.c_int), ("seq_lens", ctypes.c_void_p),
+                ("query_pos", ctypes.c_void_p), ("positions", ctypes.c_void_p)]
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("budget", ctypes.c_int), ("window", ctypes.c_int), ("sinks", ctypes.c_int)]
+
+
+_lib = None
+_VP = ctypes.c_void_p
+_I = ctypes.c_int
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library (raises if it is not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} missing: build it with key_retention_scoring_b200.build")
+    L = ctypes.CDLL(LIB_PATH)
+    L.tria_status_string.restype = ctypes.c_char_p
+    L.tria_status_string.argtypes = [_I]
+    L.tria_version.restype = ctypes.c_char_p
+    L.tria_version.argtypes = []
+    L.tria_load_stats.argtypes = [ctypes.POINTER(ModelDesc), _VP, _VP, _VP, _VP, _VP,
+                                  ctypes.POINTER(_VP)]
+    L.tria_free_stats.argtypes = [_VP]
+    L.tria_stats_desc.argtypes = [_VP, ctypes.POINTER(ModelDesc)]
+    L.tria_workspace_size.argtypes = [_VP, ctypes.POINTER(CacheView), ctypes.POINTER(Params), _I,
+                                      _I, ctypes.POINTER(ctypes.c_size_t)]
+    L.tria_score.argtypes = [_VP, ctypes.POINTER(CacheView), ctypes.POINTER(Params), _I, _I, _VP,
+                             _VP, _VP, ctypes.c_size_t, _VP]
+    L.tria_select.argtypes = [_VP, ctypes.POINTER(CacheView), ctypes.POINTER(Params), _VP, _I, _I,
+                              _VP, _VP, ctypes.c_size_t, _VP]
+    L.tria_compact.argtypes = [_VP, ctypes.POINTER(CacheView), ctypes.POINTER(Params), _VP, _I, _I,
+                               _VP, _VP, _VP]
+    L.tria_compress_pass.argtypes = [_VP, ctypes.POINTER(CacheView), ctypes.POINTER(Params), _VP,
+                                     _VP, _VP, _VP, ctypes.c_size_t, _VP]
+    L.tria_read_device_status.argtypes = [_VP, _VP, ctypes.POINTER(ctypes.c_int32)]
+    L.tria_set_pass_events.argtypes = [ctypes.POINTER(_VP)]
+    for name in EXPORTS:
+        if name not in ("tria_status_string", "tria_version"):
+            getattr(L, name).restype = _I
+    _lib = L
+    return L
+
+
+def _check(status: int, where: str):
+    if status != TRIA_OK:
+        raise TriaError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def tria_status_string(status: int) -> str:
+    return lib().tria_status_string(status).decode()
+
+
+def tria_version() -> str:
+    return lib().tria_version().decode()
+
+
+class Stats:
+    """Owner of a tria_stats handle."""
+
+    def __init__(self, handle: int, desc: ModelDesc):
+        self.handle = handle
+        self.desc = desc
+
+    def free(self):
+        if self.handle:
+            _check(lib().tria_free_stats(self.handle), "tria_free_stats")
+            self.handle = None
+
+
+def model_desc(n_layers, n_q_heads, n_kv_heads, pairing, rope_theta, offset_log2_max=16,
+               head_dim=128) -> ModelDesc:
+    return ModelDesc(n_layers, n_q_heads, n_kv_heads, head_dim, pairing, float(rope_theta),
+                     offset_log2_max)
+
+
+def tria_load_stats(desc: ModelDesc, q_mean_re, q_mean_im, q_abs_mean, band_mask=None,
+                    stream=None) -> Stats:
+    """Host fp32 arrays [n_layers][n_q_heads][head_dim/2]."""
+    arrs = [np.ascontiguousarray(a, dtype=np.float32) for a in (q_mean_re, q_mean_im, q_abs_mean)]
+    n = desc.n_layers * desc.n_q_heads * (desc.head_dim // 2)
+    for a in arrs:
+        if a.size != n:
+            raise ValueError("statistics must have n_layers * n_q_heads * head_dim/2 entries")
+    mask = None if band_mask is None else np.ascontiguousarray(band_mask, dtype=np.float32)
+    out = _VP()
+    st = lib().tria_load_stats(ctypes.byref(desc), arrs[0].ctypes.data, arrs[1].ctypes.data,
+                               arrs[2].ctypes.data,
+                               None if mask is None else mask.ctypes.data,
+                               _stream(stream), ctypes.byref(out))
+    _check(st, "tria_load_stats")
+    return Stats(out.value, desc)
+
+
+def tria_free_stats(stats: Stats):
+    stats.free()
+
+
+class Cache:
+    """A tria_cache_view over torch tensors (kept alive by this object)."""
+
+    def __init__(self, layout, k_layers, v_layers, seq_lens, query_pos, max_seq_len, *,
+                 stride_seq=0, stride_head=0, stride_token=128, stride_block=0,
+                 block_table=None, max_blocks_per_seq=0, block_size=0, positions=None):
+        self._keep = (k_layers, v_layers, seq_lens, query_pos, block_table, positions)
+        n = len(k_layers)
+        self._k = (_VP * n)(*[_ptr(t) for t in k_layers])
+        self._v = (_VP * n)(*[_ptr(t) for t in v_layers]) if v_layers is not None else None
+        self.view = CacheView(
+            layout, int(seq_lens.numel()), int(max_seq_len),
+            ctypes.cast(self._k, ctypes.POINTER(_VP)),
+            ctypes.cast(self._v, ctypes.POINTER(_VP)) if self._v is not None else None,
+            stride_seq, stride_head, stride_token, stride_block, _ptr(block_table),
+            max_blocks_per_seq, block_size, _ptr(seq_lens), _ptr(query_pos), _ptr(positions))
+
+    @classmethod
+    def from_workload(cls, w) -> "Cache":
+        """View of a ``synth.Workload``."""
+        st = w.strides
+        return cls(w.cfg.layout, w.k, w.v, w.seq_lens, w.query_pos, w.max_seq_len,
+                   stride_seq=st["seq"], stride_head=st["head"], stride_token=st["token"],
+                   stride_block=st["block"], block_table=w.block_table,
+                   max_blocks_per_seq=w.max_blocks, block_size=w.cfg.block_size,
+                   positions=w.positions)
+
+
+def params(budget, window, sinks) -> Params:
+    return Params(budget, window, sinks)
+
+
+def tria_workspace_size(stats: Stats, cache: Cache, prm: Params, layer0=0, layer1=None) -> int:
+    layer1 = stats.desc.n_layers if layer1 is None else layer1
+    out = ctypes.c_size_t()
+    _check(lib().tria_workspace_size(stats.handle, ctypes.byref(cache.view), ctypes.byref(prm),
+                                     layer0, layer1, ctypes.byref(out)), "tria_workspace_size")
+    return out.value
+
+
+def tria_score(stats, cache, prm, layer0, layer1, agg_out, scores_out, workspace, stream=None):
+    _check(lib().tria_score(stats.handle, ctypes.byref(cache.view), ctypes.byref(prm), layer0,
+                            layer1, _ptr(agg_out), _ptr(scores_out), _ptr(workspace),
+                            workspace.numel() * workspace.element_size(), _stream(stream)),
+           "tria_score")
+
+
+def tria_select(stats, cache, prm, agg, layer0, layer1, kept_idx, workspace, stream=None):
+    _check(lib().tria_select(stats.handle, ctypes.byref(cache.view), ctypes.byref(prm), _ptr(agg),
+                             layer0, layer1, _ptr(kept_idx), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream)),
+           "tria_select")
+
+
+def tria_compact(stats, cache, prm, kept_idx, layer0, layer1, freed_blocks=None, n_freed=None,
+                 stream=None):
+    _check(lib().tria_compact(stats.handle, ctypes.byref(cache.view), ctypes.byref(prm),
+                              _ptr(kept_idx), layer0, layer1, _ptr(freed_blocks), _ptr(n_freed),
+                              _stream(stream)), "tria_compact")
+
+
+def tria_compress_pass(stats, cache, prm, kept_idx, workspace, freed_blocks=None, n_freed=None,
+                       stream=None):
+    _check(lib().tria_compress_pass(stats.handle, ctypes.byref(cache.view), ctypes.byref(prm),
+                                    _ptr(kept_idx), _ptr(freed_blocks), _ptr(n_freed),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream(stream)), "tria_compress_pass")
+
+
+def tria_read_device_status(workspace, stream=None) -> int:
+    out = ctypes.c_int32()
+    _check(lib().tria_read_device_status(_ptr(workspace), _stream(stream), ctypes.byref(out)),
+           "tria_read_device_status")
+    return out.value
+
+
+def alloc_workspace(nbytes: int, device="cuda"):
+    """A 256-byte aligned device buffer (torch allocations are)."""
+    import torch
+
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def tria_set_pass_events(events):
+    """events: None or a list of 4 torch.cuda.Event (created with timing)."""
+    if events is None:
+        _check(lib().tria_set_pass_events(None), "tria_set_pass_events")
+        return
+    arr = (_VP * 4)(*[e.cuda_event for e in events])
+    _check(lib().tria_set_pass_events(arr), "tria_set_pass_events")

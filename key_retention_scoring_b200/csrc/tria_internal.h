@@ -1,0 +1,132 @@
+// Internal declarations shared by the host entry points (tria_api.cu) and the
+// kernels (tria_kernels.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/tria.h"
+
+namespace tria {
+
+constexpr int kHeadDim = 128;
+constexpr int kBands = 64;          // d / 2 RoPE bands
+constexpr int kCoefPerHead = 3 * kBands;  // Re c_f, Im c_f, w_f (fp32)
+constexpr int kTileKeys = 1024;     // keys per scheduling item of the score kernel
+constexpr int kMaxSeqTable = TRIA_MAX_SEQS + 1;
+
+// Device copy of the folded statistics.
+struct StatsDev {
+  tria_model_desc desc;
+  double2 *mu_fold;   // [L][Hq][F]  mu'_f = E[q_f] W_f mask_f   (complex, fp64)
+  double *w_norm;     // [L][Hq][F]  E|q_f| - |E q_f|            (fp64)
+  double *omega;      // [F]         theta^(-2f/d)               (fp64)
+};
+
+// Per-call geometry.
+struct Geom {
+  int n_seq;
+  int nl;        // layers in [layer0, layer1)
+  int layer0;
+  int n_layers;  // of the model
+  int hkv, hq, g;
+  int budget, window, sinks;
+  int max_seq_len;
+  int c_max;     // max_seq_len - window - sinks (>= 1)
+  int tiles_max; // ceil(c_max / kTileKeys)
+  int pairing;
+  int64_t n_units;  // n_seq * nl * hkv
+};
+
+// Cache addressing (pointers indexed by layer - layer0).
+struct CacheDev {
+  int layout;
+  int block_size;
+  int max_blocks;
+  int64_t s_seq, s_head, s_tok, s_blk;
+  const int32_t *block_table;
+  int32_t *seq_lens;
+  const int64_t *query_pos;
+  int32_t *positions;
+  int64_t pos_unit_stride;  // max_seq_len
+  const uint16_t *k[TRIA_MAX_LAYERS];
+  uint16_t *v[TRIA_MAX_LAYERS];
+};
+
+// Workspace carve-up (byte offsets from the workspace base).
+struct WsLayout {
+  size_t hdr;         // 256 B: u32 item counter, i32 status flags
+  size_t unit_done;   // n_units x u32
+  size_t seq_items;   // (n_seq + 1) x i32 prefix of scheduling items per sequence
+  size_t coef;        // n_seq x nl x hq x kCoefPerHead fp32
+  size_t moments;     // n_units x tiles_max x g x 2 fp64
+  size_t raw;         // n_units x raw_stride fp32
+  size_t agg;         // n_units x agg_stride fp32
+  size_t kept;        // n_units x budget i32
+  size_t total;
+  int64_t raw_stride; // floats per unit, multiple of 32
+  int64_t agg_stride; // floats per unit, multiple of 32
+};
+
+WsLayout ws_layout(const Geom &g);
+
+// Score-kernel parameters.
+struct ScoreParams {
+  Geom geo;
+  CacheDev cache;
+  const float *coef;
+  uint32_t *item_counter;
+  int32_t *status;
+  uint32_t *unit_done;
+  const int32_t *seq_items;
+  double *moments;
+  float *raw;           // [unit][raw_stride], per candidate G floats
+  int64_t raw_stride;
+  float *agg;           // [unit][agg_stride]
+  int64_t agg_stride;
+  int32_t *kept;        // [unit][budget] or null (score only)
+  int discard_raw;      // raw is workspace scratch: drop its L2 lines after use
+  int discard_agg;      // agg is workspace scratch
+};
+
+struct CoefParams {
+  Geom geo;
+  const double2 *mu_fold;
+  const double *w_norm;
+  const double *omega;
+  const int64_t *query_pos;
+  const int32_t *seq_lens;
+  float *coef;
+  uint32_t *item_counter;
+  uint32_t *unit_done;
+  int32_t *seq_items;
+  int32_t *status;
+  int32_t *kept;      // identity rows for units with N <= budget (may be null)
+};
+
+struct SelectParams {
+  Geom geo;
+  const int32_t *seq_lens;
+  int32_t *status;
+  const float *agg;
+  int64_t agg_stride;
+  int32_t *kept;
+};
+
+struct CompactParams {
+  Geom geo;
+  CacheDev cache;
+  const int32_t *kept;
+  int update_lens;      // layer1 == n_layers
+  int32_t *freed_blocks;
+  int32_t *n_freed;
+};
+
+// Launchers (tria_kernels.cu).  Return cudaGetLastError() of the launch.
+cudaError_t launch_coef(const CoefParams &p, cudaStream_t st);
+cudaError_t launch_score(const ScoreParams &p, cudaStream_t st);
+cudaError_t launch_select(const SelectParams &p, cudaStream_t st);
+cudaError_t launch_compact(const CompactParams &p, cudaStream_t st);
+
+}  // namespace tria
