@@ -258,5 +258,8 @@ def tria_set_pass_events(events):
     if events is None:
         _check(lib().tria_set_pass_events(None), "tria_set_pass_events")
         return
+    for e in events:
+        if not e.cuda_event:   # torch creates the CUDA event on its first record
+            e.record()
     arr = (_VP * 4)(*[e.cuda_event for e in events])
     _check(lib().tria_set_pass_events(arr), "tria_set_pass_events")

@@ -17,6 +17,8 @@
 // ghidav.me "TriAttention, or: what a rotating query already knows" ("The
 // Method"), GitHub issue #10 of the llama.cpp TurboQuant HIP fork (RoPE
 // pairing, window/sink conventions).
+#include <cstddef>
+
 #include <cuda_runtime.h>
 
 #include "tria_internal.h"
@@ -357,15 +359,16 @@ __device__ __forceinline__ float halfwarp_reduce(float (&a)[G], int hl) {
 }
 
 struct ScoreSmem {
-  int seq_items[kMaxSeqTable];
-  float coef[TRIA_MAX_GROUP * kCoefPerHead];
-  double mom[16][TRIA_MAX_GROUP][2];
+  alignas(16) float coef[TRIA_MAX_GROUP * kCoefPerHead];  // read as float4
+  alignas(16) double mom[16][TRIA_MAX_GROUP][2];
+  alignas(16) int seq_items[kMaxSeqTable];
   float mean[TRIA_MAX_GROUP];
   float inv[TRIA_MAX_GROUP];
   int item;
   int last;
   SelectSmem sel;
 };
+static_assert(offsetof(ScoreSmem, coef) % 16 == 0, "coef is read as float4");
 
 template <int G>
 __device__ void unit_tail(const ScoreParams &p, ScoreSmem &sm, int64_t u, int C, int ntiles,
