@@ -36,7 +36,10 @@
  *   - The library allocates device memory only in tria_load_stats (the stats
  *     object); scoring, selection and compaction never allocate.
  *   - bf16 K/V rows are 128 elements (256 bytes); row starts must be 16-byte
- *     aligned (strides multiples of 8 elements, 16-byte aligned bases).
+ *     aligned (strides multiples of 8 elements, 16-byte aligned bases).  The
+ *     scoring kernel reads K through TMA tensor maps that the library encodes
+ *     (and caches) per layer base pointer; a stride pattern the tensor-map
+ *     encoder rejects returns TRIA_ERR_UNSUPPORTED.
  *   - A unit whose length N is at most the budget is left unchanged.
  *   - Floating point decides the kept set only through the fp32 aggregated
  *     score agg (below); exactly equal agg go to the lower slot; -0.0 equals
@@ -76,7 +79,7 @@ typedef enum {
 } tria_layout;
 
 #define TRIA_HEAD_DIM 128
-#define TRIA_MAX_LAYERS 256
+#define TRIA_MAX_LAYERS 128
 #define TRIA_MAX_GROUP 16
 #define TRIA_MAX_SEQS 1024
 
@@ -101,7 +104,9 @@ typedef struct {
   int layout;                /* tria_layout                                          */
   int n_seq;                 /* 1 .. TRIA_MAX_SEQS                                   */
   int max_seq_len;           /* host: upper bound of every seq_lens[s]; sizes the
-                                candidate axis C_max = max_seq_len - window - sinks  */
+                                candidate axis C_max = max_seq_len - window - sinks.
+                                Contiguous layout: every (sequence, KV head) has room
+                                for max_seq_len rows.                                */
   void *const *k_layers;     /* host array [n_layers] of device pointers, bf16 K     */
   void *const *v_layers;     /* host array [n_layers] of device pointers, bf16 V;
                                 needed by compaction only                            */
@@ -112,7 +117,9 @@ typedef struct {
   int64_t stride_block;      /* elements between blocks (paged)                      */
   const int32_t *block_table;/* device [n_seq][max_blocks_per_seq] (paged)           */
   int max_blocks_per_seq;    /* paged                                                */
-  int block_size;            /* rows per block (paged), 1 .. 1024                    */
+  int block_size;            /* rows per block (paged): 8, 16, 32, 64 or 128         */
+  int64_t num_blocks;        /* paged: blocks in each layer's K (and V) pool; block
+                                ids outside [0, num_blocks) read as zero rows        */
   int32_t *seq_lens;         /* device [n_seq] cached tokens N per sequence; set to
                                 min(N, budget) by tria_compact when it covers the last
                                 layer                                                */
@@ -255,11 +262,12 @@ tria_status tria_read_device_status(void *workspace, tria_stream_t stream,
 
 /*
  * tria_set_pass_events - kernel timing hook for tria_compress_pass (tracing).
- * events: NULL to disable, or a host array of 4 cudaEvent_t created by the
+ * events: NULL to disable, or a host array of 5 cudaEvent_t created by the
  * caller; the next tria_compress_pass calls made from this host thread record
  * events[0] before the coefficient kernel, events[1] before the scoring
- * kernel, events[2] before the compaction kernel and events[3] after it, on
- * the pass's stream.  The array is copied; the events stay owned by the caller.
+ * kernel, events[2] before the normalize-then-max / selection kernel,
+ * events[3] before the compaction kernel and events[4] after it, on the
+ * pass's stream.  The array is copied; the events stay owned by the caller.
  */
 tria_status tria_set_pass_events(void *const *events);
 

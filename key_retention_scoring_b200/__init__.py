@@ -23,7 +23,7 @@ PAIR_NEOX = 0
 PAIR_INTERLEAVED = 1
 LAYOUT_CONTIGUOUS = 0
 LAYOUT_PAGED = 1
-MAX_LAYERS = 256
+MAX_LAYERS = 128
 
 EXPORTS = ["tria_status_string", "tria_version", "tria_load_stats", "tria_free_stats",
            "tria_stats_desc", "tria_workspace_size", "tria_score", "tria_select", "tria_compact",
@@ -50,7 +50,8 @@ class CacheView(ctypes.Structure):
                 ("stride_seq", ctypes.c_int64), ("stride_head", ctypes.c_int64),
                 ("stride_token", ctypes.c_int64), ("stride_block", ctypes.c_int64),
                 ("block_table", ctypes.c_void_p), ("max_blocks_per_seq", ctypes.c_int),
-                ("block_size", ctypes.c_int), ("seq_lens", ctypes.c_void_p),
+                ("block_size", ctypes.c_int), ("num_blocks", ctypes.c_int64),
+                ("seq_lens", ctypes.c_void_p),
                 ("query_pos", ctypes.c_void_p), ("positions", ctypes.c_void_p)]
 
 
@@ -175,7 +176,8 @@ class Cache:
 
     def __init__(self, layout, k_layers, v_layers, seq_lens, query_pos, max_seq_len, *,
                  stride_seq=0, stride_head=0, stride_token=128, stride_block=0,
-                 block_table=None, max_blocks_per_seq=0, block_size=0, positions=None):
+                 block_table=None, max_blocks_per_seq=0, block_size=0, num_blocks=0,
+                 positions=None):
         self._keep = (k_layers, v_layers, seq_lens, query_pos, block_table, positions)
         n = len(k_layers)
         self._k = (_VP * n)(*[_ptr(t) for t in k_layers])
@@ -185,7 +187,8 @@ class Cache:
             ctypes.cast(self._k, ctypes.POINTER(_VP)),
             ctypes.cast(self._v, ctypes.POINTER(_VP)) if self._v is not None else None,
             stride_seq, stride_head, stride_token, stride_block, _ptr(block_table),
-            max_blocks_per_seq, block_size, _ptr(seq_lens), _ptr(query_pos), _ptr(positions))
+            max_blocks_per_seq, block_size, num_blocks, _ptr(seq_lens), _ptr(query_pos),
+            _ptr(positions))
 
     @classmethod
     def from_workload(cls, w) -> "Cache":
@@ -195,7 +198,7 @@ class Cache:
                    stride_seq=st["seq"], stride_head=st["head"], stride_token=st["token"],
                    stride_block=st["block"], block_table=w.block_table,
                    max_blocks_per_seq=w.max_blocks, block_size=w.cfg.block_size,
-                   positions=w.positions)
+                   num_blocks=getattr(w, "n_blocks", 0), positions=w.positions)
 
 
 def params(budget, window, sinks) -> Params:
@@ -254,12 +257,12 @@ def alloc_workspace(nbytes: int, device="cuda"):
 
 
 def tria_set_pass_events(events):
-    """events: None or a list of 4 torch.cuda.Event (created with timing)."""
+    """events: None or a list of 5 torch.cuda.Event (created with timing)."""
     if events is None:
         _check(lib().tria_set_pass_events(None), "tria_set_pass_events")
         return
     for e in events:
         if not e.cuda_event:   # torch creates the CUDA event on its first record
             e.record()
-    arr = (_VP * 4)(*[e.cuda_event for e in events])
+    arr = (_VP * 5)(*[e.cuda_event for e in events])
     _check(lib().tria_set_pass_events(arr), "tria_set_pass_events")

@@ -10,8 +10,13 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <map>
+#include <mutex>
 #include <new>
 #include <vector>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
 
 #include <cuda_runtime.h>
 
@@ -58,8 +63,9 @@ tria_status make_geom(const tria_stats *stats, const tria_cache_view *cache,
       (cache->stride_block % 8))
     return TRIA_ERR_INVALID_ARG;
   if (cache->layout == TRIA_LAYOUT_PAGED) {
-    if (cache->block_table == nullptr || cache->block_size < 1 || cache->block_size > 1024 ||
-        cache->max_blocks_per_seq < 1)
+    const int bs = cache->block_size;
+    if (cache->block_table == nullptr || cache->max_blocks_per_seq < 1 || cache->num_blocks < 1 ||
+        !(bs == 8 || bs == 16 || bs == 32 || bs == 64 || bs == 128))
       return TRIA_ERR_INVALID_ARG;
     if ((int64_t)cache->max_blocks_per_seq * cache->block_size < cache->max_seq_len)
       return TRIA_ERR_INVALID_ARG;
@@ -80,11 +86,93 @@ tria_status make_geom(const tria_stats *stats, const tria_cache_view *cache,
   g.max_seq_len = cache->max_seq_len;
   const int cm = cache->max_seq_len - params->window - params->sinks;
   g.c_max = cm > 1 ? cm : 1;
-  g.tiles_max = (g.c_max + kTileKeys - 1) / kTileKeys;
+  // scheduling tiles are aligned to kTileKeys slots and cover [sinks, N - window)
+  const int hi = cache->max_seq_len - params->window - 1;
+  g.tiles_max = hi >= params->sinks ? hi / kTileKeys - params->sinks / kTileKeys + 1 : 1;
   g.pairing = d.pairing;
+  g.ncol = (2 * g.g < 16) ? 16 : 2 * g.g;
   g.n_units = (int64_t)g.n_seq * g.nl * g.hkv;
   if (g.n_units * (int64_t)g.tiles_max > INT32_MAX) return TRIA_ERR_UNSUPPORTED;
   *geo = g;
+  return TRIA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// TMA tensor maps of the K cache (encoded on the host, cached by pointer and
+// geometry; entries are 128 bytes).
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+struct MapKey {
+  const void *ptr;
+  int layout;
+  uint64_t dims[4];
+  uint64_t strides[3];
+  uint32_t box[4];
+  bool operator<(const MapKey &o) const { return std::memcmp(this, &o, sizeof(MapKey)) < 0; }
+};
+
+tria_status k_tensor_map(const tria_cache_view *c, int hkv, const void *base, CUtensorMap *out) {
+  MapKey key;
+  std::memset(&key, 0, sizeof(key));
+  key.ptr = base;
+  key.layout = c->layout;
+  if (c->layout == TRIA_LAYOUT_CONTIGUOUS) {
+    // [n_seq][hkv][max_seq_len][128] by strides; box = 128 rows x 64 dims
+    key.dims[0] = 128;
+    key.dims[1] = (uint64_t)c->max_seq_len;
+    key.dims[2] = (uint64_t)hkv;
+    key.dims[3] = (uint64_t)c->n_seq;
+    key.strides[0] = (uint64_t)c->stride_token * 2;
+    key.strides[1] = (uint64_t)c->stride_head * 2;
+    key.strides[2] = (uint64_t)c->stride_seq * 2;
+    key.box[0] = 64; key.box[1] = 128; key.box[2] = 1; key.box[3] = 1;
+  } else {
+    // [num_blocks][block_size][hkv][128] by strides; box = one block of one head x 64 dims
+    key.dims[0] = 128;
+    key.dims[1] = (uint64_t)hkv;
+    key.dims[2] = (uint64_t)c->block_size;
+    key.dims[3] = (uint64_t)c->num_blocks;
+    key.strides[0] = (uint64_t)c->stride_head * 2;
+    key.strides[1] = (uint64_t)c->stride_token * 2;
+    key.strides[2] = (uint64_t)c->stride_block * 2;
+    key.box[0] = 64; key.box[1] = 1; key.box[2] = (uint32_t)c->block_size; key.box[3] = 1;
+  }
+  // a dimension of extent 1 never advances: give it a stride the encoder accepts
+  for (int i = 0; i < 3; ++i)
+    if (key.dims[i + 1] == 1 && key.strides[i] == 0)
+      key.strides[i] = (i == 0 ? 256 : key.strides[i - 1] * key.dims[i]);
+  static std::mutex mu;
+  static std::map<MapKey, CUtensorMap> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) {
+    *out = it->second;
+    return TRIA_OK;
+  }
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (enc == nullptr) return TRIA_ERR_CUDA;
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUtensorMap m;
+  const CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base),
+                         key.dims, key.strides, key.box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return TRIA_ERR_UNSUPPORTED;
+  if (cache.size() > 4096) cache.clear();
+  cache.emplace(key, m);
+  *out = m;
   return TRIA_OK;
 }
 
@@ -122,7 +210,7 @@ T *at(void *ws, size_t off) {
 }
 
 CoefParams make_coef(const tria_stats *st, const Geom &g, const tria_cache_view *c, void *ws,
-                     const WsLayout &wl, int32_t *kept) {
+                     const WsLayout &wl, int32_t *kept, bool with_hist) {
   CoefParams cp{};
   cp.geo = g;
   cp.mu_fold = st->dev.mu_fold;
@@ -130,34 +218,51 @@ CoefParams make_coef(const tria_stats *st, const Geom &g, const tria_cache_view 
   cp.omega = st->dev.omega;
   cp.query_pos = c->query_pos;
   cp.seq_lens = c->seq_lens;
-  cp.coef = at<float>(ws, wl.coef);
+  cp.btile = at<uint16_t>(ws, wl.btile);
   cp.item_counter = at<uint32_t>(ws, wl.hdr);
   cp.status = at<int32_t>(ws, wl.hdr + 4);
   cp.unit_done = at<uint32_t>(ws, wl.unit_done);
   cp.seq_items = at<int32_t>(ws, wl.seq_items);
   cp.kept = kept;
+  cp.hist = with_hist ? at<uint32_t>(ws, wl.hist) : nullptr;
   return cp;
 }
 
-ScoreParams make_score(const Geom &g, const tria_cache_view *c, int layer0, int layer1, void *ws,
-                       const WsLayout &wl) {
-  ScoreParams sp{};
+tria_status make_score(const Geom &g, const tria_cache_view *c, int layer0, int layer1, void *ws,
+                       const WsLayout &wl, ScoreParams &sp) {
+  std::memset(&sp, 0, sizeof(sp));
+  for (int l = layer0; l < layer1; ++l) {
+    const tria_status st = k_tensor_map(c, g.hkv, c->k_layers[l], &sp.kmap[l - layer0]);
+    if (st != TRIA_OK) return st;
+  }
   sp.geo = g;
   sp.cache = make_cache_dev(c, layer0, layer1);
-  sp.coef = at<float>(ws, wl.coef);
+  sp.btile = at<uint16_t>(ws, wl.btile);
   sp.item_counter = at<uint32_t>(ws, wl.hdr);
   sp.status = at<int32_t>(ws, wl.hdr + 4);
-  sp.unit_done = at<uint32_t>(ws, wl.unit_done);
   sp.seq_items = at<int32_t>(ws, wl.seq_items);
   sp.moments = at<double>(ws, wl.moments);
   sp.raw = at<float>(ws, wl.raw);
   sp.raw_stride = wl.raw_stride;
-  sp.agg = at<float>(ws, wl.agg);
-  sp.agg_stride = wl.agg_stride;
-  sp.kept = nullptr;
-  sp.discard_raw = 1;
-  sp.discard_agg = 1;
-  return sp;
+  return TRIA_OK;
+}
+
+TailParams make_tail(const Geom &g, const tria_cache_view *c, void *ws, const WsLayout &wl) {
+  TailParams tp{};
+  tp.geo = g;
+  tp.seq_lens = c->seq_lens;
+  tp.status = at<int32_t>(ws, wl.hdr + 4);
+  tp.moments = at<double>(ws, wl.moments);
+  tp.raw = at<float>(ws, wl.raw);
+  tp.raw_stride = wl.raw_stride;
+  tp.agg = at<float>(ws, wl.agg);
+  tp.agg_stride = wl.agg_stride;
+  tp.kept = nullptr;
+  tp.hist = at<uint32_t>(ws, wl.hist);
+  tp.unit_done = at<uint32_t>(ws, wl.unit_done);
+  tp.discard_raw = 1;
+  tp.discard_agg = 1;
+  return tp;
 }
 
 }  // namespace
@@ -175,8 +280,9 @@ WsLayout ws_layout(const Geom &g) {
   w.hdr = take(256);
   w.unit_done = take((size_t)g.n_units * 4);
   w.seq_items = take((size_t)(g.n_seq + 1) * 4);
-  w.coef = take((size_t)g.n_seq * g.nl * g.hq * kCoefPerHead * 4);
+  w.btile = take((size_t)g.n_units * g.ncol * kCoefK * 2);
   w.moments = take((size_t)g.n_units * g.tiles_max * g.g * 2 * 8);
+  w.hist = take((size_t)g.n_units * kAggHistBins * 4);
   w.raw = take((size_t)g.n_units * w.raw_stride * 4);
   w.agg = take((size_t)g.n_units * w.agg_stride * 4);
   w.kept = take((size_t)g.n_units * g.budget * 4);
@@ -322,18 +428,23 @@ tria_status tria_score(const tria_stats *stats, const tria_cache_view *cache,
   WsLayout wl;
   if ((st = check_workspace(g, ws, ws_bytes, &wl)) != TRIA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_coef(make_coef(stats, g, cache, ws, wl, nullptr), s);
-  if (e != cudaSuccess) return TRIA_ERR_CUDA;
-  ScoreParams sp = make_score(g, cache, layer0, layer1, ws, wl);
+  static thread_local ScoreParams sp;
+  if ((st = make_score(g, cache, layer0, layer1, ws, wl, sp)) != TRIA_OK) return st;
+  TailParams tp = make_tail(g, cache, ws, wl);
   if (scores_out != nullptr) {
     sp.raw = scores_out;
     sp.raw_stride = (int64_t)g.c_max * g.g;
-    sp.discard_raw = 0;
+    tp.raw = scores_out;
+    tp.raw_stride = sp.raw_stride;
+    tp.discard_raw = 0;
   }
-  sp.agg = agg_out;
-  sp.agg_stride = g.c_max;
-  sp.discard_agg = 0;
-  return cuda_status(launch_score(sp, s));
+  tp.agg = agg_out;
+  tp.agg_stride = g.c_max;
+  tp.discard_agg = 0;
+  if (launch_coef(make_coef(stats, g, cache, ws, wl, nullptr, false), s) != cudaSuccess)
+    return TRIA_ERR_CUDA;
+  if (launch_score(sp, s) != cudaSuccess) return TRIA_ERR_CUDA;
+  return cuda_status(launch_tail(tp, s));
 }
 
 tria_status tria_select(const tria_stats *stats, const tria_cache_view *cache,
@@ -375,10 +486,10 @@ tria_status tria_compact(const tria_stats *stats, const tria_cache_view *cache,
   return cuda_status(launch_compact(p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-static thread_local cudaEvent_t g_pass_events[4] = {nullptr, nullptr, nullptr, nullptr};
+static thread_local cudaEvent_t g_pass_events[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
 
 tria_status tria_set_pass_events(void *const *events) {
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 5; ++i)
     g_pass_events[i] = events ? static_cast<cudaEvent_t>(events[i]) : nullptr;
   return TRIA_OK;
 }
@@ -403,13 +514,18 @@ tria_status tria_compress_pass(const tria_stats *stats, const tria_cache_view *c
   if ((st = check_workspace(g, ws, ws_bytes, &wl)) != TRIA_OK) return st;
   int32_t *kept = kept_idx != nullptr ? kept_idx : at<int32_t>(ws, wl.kept);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  static thread_local ScoreParams sp;
+  if ((st = make_score(g, cache, 0, L, ws, wl, sp)) != TRIA_OK) return st;
+  TailParams tp = make_tail(g, cache, ws, wl);
+  tp.kept = kept;
   if (mark(0, s) != cudaSuccess) return TRIA_ERR_CUDA;
-  if (launch_coef(make_coef(stats, g, cache, ws, wl, kept), s) != cudaSuccess) return TRIA_ERR_CUDA;
+  if (launch_coef(make_coef(stats, g, cache, ws, wl, kept, true), s) != cudaSuccess)
+    return TRIA_ERR_CUDA;
   if (mark(1, s) != cudaSuccess) return TRIA_ERR_CUDA;
-  ScoreParams sp = make_score(g, cache, 0, L, ws, wl);
-  sp.kept = kept;
   if (launch_score(sp, s) != cudaSuccess) return TRIA_ERR_CUDA;
   if (mark(2, s) != cudaSuccess) return TRIA_ERR_CUDA;
+  if (launch_tail(tp, s) != cudaSuccess) return TRIA_ERR_CUDA;
+  if (mark(3, s) != cudaSuccess) return TRIA_ERR_CUDA;
   CompactParams cp{};
   cp.geo = g;
   cp.cache = make_cache_dev(cache, 0, L);
@@ -418,7 +534,7 @@ tria_status tria_compress_pass(const tria_stats *stats, const tria_cache_view *c
   cp.freed_blocks = freed_blocks;
   cp.n_freed = n_freed;
   if (launch_compact(cp, s) != cudaSuccess) return TRIA_ERR_CUDA;
-  return cuda_status(mark(3, s));
+  return cuda_status(mark(4, s));
 }
 
 tria_status tria_read_device_status(void *ws, tria_stream_t stream, int32_t *flags_out) {

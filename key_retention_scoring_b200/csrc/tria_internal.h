@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/tria.h"
@@ -12,7 +13,7 @@ namespace tria {
 
 constexpr int kHeadDim = 128;
 constexpr int kBands = 64;          // d / 2 RoPE bands
-constexpr int kCoefPerHead = 3 * kBands;  // Re c_f, Im c_f, w_f (fp32)
+constexpr int kCoefK = 256;         // K extent of the coefficient tile: 128 key dims + 2 x 64 bands
 constexpr int kTileKeys = 1024;     // keys per scheduling item of the score kernel
 constexpr int kMaxSeqTable = TRIA_MAX_SEQS + 1;
 
@@ -26,6 +27,7 @@ struct StatsDev {
 
 // Per-call geometry.
 struct Geom {
+  int ncol;      // coefficient tile rows: max(16, 2G)
   int n_seq;
   int nl;        // layers in [layer0, layer1)
   int layer0;
@@ -34,7 +36,7 @@ struct Geom {
   int budget, window, sinks;
   int max_seq_len;
   int c_max;     // max_seq_len - window - sinks (>= 1)
-  int tiles_max; // ceil(c_max / kTileKeys)
+  int tiles_max; // upper bound of the scheduling tiles of one unit
   int pairing;
   int64_t n_units;  // n_seq * nl * hkv
 };
@@ -57,10 +59,11 @@ struct CacheDev {
 // Workspace carve-up (byte offsets from the workspace base).
 struct WsLayout {
   size_t hdr;         // 256 B: u32 item counter, i32 status flags
-  size_t unit_done;   // n_units x u32
+  size_t unit_done;   // n_units x u32: finished normalization chunks per unit
   size_t seq_items;   // (n_seq + 1) x i32 prefix of scheduling items per sequence
-  size_t coef;        // n_seq x nl x hq x kCoefPerHead fp32
+  size_t btile;       // n_units x ncol x kCoefK bf16 coefficient tiles
   size_t moments;     // n_units x tiles_max x g x 2 fp64
+  size_t hist;        // n_units x kAggHistBins u32: histogram of the top 12 bits of agg keys
   size_t raw;         // n_units x raw_stride fp32
   size_t agg;         // n_units x agg_stride fp32
   size_t kept;        // n_units x budget i32
@@ -69,23 +72,38 @@ struct WsLayout {
   int64_t agg_stride; // floats per unit, multiple of 32
 };
 
+constexpr int kAggHistBins = 4096;
+constexpr int kAggChunk = 4096;   // candidates per block of the normalization kernel
+
 WsLayout ws_layout(const Geom &g);
 
 // Score-kernel parameters.
 struct ScoreParams {
+  CUtensorMap kmap[TRIA_MAX_LAYERS];  // K of each layer in [layer0, layer1): 128B-swizzled boxes
   Geom geo;
   CacheDev cache;
-  const float *coef;
+  const uint16_t *btile;  // [unit][ncol][kCoefK] bf16, shared-memory image
   uint32_t *item_counter;
   int32_t *status;
-  uint32_t *unit_done;
   const int32_t *seq_items;
   double *moments;
   float *raw;           // [unit][raw_stride], per candidate G floats
   int64_t raw_stride;
-  float *agg;           // [unit][agg_stride]
+};
+
+// Normalize-then-max (and selection) kernel parameters.
+struct TailParams {
+  Geom geo;
+  const int32_t *seq_lens;
+  int32_t *status;
+  const double *moments;
+  float *raw;
+  int64_t raw_stride;
+  float *agg;
   int64_t agg_stride;
-  int32_t *kept;        // [unit][budget] or null (score only)
+  int32_t *kept;        // null: agg only
+  uint32_t *hist;       // [unit][kAggHistBins]
+  uint32_t *unit_done;  // [unit]
   int discard_raw;      // raw is workspace scratch: drop its L2 lines after use
   int discard_agg;      // agg is workspace scratch
 };
@@ -97,12 +115,13 @@ struct CoefParams {
   const double *omega;
   const int64_t *query_pos;
   const int32_t *seq_lens;
-  float *coef;
+  uint16_t *btile;
   uint32_t *item_counter;
   uint32_t *unit_done;
   int32_t *seq_items;
   int32_t *status;
   int32_t *kept;      // identity rows for units with N <= budget (may be null)
+  uint32_t *hist;     // zeroed per unit (may be null)
 };
 
 struct SelectParams {
@@ -126,6 +145,7 @@ struct CompactParams {
 // Launchers (tria_kernels.cu).  Return cudaGetLastError() of the launch.
 cudaError_t launch_coef(const CoefParams &p, cudaStream_t st);
 cudaError_t launch_score(const ScoreParams &p, cudaStream_t st);
+cudaError_t launch_tail(const TailParams &p, cudaStream_t st);
 cudaError_t launch_select(const SelectParams &p, cudaStream_t st);
 cudaError_t launch_compact(const CompactParams &p, cudaStream_t st);
 

@@ -1,0 +1,663 @@
+// Scoring kernel of the compression pass on the sm_100a tensor cores.
+//
+// Per unit (sequence, layer, KV head) the averaged score of G query heads is
+//   S~_g(k) = sum_f Re(c_gf conj(ktilde_f)) + w_gf |ktilde_f|
+// with ktilde the post-RoPE key, c_gf = mu'_gf e^{i omega_f p_q} the folded
+// center turned to the query position (academ.us article 2607.13051, Eqs. 3,
+// 6, 7: the key position cancels because conj(k_f) e^{i omega_f (p_q - p_k)}
+// = conj(ktilde_f) e^{i omega_f p_q}) and w_gf = E|q_f| - |E q_f| the norm-term
+// weight.  Over a tile of 128 keys both sums are one dense contraction
+//   D[128 x 2G] = [ktilde | m_hi | m_lo] (128 x 256) . Bcoef (256 x 2G)
+// where m = |ktilde_f| is split into bf16 hi + lo parts and every fp32
+// coefficient x into bf16 hi + lo columns (D[:,2g] + D[:,2g+1] = S~_g up to a
+// relative 2^-16 of the terms).  The keys are bf16 already, so the product is
+// exact and accumulates in fp32 in tensor memory.
+//
+// Roles (one CTA per SM, persistent, dynamic items of kTileKeys slots):
+//   warp 16     producer: TMA tensor loads of 128-slot K tiles (two 64-dim
+//               boxes, or one box per paged block) into a ring of 128-byte-
+//               swizzled K-major tiles, plus the unit's coefficient image
+//               (one bulk copy per item); completion as mbarrier tx bytes;
+//   warp 17     one lane issues tcgen05.mma (M=128, N=16|32, K=16): 8 steps
+//               with A = the K tile in shared memory (then the K stage is
+//               released), 8 steps with A = the magnitude tile in tensor
+//               memory, and tcgen05.commit;
+//   warps 0-15  band magnitudes -> tensor memory (tcgen05.st; warp w takes
+//               rows 32(w%4).. and bands 16(w/4)..), epilogue (tcgen05.ld,
+//               raw scores, fp64 moment partials per item).
+// Normalize-then-max and the selection run in the next kernel (tail_kernel).
+// Every wait is bounded (2 s); on expiry the kernel flags status bit 1, lets
+// its own loads and MMAs land, frees its tensor memory and returns.
+#include <cuda_bf16.h>
+
+#include "tria_device.cuh"
+
+namespace tria {
+namespace {
+
+using namespace dev;
+
+constexpr int kRows = 128;                  // keys per MMA tile (M)
+constexpr int kComputeWarps = 16;
+constexpr int kComputeThreads = 512;
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kTcThreads = 576;
+constexpr int kBarCompute = 1;
+constexpr int kHalfBlock = kRows * 128;     // 128 rows x 64 bf16, swizzled
+constexpr int kFlagFirst = 1, kFlagLast = 2, kFlagEnd = 4;
+constexpr uint32_t kTmemCols = 256;         // [0, 2*NCOL): accumulators; [64, 192): magnitude tiles
+constexpr uint32_t kTmemMag = 64;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+struct SubRec {
+  long long u;
+  int s, lrel, h, tile, N;
+  int slot0, flags, bpar;  // first slot of the 128-row tile (a multiple of 128)
+};
+
+template <int G>
+struct TcCfg {
+  static constexpr int NCOL = (2 * G < 16) ? 16 : 2 * G;   // MMA N
+  static constexpr int STAGES = (G <= 8) ? 6 : 5;
+  static constexpr int GQ = (G >= 4) ? G / 4 : 1;          // heads per band quarter
+  static constexpr int BBLK = NCOL * 128;                  // bytes per 64-wide K block of B
+};
+
+template <int G>
+struct TcSmem {
+  alignas(1024) uint8_t k[TcCfg<G>::STAGES][2][kHalfBlock];
+  alignas(1024) uint8_t b[2][4][TcCfg<G>::BBLK];
+  alignas(8) uint64_t full[TcCfg<G>::STAGES];
+  alignas(8) uint64_t kempty[TcCfg<G>::STAGES];
+  alignas(8) uint64_t aready[2];
+  alignas(8) uint64_t accfull[2];
+  alignas(8) uint64_t bempty[2];
+  SubRec rec[TcCfg<G>::STAGES];
+  alignas(16) double mom[kComputeWarps][TcCfg<G>::GQ][2];
+  alignas(16) int seq_items[kMaxSeqTable];
+  int seq_len[kMaxSeqTable];
+  uint32_t tmem_base;
+  volatile int abort_flag;
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *b, int count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait for the phase of `parity`; false on expiry or abort.
+__device__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                          int32_t *status) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try(a, parity)) return true;
+  const uint64_t t0 = global_timer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(a, parity)) return true;
+    if ((it & 255u) == 0u) {
+      if (*abort_flag) return false;
+      if (global_timer() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        atomicOr(status, 2);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)),
+               "r"(bytes)
+               : "memory");
+}
+
+// TMA tile load of a 4-D box into shared memory, completion as transaction
+// bytes on `bar`.  x (the innermost coordinate) is 0 or 64 elements.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            int z, int w, uint64_t *bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::"
+      "cache_hint [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar)),
+      "l"(pol)
+      : "memory");
+}
+
+// Contiguous bulk copy global -> shared (16-byte aligned, multiple of 16 bytes).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst, int ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, int ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// Shared-memory matrix descriptor: 128-byte swizzle, K-major, 8-row groups
+// 1024 bytes apart (the tile base is 1024-byte aligned).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(16u >> 4) << 16;    // leading-dimension byte offset (unused when swizzled)
+  d |= (uint64_t)(1024u >> 4) << 32;  // stride byte offset
+  d |= (uint64_t)1 << 46;             // descriptor version of sm_100
+  d |= (uint64_t)2 << 61;             // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor of kind::f16: bf16 x bf16 -> f32, both K-major.
+template <int NCOL>
+__host__ __device__ constexpr uint32_t idesc_bf16_m128() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(NCOL >> 3) << 17) |
+         ((uint32_t)(kRows >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+// Store 8 consecutive 32-bit columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// D (tmem) (+)= A (tmem, 128 lanes x 16 bf16 in 8 columns) . B (smem descriptor)
+__device__ __forceinline__ void mma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[N]) {
+  uint32_t r[N];
+  if constexpr (N == 2) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];"
+                 : "=r"(r[0]), "=r"(r[1])
+                 : "r"(taddr));
+  } else if constexpr (N == 4) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+  } else if constexpr (N == 8) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+  } else {
+    static_assert(N == 16, "tmem_ld width");
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+  }
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < N; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ uint4 lds128(const uint8_t *p) { return *reinterpret_cast<const uint4 *>(p); }
+
+// bf16 hi/lo split of two floats, packed low-address-first: hi = x with its
+// low 16 bits cleared (exact in bf16), lo = bf16(x - hi) rounded to nearest;
+// |x - hi - lo| < 2^-16 |x|.
+__device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t &lo) {
+  const uint32_t ua = __float_as_uint(a) & 0xffff0000u, ub = __float_as_uint(b) & 0xffff0000u;
+  hi = (ua >> 16) | ub;
+  const __nv_bfloat162 l = __floats2bfloat162_rn(a - __uint_as_float(ua), b - __uint_as_float(ub));
+  lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+
+// ---------------------------------------------------------------------------
+// producer warp
+// ---------------------------------------------------------------------------
+template <int G, int LAYOUT>
+__device__ void producer(const ScoreParams &p, TcSmem<G> &sm, int n_items, int lane) {
+  constexpr int ST = TcCfg<G>::STAGES, NCOL = TcCfg<G>::NCOL;
+  constexpr uint32_t kBBytes = NCOL * kCoefK * 2;
+  const Geom &geo = p.geo;
+  const uint64_t pol = evict_first_policy();
+  const int units_per_seq = geo.nl * geo.hkv;
+  const int W = geo.window, S = geo.sinks;
+  int i = 0, items = 0, sub = 0, sub_first = 0, sub_end = 0;
+  int s = 0, lrel = 0, h = 0, tile = 0, ntiles = 1, N = 0, tbase = 0;
+  long long u = 0;
+  bool ok = true;
+  // the next item index is claimed one item ahead
+  uint32_t nxt = 0;
+  if (lane == 0) nxt = atomicAdd(p.item_counter, 1u);
+  for (;;) {
+    if (sub == sub_end) {
+      const int it = (int)__shfl_sync(kFull, nxt, 0);
+      if (it >= n_items) break;
+      if (lane == 0) nxt = atomicAdd(p.item_counter, 1u);
+      int lo = 0, hi = geo.n_seq - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (sm.seq_items[mid] <= it) lo = mid; else hi = mid - 1;
+      }
+      s = lo;
+      ntiles = (sm.seq_items[s + 1] - sm.seq_items[s]) / units_per_seq;
+      const int rem = it - sm.seq_items[s];
+      const int ul = rem / ntiles;
+      tile = rem % ntiles;
+      lrel = ul / geo.hkv;
+      h = ul % geo.hkv;
+      u = (long long)s * units_per_seq + ul;
+      N = sm.seq_len[s];
+      tbase = (S / kTileKeys + tile) * kTileKeys;
+      const int c_lo = max(S, tbase), c_hi = min(N - W, tbase + kTileKeys);
+      sub_first = (c_lo - tbase) / kRows;
+      sub = sub_first;
+      sub_end = (c_hi - tbase + kRows - 1) / kRows;
+      ++items;
+    }
+    const int stage = i % ST;
+    if (i >= ST) {
+      if (lane == 0) ok = mbar_wait(&sm.kempty[stage], ((i / ST) - 1) & 1, &sm.abort_flag, p.status);
+      ok = __shfl_sync(kFull, ok, 0);
+      if (!ok) break;
+    }
+    const int bpar = (items - 1) & 1;
+    const bool first = (sub == sub_first);
+    if (first && items > 2) {
+      // the coefficient buffer is free once the MMAs of the item two back are done
+      if (lane == 0) ok = mbar_wait(&sm.bempty[bpar], ((items - 3) >> 1) & 1, &sm.abort_flag, p.status);
+      ok = __shfl_sync(kFull, ok, 0);
+      if (!ok) break;
+    }
+    const int slot0 = tbase + sub * kRows;
+    const uint32_t kdst = smem_u32(&sm.k[stage][0][0]);
+    uint32_t bytes = first ? kBBytes : 0u;
+    int blk = 0;
+    bool bvalid = false;
+    if (LAYOUT == TRIA_LAYOUT_CONTIGUOUS) {
+      bytes += 2u * kHalfBlock;
+    } else {
+      // one box per block of this tile that holds a candidate row
+      const int bs = p.cache.block_size;
+      const int slot_b = slot0 + lane * bs;
+      const int bidx = slot_b / bs;
+      bvalid = lane < kRows / bs && slot_b < N - W && slot_b + bs > S && bidx < p.cache.max_blocks;
+      if (bvalid) blk = p.cache.block_table[(int64_t)s * p.cache.max_blocks + bidx];
+      bytes += (uint32_t)__popc(__ballot_sync(kFull, bvalid)) * (uint32_t)bs * 256u;
+    }
+    if (lane == 0) {
+      SubRec &r = sm.rec[stage];
+      r.u = u; r.s = s; r.lrel = lrel; r.h = h; r.tile = tile; r.N = N; r.slot0 = slot0;
+      r.flags = (first ? kFlagFirst : 0) | (sub == sub_end - 1 ? kFlagLast : 0);
+      r.bpar = bpar;
+      mbar_arrive_expect_tx(&sm.full[stage], bytes);
+      if (first)
+        bulk_load(smem_u32(&sm.b[bpar][0][0]), p.btile + u * NCOL * kCoefK, kBBytes, &sm.full[stage]);
+    }
+    const CUtensorMap *map = &p.kmap[lrel];
+    if (LAYOUT == TRIA_LAYOUT_CONTIGUOUS) {
+      if (lane < 2)
+        tma_load_4d(kdst + lane * kHalfBlock, map, lane * 64, slot0, h, s, &sm.full[stage], pol);
+    } else if (bvalid) {
+      const uint32_t off = (uint32_t)(lane * p.cache.block_size * 128);
+      tma_load_4d(kdst + off, map, 0, h, 0, blk, &sm.full[stage], pol);
+      tma_load_4d(kdst + kHalfBlock + off, map, 64, h, 0, blk, &sm.full[stage], pol);
+    }
+    ++sub;
+    ++i;
+  }
+  if (ok) {
+    // end marker for the compute warps and the MMA issuer
+    const int stage = i % ST;
+    if (i >= ST) {
+      if (lane == 0) ok = mbar_wait(&sm.kempty[stage], ((i / ST) - 1) & 1, &sm.abort_flag, p.status);
+      ok = __shfl_sync(kFull, ok, 0);
+    }
+    if (ok && lane == 0) {
+      sm.rec[stage].flags = kFlagEnd;
+      mbar_arrive(&sm.full[stage]);
+    }
+  }
+  if (!ok && lane == 0) {
+    // aborted: let the loads already issued land before the block exits
+    for (int j = (i > ST ? i - ST : 0); j < i; ++j)
+      mbar_wait(&sm.full[j % ST], (j / ST) & 1, &sm.abort_flag, p.status) ||
+          mbar_try(smem_u32(&sm.full[j % ST]), (j / ST) & 1);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// MMA issuer (one lane)
+// ---------------------------------------------------------------------------
+template <int G>
+__device__ void mma_issuer(const ScoreParams &p, TcSmem<G> &sm, uint32_t tmem) {
+  constexpr int ST = TcCfg<G>::STAGES, NCOL = TcCfg<G>::NCOL, BBLK = TcCfg<G>::BBLK;
+  constexpr uint32_t idesc = idesc_bf16_m128<NCOL>();
+  int i = 0;
+  for (;; ++i) {
+    if (!mbar_wait(&sm.aready[i & 1], (i >> 1) & 1, &sm.abort_flag, p.status)) break;
+    tc_fence_after();
+    const int stage = i % ST, ab = i & 1;
+    const SubRec &rec = sm.rec[stage];
+    if (rec.flags & kFlagEnd) break;
+    const uint32_t d = tmem + (uint32_t)(ab * NCOL);
+    const uint32_t ka = smem_u32(&sm.k[stage][0][0]);
+    const uint32_t ta = tmem + kTmemMag + (uint32_t)(ab * 64);
+    const uint32_t bb = smem_u32(&sm.b[rec.bpar][0][0]);
+    const bool last = (rec.flags & kFlagLast) != 0;
+    const int bpar = rec.bpar;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const uint32_t a_addr = ka + (s >> 2) * kHalfBlock + (s & 3) * 32;
+      const uint32_t b_addr = bb + (s >> 2) * BBLK + (s & 3) * 32;
+      mma_bf16(d, sw128_desc(a_addr), sw128_desc(b_addr), idesc, s > 0 ? 1u : 0u);
+    }
+    mma_commit(&sm.kempty[stage]);  // the K tile is consumed: the producer may refill it
+#pragma unroll
+    for (int s = 8; s < 16; ++s) {
+      const uint32_t b_addr = bb + (s >> 2) * BBLK + (s & 3) * 32;
+      mma_bf16_ta(d, ta + (uint32_t)((s - 8) * 8), sw128_desc(b_addr), idesc, 1u);
+    }
+    if (last) mma_commit(&sm.bempty[bpar]);
+    mma_commit(&sm.accfull[ab]);  // issued last: the final wait below covers all
+  }
+  if (i > 0) mbar_wait(&sm.accfull[(i - 1) & 1], ((i - 1) >> 1) & 1, &sm.abort_flag, p.status);
+}
+
+// ---------------------------------------------------------------------------
+// compute warps
+// ---------------------------------------------------------------------------
+// Band magnitudes of row r, bands [16q, 16q + 16), split into bf16 hi and
+// lo parts and stored to the row's tensor-memory lane: hi at columns
+// [8q, 8q + 8), lo at [32 + 8q, ...) of the magnitude tile (two bf16 per
+// column, band order).
+template <int PAIR>
+__device__ __forceinline__ void mags(const uint8_t *kt, uint32_t tcol, int r, int q) {
+  const int sw = r & 7;
+  uint32_t hi[8], lo[8];
+  if (PAIR == TRIA_PAIR_NEOX) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int cc = 2 * q + j;
+      const uint4 re = lds128(kt + r * 128 + ((cc ^ sw) << 4));
+      const uint4 im = lds128(kt + kHalfBlock + r * 128 + ((cc ^ sw) << 4));
+      const uint32_t rw[4] = {re.x, re.y, re.z, re.w}, iw[4] = {im.x, im.y, im.z, im.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float ra = bf_lo(rw[e]), rb = bf_hi(rw[e]);
+        const float ia = bf_lo(iw[e]), ib = bf_hi(iw[e]);
+        const float ma = sqrt_approx(fmaf(ra, ra, ia * ia));
+        const float mb = sqrt_approx(fmaf(rb, rb, ib * ib));
+        split2(ma, mb, hi[4 * j + e], lo[4 * j + e]);
+      }
+    }
+  } else {
+    const uint8_t *kh = kt + (q >> 1) * kHalfBlock;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int cc = 4 * (q & 1) + j;
+      const uint4 x = lds128(kh + r * 128 + ((cc ^ sw) << 4));
+      const float m0 = sqrt_approx(fmaf(bf_lo(x.x), bf_lo(x.x), bf_hi(x.x) * bf_hi(x.x)));
+      const float m1 = sqrt_approx(fmaf(bf_lo(x.y), bf_lo(x.y), bf_hi(x.y) * bf_hi(x.y)));
+      const float m2 = sqrt_approx(fmaf(bf_lo(x.z), bf_lo(x.z), bf_hi(x.z) * bf_hi(x.z)));
+      const float m3 = sqrt_approx(fmaf(bf_lo(x.w), bf_lo(x.w), bf_hi(x.w) * bf_hi(x.w)));
+      split2(m0, m1, hi[2 * j], lo[2 * j]);
+      split2(m2, m3, hi[2 * j + 1], lo[2 * j + 1]);
+    }
+  }
+  tmem_st8(tcol + (uint32_t)(8 * q), hi);
+  tmem_st8(tcol + (uint32_t)(32 + 8 * q), lo);
+}
+
+template <int G, int PAIR>
+__device__ void compute(const ScoreParams &p, TcSmem<G> &sm, uint32_t tmem, int tid) {
+  constexpr int ST = TcCfg<G>::STAGES, NCOL = TcCfg<G>::NCOL, GQ = TcCfg<G>::GQ;
+  const Geom &geo = p.geo;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int q = warp >> 2, r = (warp & 3) * 32 + lane;
+  const bool active = (G >= 4) || q < G;  // quarter q scores heads [q GQ, (q + 1) GQ)
+  const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+  double msum[GQ], msq[GQ];
+#pragma unroll
+  for (int g = 0; g < GQ; ++g) msum[g] = msq[g] = 0.0;
+  SubRec prev{};
+  bool have_prev = false;
+  for (int i = 0;; ++i) {
+    const int stage = i % ST;
+    mbar_wait(&sm.full[stage], (i / ST) & 1, &sm.abort_flag, p.status);
+    csync<kBarCompute, kComputeThreads>();
+    if (sm.abort_flag) break;
+    const SubRec rec = sm.rec[stage];
+    const bool end = (rec.flags & kFlagEnd) != 0;
+    if (!end) {
+      mags<PAIR>(&sm.k[stage][0][0], tmem + lane_base + kTmemMag + (uint32_t)((i & 1) * 64), r, q);
+      tmem_wait_st();
+      tc_fence_before();
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.aready[i & 1]);
+    if (have_prev) {
+      const int j = i - 1;
+      mbar_wait(&sm.accfull[j & 1], (j >> 1) & 1, &sm.abort_flag, p.status);
+      csync<kBarCompute, kComputeThreads>();
+      if (sm.abort_flag) break;
+      tc_fence_after();
+      if (prev.flags & kFlagFirst) {
+#pragma unroll
+        for (int g = 0; g < GQ; ++g) msum[g] = msq[g] = 0.0;
+      }
+      if (active) {
+        float v[2 * GQ];
+        tmem_ld<2 * GQ>(tmem + lane_base + (uint32_t)((j & 1) * NCOL + q * 2 * GQ), v);
+        const int slot = prev.slot0 + r;
+        if (slot >= geo.sinks && slot < prev.N - geo.window) {
+          float sc[GQ];
+#pragma unroll
+          for (int g = 0; g < GQ; ++g) {
+            sc[g] = v[2 * g] + v[2 * g + 1];
+            msum[g] += (double)sc[g];
+            msq[g] = fma((double)sc[g], (double)sc[g], msq[g]);
+          }
+          float *dst = p.raw + prev.u * p.raw_stride + (int64_t)(slot - geo.sinks) * G + q * GQ;
+          if constexpr (GQ == 4) {
+            *reinterpret_cast<float4 *>(dst) = make_float4(sc[0], sc[1], sc[2], sc[3]);
+          } else if constexpr (GQ == 2) {
+            *reinterpret_cast<float2 *>(dst) = make_float2(sc[0], sc[1]);
+          } else {
+            dst[0] = sc[0];
+          }
+        }
+      }
+      tc_fence_before();
+      if (prev.flags & kFlagLast) {
+        // item done: its moment partials, summed over rows in a fixed order
+#pragma unroll
+        for (int g = 0; g < GQ; ++g) {
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) {
+            msum[g] += __shfl_xor_sync(kFull, msum[g], o);
+            msq[g] += __shfl_xor_sync(kFull, msq[g], o);
+          }
+          if (lane == 0) {
+            sm.mom[warp][g][0] = msum[g];
+            sm.mom[warp][g][1] = msq[g];
+          }
+        }
+        csync<kBarCompute, kComputeThreads>();
+        if (tid < G) {
+          const int qq = tid / GQ, gl = tid % GQ;
+          double s1 = 0.0, s2 = 0.0;
+          for (int w = 4 * qq; w < 4 * qq + 4; ++w) {
+            s1 += sm.mom[w][gl][0];
+            s2 += sm.mom[w][gl][1];
+          }
+          double *m = p.moments + ((prev.u * geo.tiles_max + prev.tile) * G + tid) * 2;
+          m[0] = s1;
+          m[1] = s2;
+        }
+      }
+    }
+    if (end) break;
+    prev = rec;
+    have_prev = true;
+  }
+}
+
+template <int G, int PAIR, int LAYOUT>
+__global__ void __launch_bounds__(kTcThreads, 1) score_tc_kernel(const __grid_constant__ ScoreParams p) {
+  using Cfg = TcCfg<G>;
+  extern __shared__ uint8_t smem_dyn[];
+  TcSmem<G> &sm = *reinterpret_cast<TcSmem<G> *>(
+      (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
+  const Geom &geo = p.geo;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  for (int i = tid; i <= geo.n_seq; i += kTcThreads) sm.seq_items[i] = p.seq_items[i];
+  for (int i = tid; i < geo.n_seq; i += kTcThreads) sm.seq_len[i] = p.cache.seq_lens[i];
+  if (tid == 0) {
+    for (int i = 0; i < Cfg::STAGES; ++i) {
+      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.kempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.aready[i], kComputeWarps);
+      mbar_init(&sm.accfull[i], 1);
+      mbar_init(&sm.bempty[i], 1);
+    }
+    sm.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == kMmaWarp) tmem_alloc(&sm.tmem_base, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const int n_items = sm.seq_items[geo.n_seq];
+
+  if (warp < kComputeWarps) {
+    compute<G, PAIR>(p, sm, tmem, tid);
+  } else if (warp == kProducerWarp) {
+    producer<G, LAYOUT>(p, sm, n_items, lane);
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) mma_issuer<G>(p, sm, tmem);
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int G, int PAIR, int LAYOUT>
+cudaError_t launch_t(const ScoreParams &p, cudaStream_t st) {
+  auto kern = score_tc_kernel<G, PAIR, LAYOUT>;
+  const int smem = (int)sizeof(TcSmem<G>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  kern<<<sms, kTcThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int G>
+cudaError_t launch_g(const ScoreParams &p, cudaStream_t st) {
+  const bool paged = p.cache.layout == TRIA_LAYOUT_PAGED;
+  if (p.geo.pairing == TRIA_PAIR_NEOX)
+    return paged ? launch_t<G, TRIA_PAIR_NEOX, TRIA_LAYOUT_PAGED>(p, st)
+                 : launch_t<G, TRIA_PAIR_NEOX, TRIA_LAYOUT_CONTIGUOUS>(p, st);
+  return paged ? launch_t<G, TRIA_PAIR_INTERLEAVED, TRIA_LAYOUT_PAGED>(p, st)
+               : launch_t<G, TRIA_PAIR_INTERLEAVED, TRIA_LAYOUT_CONTIGUOUS>(p, st);
+}
+
+static_assert(sizeof(TcSmem<8>) + 1024 <= 232448, "shared memory of the G=8 kernel");
+static_assert(sizeof(TcSmem<16>) + 1024 <= 232448, "shared memory of the G=16 kernel");
+
+}  // namespace
+
+cudaError_t launch_score(const ScoreParams &p, cudaStream_t st) {
+  switch (p.geo.g) {
+    case 1: return launch_g<1>(p, st);
+    case 2: return launch_g<2>(p, st);
+    case 4: return launch_g<4>(p, st);
+    case 8: return launch_g<8>(p, st);
+    case 16: return launch_g<16>(p, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace tria
