@@ -191,6 +191,21 @@ def run_reference(args, rank, world):
     return 0
 
 
+def rank_config(base, rank: int):
+    """Weak scaling: every rank compresses its own sequence of the workload
+    (same shape, its own seed); no data crosses ranks."""
+    return base.scaled(seed=base.seed + 1000 * rank)
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The slowest rank's time (all ranks call it in the same order)."""
+    import torch
+
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def config_desc(cfg, extra=None):
     d = {"workload": cfg.name, "layers": cfg.n_layers, "q_heads": cfg.n_q_heads,
          "kv_heads": cfg.n_kv_heads, "head_dim": cfg.head_dim, "seq_len": cfg.seq_len,
@@ -218,6 +233,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, run16 and CPU baseline")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="override the workload's layer count (small profiling cases)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -243,7 +260,9 @@ def main():
     synth.build()
 
     base = synth.CONFIGS[args.config]
-    cfg = base.scaled(seed=base.seed + 1000 * rank)   # each rank: its own sequence (weak scaling)
+    if args.layers:
+        base = base.scaled(n_layers=args.layers)
+    cfg = rank_config(base, rank)
     w = synth.Workload(cfg)
     re, im, am = w.stats
     st = T.tria_load_stats(T.model_desc(cfg.n_layers, cfg.n_q_heads, cfg.n_kv_heads, cfg.pairing,
@@ -314,9 +333,7 @@ def main():
     compact_ms = [e[3].elapsed_time(e[4]) for e in all_evs]
     ms = statistics.mean(pass_ms)
     if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dist, "cuda")
 
     N = cfg.seq_len
     units = cfg.n_seq * cfg.n_layers * cfg.n_kv_heads

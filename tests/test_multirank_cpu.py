@@ -1,0 +1,75 @@
+"""Multi-rank host logic of bench.py on CPU with gloo (world size 2): each
+rank gets its own sequence (weak scaling, no data exchange) and the reported
+time is the max over ranks."""
+import os
+import socket
+
+import pytest
+
+torch = pytest.importorskip("torch")
+import torch.distributed as dist  # noqa: E402
+import torch.multiprocessing as mp  # noqa: E402
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, out):
+    import sys
+
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    import synth
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    from datetime import timedelta
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        cfg = bench.rank_config(synth.CONFIGS[2], rank)
+        # every rank draws a different sequence of the same shape
+        stats = synth.make_stats(cfg)
+        digest = float(stats[0][0, 0, 0])
+        t = bench.max_over_ranks(1.0 + rank * 2.5, dist, "cpu")
+        gathered = [None] * world
+        dist.all_gather_object(gathered, (cfg.seed, cfg.n_layers, digest))
+        out.put((rank, t, gathered))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_two_ranks_weak_scaling_and_max_time():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=180) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, t, gathered in res:
+        assert t == pytest.approx(3.5)  # max of 1.0 and 3.5
+        seeds = [g[0] for g in gathered]
+        assert len(set(seeds)) == 2                      # distinct sequences
+        assert gathered[0][1] == gathered[1][1] == 64    # same shape
+        assert gathered[0][2] != gathered[1][2]          # different draws
+
+
+def test_reference_arm_rank_gating(capsys, monkeypatch):
+    import bench
+
+    class A:
+        steps, warmup, config = 1, 0, 0
+
+    # a non-zero rank prints nothing and exits 0 without work
+    assert bench.run_reference(A(), 1, 2) == 0
+    assert capsys.readouterr().out == ""
