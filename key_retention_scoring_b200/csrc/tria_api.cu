@@ -281,7 +281,7 @@ WsLayout ws_layout(const Geom &g) {
   w.unit_done = take((size_t)g.n_units * 4);
   w.seq_items = take((size_t)(g.n_seq + 1) * 4);
   w.btile = take((size_t)g.n_units * g.ncol * kCoefK * 2);
-  w.moments = take((size_t)g.n_units * g.tiles_max * g.g * 2 * 8);
+  w.moments = take((size_t)g.n_units * g.tiles_max * kRowGroups * g.g * 2 * 8);
   w.hist = take((size_t)g.n_units * kAggHistBins * 4);
   w.raw = take((size_t)g.n_units * w.raw_stride * 4);
   w.agg = take((size_t)g.n_units * w.agg_stride * 4);

@@ -134,6 +134,7 @@ struct SelScalars {
   int list_n;
   float mean[TRIA_MAX_GROUP];
   float inv[TRIA_MAX_GROUP];
+  double red[8][TRIA_MAX_GROUP][2];
 };
 
 // Histogram increment with lanes of equal bins merged first.
@@ -363,30 +364,57 @@ __device__ void select_unit(const float *agg, int C, int K, int N, int B, int W,
 // ---------------------------------------------------------------------------
 // Normalize-then-max of a range of candidates of one unit.
 // unit_norm: population mean and 1/(std + eps) of every head over the C
-// candidates, from the per-item moment partials (fp64, summed in item order).
+// candidates, from the moment partials of each (item, 32-row group) (fp64,
+// summed in item order, then row-group order).
 // agg_range: agg[c] = max_g (S_g[c] - mean_g) * inv_g for c in [c0, c1), with
 // the histogram of the top 12 key bits added into hist when it is non-null.
 // ---------------------------------------------------------------------------
-template <int G>
-__device__ void unit_norm(const double *mom_unit, int ntiles, int C, int tid, float *s_mean,
-                          float *s_inv) {
-  if (tid < G) {
-    double s1 = 0.0, s2 = 0.0;
-    for (int i = 0; i < ntiles; ++i) {
-      s1 += __ldcg(mom_unit + (int64_t)i * G * 2 + tid * 2);
-      s2 += __ldcg(mom_unit + (int64_t)i * G * 2 + tid * 2 + 1);
+template <int G, int BAR, int NT>
+__device__ void unit_norm(const double *mom_unit, int ntiles, int C, int tid, SelScalars &sc) {
+  // every thread sums a fixed subset of the partials, then a fixed-order
+  // butterfly over the warp and a sequential sum over the warps
+  double s1[G], s2[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) s1[g] = s2[g] = 0.0;
+  const int n = ntiles * kRowGroups;
+  for (int i = tid; i < n; i += NT) {
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      s1[g] += __ldcg(mom_unit + ((int64_t)i * G + g) * 2);
+      s2[g] += __ldcg(mom_unit + ((int64_t)i * G + g) * 2 + 1);
     }
-    const double mean = s1 / C;
-    double var = s2 / C - mean * mean;
+  }
+  const int lane = tid & 31, w = tid >> 5;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      s1[g] += __shfl_xor_sync(kFull, s1[g], o);
+      s2[g] += __shfl_xor_sync(kFull, s2[g], o);
+    }
+    if (lane == 0) {
+      sc.red[w][g][0] = s1[g];
+      sc.red[w][g][1] = s2[g];
+    }
+  }
+  csync<BAR, NT>();
+  if (tid < G) {
+    double a = 0.0, b = 0.0;
+    for (int i = 0; i < NT / 32; ++i) {
+      a += sc.red[i][tid][0];
+      b += sc.red[i][tid][1];
+    }
+    const double mean = a / C;
+    double var = b / C - mean * mean;
     var = var > 0.0 ? var : 0.0;
-    s_mean[tid] = (float)mean;
-    s_inv[tid] = (float)(1.0 / (sqrt(var) + 1e-6));
+    sc.mean[tid] = (float)mean;
+    sc.inv[tid] = (float)(1.0 / (sqrt(var) + 1e-6));
   }
 }
 
 template <int G, int NT>
-__device__ void agg_range(const float *raw, float *agg, int c0, int c1, const float *s_mean,
-                          const float *s_inv, uint32_t *hist, int tid) {
+__device__ void agg_range(const float *__restrict__ raw, float *agg, int c0, int c1,
+                          const float *s_mean, const float *s_inv, uint32_t *hist, int tid) {
   const int lane = tid & 31;
   float mean[G], inv[G];
 #pragma unroll
@@ -405,8 +433,9 @@ __device__ void agg_range(const float *raw, float *agg, int c0, int c1, const fl
     }
     return nan ? __int_as_float(0x7fc00000) : a;
   };
-  // E consecutive candidates per thread per step: E*G/4 float4 loads in flight
-  constexpr int E = (G >= 16) ? 2 : 8;
+  // E consecutive candidates per thread per step: E*G/4 float4 loads in
+  // flight (through L1: the two halves of a 32-byte sector hit it once)
+  constexpr int E = (G >= 8) ? 16 / G * 2 : 8;
   int c = c0;
   if (aligned16p(raw + (int64_t)c0 * G)) {
     for (; c + NT * E <= c1; c += NT * E) {
@@ -415,7 +444,7 @@ __device__ void agg_range(const float *raw, float *agg, int c0, int c1, const fl
       const float4 *src = reinterpret_cast<const float4 *>(raw + (int64_t)cc * G);
 #pragma unroll
       for (int i = 0; i < (E * G) / 4; ++i) {
-        const float4 x = __ldcg(src + i);
+        const float4 x = __ldg(src + i);
         v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
       }
 #pragma unroll
@@ -429,7 +458,7 @@ __device__ void agg_range(const float *raw, float *agg, int c0, int c1, const fl
   for (int cc = c + tid; cc < c1; cc += NT) {
     float v[G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) v[g] = __ldcg(raw + (int64_t)cc * G + g);
+    for (int g = 0; g < G; ++g) v[g] = __ldg(raw + (int64_t)cc * G + g);
     const float a = agg_of(v);
     agg[cc] = a;
     if (hist != nullptr) atomicAdd(hist + (order_key(a) >> 20), 1u);

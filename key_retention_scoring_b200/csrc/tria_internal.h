@@ -15,6 +15,7 @@ constexpr int kHeadDim = 128;
 constexpr int kBands = 64;          // d / 2 RoPE bands
 constexpr int kCoefK = 256;         // K extent of the coefficient tile: 128 key dims + 2 x 64 bands
 constexpr int kTileKeys = 1024;     // keys per scheduling item of the score kernel
+constexpr int kRowGroups = 4;       // moment partials per item: one per 32-row group of a tile
 constexpr int kMaxSeqTable = TRIA_MAX_SEQS + 1;
 
 // Device copy of the folded statistics.
@@ -62,7 +63,7 @@ struct WsLayout {
   size_t unit_done;   // n_units x u32: finished normalization chunks per unit
   size_t seq_items;   // (n_seq + 1) x i32 prefix of scheduling items per sequence
   size_t btile;       // n_units x ncol x kCoefK bf16 coefficient tiles
-  size_t moments;     // n_units x tiles_max x g x 2 fp64
+  size_t moments;     // n_units x tiles_max x kRowGroups x g x 2 fp64
   size_t hist;        // n_units x kAggHistBins u32: histogram of the top 12 bits of agg keys
   size_t raw;         // n_units x raw_stride fp32
   size_t agg;         // n_units x agg_stride fp32

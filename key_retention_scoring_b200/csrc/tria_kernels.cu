@@ -165,8 +165,8 @@ __global__ void __launch_bounds__(kThreads) tail_kernel(const __grid_constant__ 
   const int nch = (C + kAggChunk - 1) / kAggChunk;
   if (chunk >= nch) return;
   const int t = threadIdx.x;
-  unit_norm<G>(p.moments + u * geo.tiles_max * G * 2, unit_tiles(N, geo.window, geo.sinks), C, t,
-               sc.mean, sc.inv);
+  unit_norm<G, 0, kThreads>(p.moments + u * geo.tiles_max * kRowGroups * G * 2,
+                            unit_tiles(N, geo.window, geo.sinks), C, t, sc);
   const bool sel = p.kept != nullptr;
   if (sel) clear_words<kThreads>(ts.hist, kAggHistBins, t);
   __syncthreads();

@@ -23,8 +23,10 @@
 //               released), 8 steps with A = the magnitude tile in tensor
 //               memory, and tcgen05.commit;
 //   warps 0-15  band magnitudes -> tensor memory (tcgen05.st; warp w takes
-//               rows 32(w%4).. and bands 16(w/4)..), epilogue (tcgen05.ld,
-//               raw scores, fp64 moment partials per item).
+//               rows 32(w%4).. and bands 16(w/4)..), then, kLag tiles later,
+//               the epilogue (tcgen05.ld, raw scores, fp64 moment partials).
+//               Magnitude tiles and accumulators rotate through kNB
+//               tensor-memory buffers, so kLag MMA chains stay in flight.
 // Normalize-then-max and the selection run in the next kernel (tail_kernel).
 // Every wait is bounded (2 s); on expiry the kernel flags status bit 1, lets
 // its own loads and MMAs land, frees its tensor memory and returns.
@@ -39,15 +41,19 @@ using namespace dev;
 
 constexpr int kRows = 128;                  // keys per MMA tile (M)
 constexpr int kComputeWarps = 16;
-constexpr int kComputeThreads = 512;
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
 constexpr int kTcThreads = 576;
-constexpr int kBarCompute = 1;
 constexpr int kHalfBlock = kRows * 128;     // 128 rows x 64 bf16, swizzled
 constexpr int kFlagFirst = 1, kFlagLast = 2, kFlagEnd = 4;
-constexpr uint32_t kTmemCols = 256;         // [0, 2*NCOL): accumulators; [64, 192): magnitude tiles
-constexpr uint32_t kTmemMag = 64;
+// The epilogue of tile i runs after the magnitudes of tile i + 2, so two MMA
+// chains are in flight while the compute warps work; magnitude tiles and
+// accumulators rotate through kNB tensor-memory buffers (tile i uses i % kNB,
+// whose previous user, tile i - kNB, finished its epilogue before the
+// magnitudes of tile i - 1).
+constexpr int kNB = 4;
+constexpr uint32_t kTmemCols = 512;         // [0, kNB*NCOL): accumulators; [128, 384): magnitude tiles
+constexpr uint32_t kTmemMag = 128;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 struct SubRec {
@@ -70,11 +76,10 @@ struct TcSmem {
   alignas(1024) uint8_t b[2][4][TcCfg<G>::BBLK];
   alignas(8) uint64_t full[TcCfg<G>::STAGES];
   alignas(8) uint64_t kempty[TcCfg<G>::STAGES];
-  alignas(8) uint64_t aready[2];
-  alignas(8) uint64_t accfull[2];
+  alignas(8) uint64_t aready[kNB];
+  alignas(8) uint64_t accfull[kNB];
   alignas(8) uint64_t bempty[2];
   SubRec rec[TcCfg<G>::STAGES];
-  alignas(16) double mom[kComputeWarps][TcCfg<G>::GQ][2];
   alignas(16) int seq_items[kMaxSeqTable];
   int seq_len[kMaxSeqTable];
   uint32_t tmem_base;
@@ -271,16 +276,49 @@ __device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[N]) {
 
 __device__ __forceinline__ uint4 lds128(const uint8_t *p) { return *reinterpret_cast<const uint4 *>(p); }
 
-// bf16 hi/lo split of two floats, packed low-address-first: hi = x with its
-// low 16 bits cleared (exact in bf16), lo = bf16(x - hi) rounded to nearest;
-// |x - hi - lo| < 2^-16 |x|.
-__device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t &lo) {
-  const uint32_t ua = __float_as_uint(a) & 0xffff0000u, ub = __float_as_uint(b) & 0xffff0000u;
-  hi = (ua >> 16) | ub;
-  const __nv_bfloat162 l = __floats2bfloat162_rn(a - __uint_as_float(ua), b - __uint_as_float(ub));
-  lo = *reinterpret_cast<const uint32_t *>(&l);
+// Packed fp32 pairs (sm_100 f32x2 arithmetic).
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void up2(uint64_t v, float &a, float &b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
 }
 
+// Magnitudes of two bands from their bf16 re/im parts, split into bf16
+// hi + lo parts: hi = the top halves of the fp32 bit patterns (truncation),
+// lo = bf16(x - hi) rounded to nearest.  |x - hi - lo| <= 2^-16 x.
+__device__ __forceinline__ void mag_pair(float ra, float rb, float ia, float ib, uint32_t &hi,
+                                         uint32_t &lo) {
+  const uint64_t sq = fma2(pk2(ia, ib), pk2(ia, ib), mul2(pk2(ra, rb), pk2(ra, rb)));
+  float sa, sb;
+  up2(sq, sa, sb);
+  const float ma = sqrt_approx(sa), mb = sqrt_approx(sb);
+  const uint32_t ua = __float_as_uint(ma), ub = __float_as_uint(mb);
+  hi = __byte_perm(ua, ub, 0x7632);
+  const uint64_t res = sub2(pk2(ma, mb), pk2(__uint_as_float(ua & 0xffff0000u),
+                                             __uint_as_float(ub & 0xffff0000u)));
+  float xa, xb;
+  up2(res, xa, xb);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(xa, xb);
+  lo = *reinterpret_cast<const uint32_t *>(&l);
+}
 
 // ---------------------------------------------------------------------------
 // producer warp
@@ -377,8 +415,8 @@ __device__ void producer(const ScoreParams &p, TcSmem<G> &sm, int n_items, int l
     ++sub;
     ++i;
   }
+  // end marker, read by the compute warps and the MMA issuer
   if (ok) {
-    // end marker for the compute warps and the MMA issuer
     const int stage = i % ST;
     if (i >= ST) {
       if (lane == 0) ok = mbar_wait(&sm.kempty[stage], ((i / ST) - 1) & 1, &sm.abort_flag, p.status);
@@ -388,6 +426,7 @@ __device__ void producer(const ScoreParams &p, TcSmem<G> &sm, int n_items, int l
       sm.rec[stage].flags = kFlagEnd;
       mbar_arrive(&sm.full[stage]);
     }
+    ++i;
   }
   if (!ok && lane == 0) {
     // aborted: let the loads already issued land before the block exits
@@ -406,9 +445,9 @@ __device__ void mma_issuer(const ScoreParams &p, TcSmem<G> &sm, uint32_t tmem) {
   constexpr uint32_t idesc = idesc_bf16_m128<NCOL>();
   int i = 0;
   for (;; ++i) {
-    if (!mbar_wait(&sm.aready[i & 1], (i >> 1) & 1, &sm.abort_flag, p.status)) break;
+    if (!mbar_wait(&sm.aready[i % kNB], (i / kNB) & 1, &sm.abort_flag, p.status)) break;
     tc_fence_after();
-    const int stage = i % ST, ab = i & 1;
+    const int stage = i % ST, ab = i % kNB;
     const SubRec &rec = sm.rec[stage];
     if (rec.flags & kFlagEnd) break;
     const uint32_t d = tmem + (uint32_t)(ab * NCOL);
@@ -432,16 +471,15 @@ __device__ void mma_issuer(const ScoreParams &p, TcSmem<G> &sm, uint32_t tmem) {
     if (last) mma_commit(&sm.bempty[bpar]);
     mma_commit(&sm.accfull[ab]);  // issued last: the final wait below covers all
   }
-  if (i > 0) mbar_wait(&sm.accfull[(i - 1) & 1], ((i - 1) >> 1) & 1, &sm.abort_flag, p.status);
+  if (i > 0) mbar_wait(&sm.accfull[(i - 1) % kNB], ((i - 1) / kNB) & 1, &sm.abort_flag, p.status);
 }
 
 // ---------------------------------------------------------------------------
 // compute warps
 // ---------------------------------------------------------------------------
-// Band magnitudes of row r, bands [16q, 16q + 16), split into bf16 hi and
-// lo parts and stored to the row's tensor-memory lane: hi at columns
-// [8q, 8q + 8), lo at [32 + 8q, ...) of the magnitude tile (two bf16 per
-// column, band order).
+// Band magnitudes of row r, bands [16q, 16q + 16), stored to the row's
+// tensor-memory lane: hi parts at columns [8q, 8q + 8), lo parts at
+// [32 + 8q, ...) of the magnitude tile (two bf16 per column, band order).
 template <int PAIR>
 __device__ __forceinline__ void mags(const uint8_t *kt, uint32_t tcol, int r, int q) {
   const int sw = r & 7;
@@ -454,13 +492,8 @@ __device__ __forceinline__ void mags(const uint8_t *kt, uint32_t tcol, int r, in
       const uint4 im = lds128(kt + kHalfBlock + r * 128 + ((cc ^ sw) << 4));
       const uint32_t rw[4] = {re.x, re.y, re.z, re.w}, iw[4] = {im.x, im.y, im.z, im.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float ra = bf_lo(rw[e]), rb = bf_hi(rw[e]);
-        const float ia = bf_lo(iw[e]), ib = bf_hi(iw[e]);
-        const float ma = sqrt_approx(fmaf(ra, ra, ia * ia));
-        const float mb = sqrt_approx(fmaf(rb, rb, ib * ib));
-        split2(ma, mb, hi[4 * j + e], lo[4 * j + e]);
-      }
+      for (int e = 0; e < 4; ++e)
+        mag_pair(bf_lo(rw[e]), bf_hi(rw[e]), bf_lo(iw[e]), bf_hi(iw[e]), hi[4 * j + e], lo[4 * j + e]);
     }
   } else {
     const uint8_t *kh = kt + (q >> 1) * kHalfBlock;
@@ -468,109 +501,113 @@ __device__ __forceinline__ void mags(const uint8_t *kt, uint32_t tcol, int r, in
     for (int j = 0; j < 4; ++j) {
       const int cc = 4 * (q & 1) + j;
       const uint4 x = lds128(kh + r * 128 + ((cc ^ sw) << 4));
-      const float m0 = sqrt_approx(fmaf(bf_lo(x.x), bf_lo(x.x), bf_hi(x.x) * bf_hi(x.x)));
-      const float m1 = sqrt_approx(fmaf(bf_lo(x.y), bf_lo(x.y), bf_hi(x.y) * bf_hi(x.y)));
-      const float m2 = sqrt_approx(fmaf(bf_lo(x.z), bf_lo(x.z), bf_hi(x.z) * bf_hi(x.z)));
-      const float m3 = sqrt_approx(fmaf(bf_lo(x.w), bf_lo(x.w), bf_hi(x.w) * bf_hi(x.w)));
-      split2(m0, m1, hi[2 * j], lo[2 * j]);
-      split2(m2, m3, hi[2 * j + 1], lo[2 * j + 1]);
+      mag_pair(bf_lo(x.x), bf_lo(x.y), bf_hi(x.x), bf_hi(x.y), hi[2 * j], lo[2 * j]);
+      mag_pair(bf_lo(x.z), bf_lo(x.w), bf_hi(x.z), bf_hi(x.w), hi[2 * j + 1], lo[2 * j + 1]);
     }
   }
   tmem_st8(tcol + (uint32_t)(8 * q), hi);
   tmem_st8(tcol + (uint32_t)(32 + 8 * q), lo);
 }
 
+// Lane 0 waits on the barrier for the whole warp; __syncwarp orders the other
+// lanes after it.  Returns false (uniformly over the warp) on expiry/abort.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          int32_t *status, int lane) {
+  bool ok = true;
+  if (lane == 0) ok = mbar_wait(bar, parity, abort_flag, status);
+  ok = __shfl_sync(kFull, ok, 0) != 0;
+  __syncwarp();
+  return ok;
+}
+
+// Epilogue of tile j (record pr): raw scores of this warp's 32 rows and GQ
+// heads, fp64 moment sums, and the item's moment partials after its last tile.
+template <int G>
+__device__ __forceinline__ bool epilogue(const ScoreParams &p, TcSmem<G> &sm, uint32_t tmem, int j,
+                                         const SubRec &pr, int q, int rg, int lane,
+                                         double (&msum)[TcCfg<G>::GQ], double (&msq)[TcCfg<G>::GQ]) {
+  constexpr int NCOL = TcCfg<G>::NCOL, GQ = TcCfg<G>::GQ;
+  const Geom &geo = p.geo;
+  const bool active = (G >= 4) || q < G;  // quarter q scores heads [q GQ, (q + 1) GQ)
+  if (!warp_wait(&sm.accfull[j % kNB], (j / kNB) & 1, &sm.abort_flag, p.status, lane)) return false;
+  tc_fence_after();
+  if (pr.flags & kFlagFirst) {
+#pragma unroll
+    for (int g = 0; g < GQ; ++g) msum[g] = msq[g] = 0.0;
+  }
+  if (active) {
+    float v[2 * GQ];
+    tmem_ld<2 * GQ>(tmem + ((uint32_t)(32 * rg) << 16) + (uint32_t)((j % kNB) * NCOL + q * 2 * GQ), v);
+    const int slot = pr.slot0 + rg * 32 + lane;
+    if (slot >= geo.sinks && slot < pr.N - geo.window) {
+      float sc[GQ];
+#pragma unroll
+      for (int g = 0; g < GQ; ++g) {
+        sc[g] = v[2 * g] + v[2 * g + 1];
+        msum[g] += (double)sc[g];
+        msq[g] = fma((double)sc[g], (double)sc[g], msq[g]);
+      }
+      float *dst = p.raw + pr.u * p.raw_stride + (int64_t)(slot - geo.sinks) * G + q * GQ;
+      if constexpr (GQ == 4) {
+        *reinterpret_cast<float4 *>(dst) = make_float4(sc[0], sc[1], sc[2], sc[3]);
+      } else if constexpr (GQ == 2) {
+        *reinterpret_cast<float2 *>(dst) = make_float2(sc[0], sc[1]);
+      } else {
+        dst[0] = sc[0];
+      }
+    }
+  }
+  tc_fence_before();
+  if ((pr.flags & kFlagLast) && active) {
+#pragma unroll
+    for (int g = 0; g < GQ; ++g) {
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) {
+        msum[g] += __shfl_xor_sync(kFull, msum[g], o);
+        msq[g] += __shfl_xor_sync(kFull, msq[g], o);
+      }
+    }
+    if (lane == 0) {
+      double *m = p.moments + (((pr.u * geo.tiles_max + pr.tile) * kRowGroups + rg) * G + q * GQ) * 2;
+#pragma unroll
+      for (int g = 0; g < GQ; ++g) {
+        m[2 * g] = msum[g];
+        m[2 * g + 1] = msq[g];
+      }
+    }
+  }
+  return true;
+}
+
 template <int G, int PAIR>
 __device__ void compute(const ScoreParams &p, TcSmem<G> &sm, uint32_t tmem, int tid) {
-  constexpr int ST = TcCfg<G>::STAGES, NCOL = TcCfg<G>::NCOL, GQ = TcCfg<G>::GQ;
-  const Geom &geo = p.geo;
+  constexpr int ST = TcCfg<G>::STAGES, GQ = TcCfg<G>::GQ;
   const int warp = tid >> 5, lane = tid & 31;
-  const int q = warp >> 2, r = (warp & 3) * 32 + lane;
-  const bool active = (G >= 4) || q < G;  // quarter q scores heads [q GQ, (q + 1) GQ)
-  const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+  const int q = warp >> 2, rg = warp & 3, r = rg * 32 + lane;
+  const uint32_t mag_base = tmem + ((uint32_t)(32 * rg) << 16) + kTmemMag;
   double msum[GQ], msq[GQ];
 #pragma unroll
   for (int g = 0; g < GQ; ++g) msum[g] = msq[g] = 0.0;
-  SubRec prev{};
-  bool have_prev = false;
+  SubRec p0, p1;  // records of tiles i - 2 and i - 1
   for (int i = 0;; ++i) {
     const int stage = i % ST;
-    mbar_wait(&sm.full[stage], (i / ST) & 1, &sm.abort_flag, p.status);
-    csync<kBarCompute, kComputeThreads>();
-    if (sm.abort_flag) break;
+    if (!warp_wait(&sm.full[stage], (i / ST) & 1, &sm.abort_flag, p.status, lane)) return;
     const SubRec rec = sm.rec[stage];
     const bool end = (rec.flags & kFlagEnd) != 0;
     if (!end) {
-      mags<PAIR>(&sm.k[stage][0][0], tmem + lane_base + kTmemMag + (uint32_t)((i & 1) * 64), r, q);
+      mags<PAIR>(&sm.k[stage][0][0], mag_base + (uint32_t)((i % kNB) * 64), r, q);
       tmem_wait_st();
       tc_fence_before();
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.aready[i & 1]);
-    if (have_prev) {
-      const int j = i - 1;
-      mbar_wait(&sm.accfull[j & 1], (j >> 1) & 1, &sm.abort_flag, p.status);
-      csync<kBarCompute, kComputeThreads>();
-      if (sm.abort_flag) break;
-      tc_fence_after();
-      if (prev.flags & kFlagFirst) {
-#pragma unroll
-        for (int g = 0; g < GQ; ++g) msum[g] = msq[g] = 0.0;
-      }
-      if (active) {
-        float v[2 * GQ];
-        tmem_ld<2 * GQ>(tmem + lane_base + (uint32_t)((j & 1) * NCOL + q * 2 * GQ), v);
-        const int slot = prev.slot0 + r;
-        if (slot >= geo.sinks && slot < prev.N - geo.window) {
-          float sc[GQ];
-#pragma unroll
-          for (int g = 0; g < GQ; ++g) {
-            sc[g] = v[2 * g] + v[2 * g + 1];
-            msum[g] += (double)sc[g];
-            msq[g] = fma((double)sc[g], (double)sc[g], msq[g]);
-          }
-          float *dst = p.raw + prev.u * p.raw_stride + (int64_t)(slot - geo.sinks) * G + q * GQ;
-          if constexpr (GQ == 4) {
-            *reinterpret_cast<float4 *>(dst) = make_float4(sc[0], sc[1], sc[2], sc[3]);
-          } else if constexpr (GQ == 2) {
-            *reinterpret_cast<float2 *>(dst) = make_float2(sc[0], sc[1]);
-          } else {
-            dst[0] = sc[0];
-          }
-        }
-      }
-      tc_fence_before();
-      if (prev.flags & kFlagLast) {
-        // item done: its moment partials, summed over rows in a fixed order
-#pragma unroll
-        for (int g = 0; g < GQ; ++g) {
-#pragma unroll
-          for (int o = 16; o >= 1; o >>= 1) {
-            msum[g] += __shfl_xor_sync(kFull, msum[g], o);
-            msq[g] += __shfl_xor_sync(kFull, msq[g], o);
-          }
-          if (lane == 0) {
-            sm.mom[warp][g][0] = msum[g];
-            sm.mom[warp][g][1] = msq[g];
-          }
-        }
-        csync<kBarCompute, kComputeThreads>();
-        if (tid < G) {
-          const int qq = tid / GQ, gl = tid % GQ;
-          double s1 = 0.0, s2 = 0.0;
-          for (int w = 4 * qq; w < 4 * qq + 4; ++w) {
-            s1 += sm.mom[w][gl][0];
-            s2 += sm.mom[w][gl][1];
-          }
-          double *m = p.moments + ((prev.u * geo.tiles_max + prev.tile) * G + tid) * 2;
-          m[0] = s1;
-          m[1] = s2;
-        }
-      }
+    if (lane == 0) mbar_arrive(&sm.aready[i % kNB]);
+    if (i >= 2 && !epilogue<G>(p, sm, tmem, i - 2, p0, q, rg, lane, msum, msq)) return;
+    if (end) {
+      if (i >= 1) epilogue<G>(p, sm, tmem, i - 1, p1, q, rg, lane, msum, msq);
+      return;
     }
-    if (end) break;
-    prev = rec;
-    have_prev = true;
+    p0 = p1;
+    p1 = rec;
   }
 }
 
@@ -590,11 +627,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) score_tc_kernel(const __grid_co
       mbar_init(&sm.full[i], 1);
       mbar_init(&sm.kempty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kNB; ++i) {
       mbar_init(&sm.aready[i], kComputeWarps);
       mbar_init(&sm.accfull[i], 1);
-      mbar_init(&sm.bempty[i], 1);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(&sm.bempty[i], 1);
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
