@@ -250,6 +250,50 @@ tria_status tria_compress_pass(const tria_stats *stats, const tria_cache_view *c
                                tria_stream_t stream);
 
 /*
+ * tria_compress_pass_static - tria_compress_pass without a workspace
+ * argument: the scratch is a fixed device array inside this library.  The
+ * paper has no counterpart of this call; it serves callers that cannot give
+ * the library a workspace allocation, such as a serving engine that reserves
+ * all free device memory for its KV-cache block pool at start-up (a later
+ * cudaMalloc would fail or eat into the pool), or a decode loop that must not
+ * stall other streams (cudaMalloc and cudaFree may synchronise the device).
+ * The call allocates nothing: no cudaMalloc, cudaFree or allocating library
+ * routine.  On `stream` it enqueues a memset of the scratch header, the
+ * pass's kernels and, with device_status, one device-to-device copy.
+ *
+ * Scratch: TRIA_STATIC_SCRATCH_BYTES (32 MiB, 256-byte aligned) of device
+ * memory per device, held for as long as the library is loaded.  The first
+ * call made while a given device is current looks up that device's address
+ * of the array (cudaGetSymbolAddress, which may load the library's device
+ * code on that device) and keeps it; make that first call on each device
+ * before any stream capture begins.  The current device's array is used:
+ * `stream` must belong to the current device.
+ * Limit: the pass over all layers must need at most TRIA_STATIC_SCRATCH_BYTES
+ * of workspace (tria_workspace_size with layers [0, n_layers)); a larger one
+ * returns TRIA_ERR_WORKSPACE with nothing enqueued.  32 MiB holds, for
+ * example, one 32K-token sequence of 8 KV heads x 8 query heads per KV head
+ * for up to 3 layers.
+ * Zeroing: each call clears the scratch header (work counter and status
+ * flags) on `stream` before its kernels; the kernels rewrite every other
+ * scratch region before reading it, so nothing carries over between calls.
+ * Races: every call on a device uses the same array.  Calls ordered on one
+ * stream are safe; calls that may overlap on the device (other streams or
+ * host threads with no ordering between them) race on the scratch and give
+ * undefined results.
+ * device_status: optional device int32; receives this call's status flags
+ * (bits as in tria_read_device_status) after the compaction.
+ * kept_idx, freed_blocks, n_freed, results and errors as in
+ * tria_compress_pass; also UNSUPPORTED when the current device ordinal is 64
+ * or more.
+ */
+#define TRIA_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+tria_status tria_compress_pass_static(const tria_stats *stats, const tria_cache_view *cache,
+                                      const tria_params *params, int32_t *kept_idx,
+                                      int32_t *freed_blocks, int32_t *n_freed,
+                                      int32_t *device_status, tria_stream_t stream);
+
+/*
  * tria_read_device_status - errors the kernels found in device-resident
  * inputs during the calls that used this workspace (bit 0: a seq_lens entry
  * outside [0, max_seq_len]; such a unit is skipped and its kept row is all

@@ -27,7 +27,9 @@ MAX_LAYERS = 128
 
 EXPORTS = ["tria_status_string", "tria_version", "tria_load_stats", "tria_free_stats",
            "tria_stats_desc", "tria_workspace_size", "tria_score", "tria_select", "tria_compact",
-           "tria_compress_pass", "tria_read_device_status", "tria_set_pass_events"]
+           "tria_compress_pass", "tria_read_device_status", "tria_set_pass_events",
+           "tria_compress_pass_static"]
+STATIC_SCRATCH_BYTES = 32 * 1024 * 1024   # TRIA_STATIC_SCRATCH_BYTES
 
 
 class TriaError(RuntimeError):
@@ -92,6 +94,8 @@ def lib() -> ctypes.CDLL:
                                      _VP, _VP, _VP, ctypes.c_size_t, _VP]
     L.tria_read_device_status.argtypes = [_VP, _VP, ctypes.POINTER(ctypes.c_int32)]
     L.tria_set_pass_events.argtypes = [ctypes.POINTER(_VP)]
+    L.tria_compress_pass_static.argtypes = [_VP, ctypes.POINTER(CacheView),
+                                            ctypes.POINTER(Params), _VP, _VP, _VP, _VP, _VP]
     for name in EXPORTS:
         if name not in ("tria_status_string", "tria_version"):
             getattr(L, name).restype = _I
@@ -240,6 +244,25 @@ def tria_compress_pass(stats, cache, prm, kept_idx, workspace, freed_blocks=None
                                     _ptr(kept_idx), _ptr(freed_blocks), _ptr(n_freed),
                                     _ptr(workspace), workspace.numel() * workspace.element_size(),
                                     _stream(stream)), "tria_compress_pass")
+
+
+def tria_compress_pass_static(stats, cache, prm, kept_idx=None, freed_blocks=None,
+                              n_freed=None, device_status=None, stream=None):
+    """tria_compress_pass with the library's fixed 32 MiB device scratch instead
+    of a workspace: for callers that may not allocate device memory (an engine
+    whose KV-cache pool holds all free memory, a loop that must not stall on
+    cudaMalloc/cudaFree).  One scratch per device, shared by every call: calls
+    that may overlap on the device race.  Make the first call on each device
+    before any stream capture (it looks up the scratch address)."""
+    rc = lib().tria_compress_pass_static(stats.handle, ctypes.byref(cache.view),
+                                         ctypes.byref(prm), _ptr(kept_idx), _ptr(freed_blocks),
+                                         _ptr(n_freed), _ptr(device_status), _stream(stream))
+    if rc == 3:  # TRIA_ERR_WORKSPACE: say how much the pass needs
+        need = tria_workspace_size(stats, cache, prm)
+        raise TriaError(rc, f"tria_compress_pass_static: the pass needs {need} bytes of scratch, "
+                            f"the static scratch holds {STATIC_SCRATCH_BYTES}; use "
+                            f"tria_compress_pass with a workspace")
+    _check(rc, "tria_compress_pass_static")
 
 
 def tria_read_device_status(workspace, stream=None) -> int:
