@@ -518,13 +518,16 @@ tria_status tria_compress_pass(const tria_stats *stats, const tria_cache_view *c
   if ((st = make_score(g, cache, 0, L, ws, wl, sp)) != TRIA_OK) return st;
   TailParams tp = make_tail(g, cache, ws, wl);
   tp.kept = kept;
+  // one block per unit when its candidates' keys fit in shared memory, else
+  // blocks over candidate chunks with a histogram in the workspace
+  const bool per_unit = unit_tail_fits(g);
   if (mark(0, s) != cudaSuccess) return TRIA_ERR_CUDA;
-  if (launch_coef(make_coef(stats, g, cache, ws, wl, kept, true), s) != cudaSuccess)
+  if (launch_coef(make_coef(stats, g, cache, ws, wl, kept, !per_unit), s) != cudaSuccess)
     return TRIA_ERR_CUDA;
   if (mark(1, s) != cudaSuccess) return TRIA_ERR_CUDA;
   if (launch_score(sp, s) != cudaSuccess) return TRIA_ERR_CUDA;
   if (mark(2, s) != cudaSuccess) return TRIA_ERR_CUDA;
-  if (launch_tail(tp, s) != cudaSuccess) return TRIA_ERR_CUDA;
+  if ((per_unit ? launch_unit_tail(tp, s) : launch_tail(tp, s)) != cudaSuccess) return TRIA_ERR_CUDA;
   if (mark(3, s) != cudaSuccess) return TRIA_ERR_CUDA;
   CompactParams cp{};
   cp.geo = g;

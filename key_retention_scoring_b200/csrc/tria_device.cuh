@@ -151,8 +151,8 @@ __device__ __forceinline__ void clear_words(uint32_t *w, int n, int tid) {
 
 // Pick the bin holding the `remaining`-th largest key among nbins bins
 // (digit at `shift`); updates prefix, remaining, bin_count.
-template <int BAR, int NT>
-__device__ void pick_bin(const uint32_t *hist, int nbins, SelScalars &sc, int shift, int tid) {
+template <int BAR, int NT, class Sc>
+__device__ void pick_bin(const uint32_t *hist, int nbins, Sc &sc, int shift, int tid) {
   const int per = nbins / NT;  // bins per thread, descending
   int v = 0;
   for (int e = 0; e < per; ++e) v += (int)hist[nbins - 1 - (tid * per + e)];
@@ -369,33 +369,30 @@ __device__ void select_unit(const float *agg, int C, int K, int N, int B, int W,
 // agg_range: agg[c] = max_g (S_g[c] - mean_g) * inv_g for c in [c0, c1), with
 // the histogram of the top 12 key bits added into hist when it is non-null.
 // ---------------------------------------------------------------------------
-template <int G, int BAR, int NT>
-__device__ void unit_norm(const double *mom_unit, int ntiles, int C, int tid, SelScalars &sc) {
-  // every thread sums a fixed subset of the partials, then a fixed-order
-  // butterfly over the warp and a sequential sum over the warps
-  double s1[G], s2[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) s1[g] = s2[g] = 0.0;
+template <int G, int BAR, int NT, class Sc>
+__device__ void unit_norm(const double *mom_unit, int ntiles, int C, int tid, Sc &sc) {
+  // thread tid sums head g = tid % G over the partials i = tid / G + k NT / G
+  // (coalesced 16-byte loads), then lanes of equal head reduce by a fixed
+  // butterfly and warp results are summed in warp order
+  static_assert(NT % 32 == 0 && 32 % G == 0, "heads per warp");
+  const int g = tid % G;
+  double s1 = 0.0, s2 = 0.0;
   const int n = ntiles * kRowGroups;
-  for (int i = tid; i < n; i += NT) {
+  const double2 *m2 = reinterpret_cast<const double2 *>(mom_unit);
+  for (int i = tid / G; i < n; i += NT / G) {
+    const double2 v = __ldcg(m2 + (int64_t)i * G + g);
+    s1 += v.x;
+    s2 += v.y;
+  }
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      s1[g] += __ldcg(mom_unit + ((int64_t)i * G + g) * 2);
-      s2[g] += __ldcg(mom_unit + ((int64_t)i * G + g) * 2 + 1);
-    }
+  for (int o = 16; o >= G; o >>= 1) {
+    s1 += __shfl_xor_sync(kFull, s1, o);
+    s2 += __shfl_xor_sync(kFull, s2, o);
   }
   const int lane = tid & 31, w = tid >> 5;
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      s1[g] += __shfl_xor_sync(kFull, s1[g], o);
-      s2[g] += __shfl_xor_sync(kFull, s2[g], o);
-    }
-    if (lane == 0) {
-      sc.red[w][g][0] = s1[g];
-      sc.red[w][g][1] = s2[g];
-    }
+  if (lane < G) {
+    sc.red[w][g][0] = s1;
+    sc.red[w][g][1] = s2;
   }
   csync<BAR, NT>();
   if (tid < G) {
@@ -462,6 +459,187 @@ __device__ void agg_range(const float *__restrict__ raw, float *agg, int c0, int
     const float a = agg_of(v);
     agg[cc] = a;
     if (hist != nullptr) atomicAdd(hist + (order_key(a) >> 20), 1u);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Per-unit tail with the candidates' agg keys in shared memory (one block of
+// NT threads per unit).
+// unit_keys: keys[c] = order_key(agg[c]), agg[c] = max_g (S_g[c] - mean_g)
+// inv_g (NaN when any term is), from one coalesced pass over the unit's raw
+// scores [C][G]; adds the top 12 key bits of every candidate to hist.
+// select_keys: radix top-K over the keys (digits of 12, 12 and 8 bits), then
+// the ascending kept list: sinks, the K candidates above the threshold key T
+// plus the lowest-slot keys equal to T, the window.
+// ---------------------------------------------------------------------------
+struct UnitScalars {
+  int warp_tmp[32];
+  uint32_t prefix;
+  int remaining;
+  int digit;
+  int above;
+  int bin_count;
+  int warp_gt[32];
+  int warp_eq[32];
+  float mean[TRIA_MAX_GROUP];
+  float inv[TRIA_MAX_GROUP];
+  double red[32][TRIA_MAX_GROUP][2];
+};
+
+template <int G, int NT>
+__device__ void unit_keys(const float *raw, int C, const float *s_mean, const float *s_inv,
+                          uint32_t *keys, uint32_t *hist, int tid) {
+  const int lane = tid & 31;
+  constexpr int U = 4;  // float4 loads in flight per thread
+  const float4 *src = reinterpret_cast<const float4 *>(raw);
+  if constexpr (G >= 4) {
+    // LPC lanes per candidate, each with 4 of its G heads
+    constexpr int LPC = G / 4;
+    const int h0 = (tid % LPC) * 4;
+    float m[4], iv[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      m[k] = s_mean[h0 + k];
+      iv[k] = s_inv[h0 + k];
+    }
+    const int n4 = C * LPC;
+    for (int j0 = 0; j0 < n4; j0 += NT * U) {
+      float4 x[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = j0 + u * NT + tid;
+        x[u] = (j < n4) ? __ldcs(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = j0 + u * NT + tid;
+        const float z0 = __fmul_rn(__fsub_rn(x[u].x, m[0]), iv[0]);
+        const float z1 = __fmul_rn(__fsub_rn(x[u].y, m[1]), iv[1]);
+        const float z2 = __fmul_rn(__fsub_rn(x[u].z, m[2]), iv[2]);
+        const float z3 = __fmul_rn(__fsub_rn(x[u].w, m[3]), iv[3]);
+        int nan = (z0 != z0) | (z1 != z1) | (z2 != z2) | (z3 != z3);
+        float a = fmaxf(fmaxf(z0, z1), fmaxf(z2, z3));
+#pragma unroll
+        for (int o = 1; o < LPC; o <<= 1) {
+          a = fmaxf(a, __shfl_xor_sync(kFull, a, o));
+          nan |= __shfl_xor_sync(kFull, nan, o);
+        }
+        const uint32_t k = nan ? 0u : order_key(a);
+        const bool lead = (j < n4) && (tid % LPC) == 0;
+        if (lead) keys[j / LPC] = k;
+        hist_add(hist, k >> 20, lead, lane);
+      }
+    }
+  } else {
+    // a float4 holds CPF = 4 / G candidates
+    constexpr int CPF = 4 / G;
+    float m[G], iv[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      m[g] = s_mean[g];
+      iv[g] = s_inv[g];
+    }
+    const int n4 = (C + CPF - 1) / CPF;
+    for (int j0 = 0; j0 < n4; j0 += NT * U) {
+      float4 x[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = j0 + u * NT + tid;
+        x[u] = (j < n4) ? __ldcs(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = j0 + u * NT + tid;
+        const float v[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+        for (int e = 0; e < CPF; ++e) {
+          const int c = j * CPF + e;
+          float a = 0.0f;
+          int nan = 0;
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float z = __fmul_rn(__fsub_rn(v[e * G + g], m[g]), iv[g]);
+            a = (g == 0) ? z : fmaxf(a, z);
+            nan |= (z != z);
+          }
+          const uint32_t k = nan ? 0u : order_key(a);
+          const bool in = (j < n4) && c < C;
+          if (in) keys[c] = k;
+          hist_add(hist, k >> 20, in, lane);
+        }
+      }
+    }
+  }
+}
+
+template <int NT>
+__device__ void select_keys(const uint32_t *keys, int C, int K, int N, int B, int W, int S,
+                            int32_t *kept, uint32_t *hist, UnitScalars &sc, int tid) {
+  const int lane = tid & 31, warp = tid >> 5;
+  for (int j = tid; j < S; j += NT) kept[j] = j;
+  for (int j = tid; j < W; j += NT) kept[B - W + j] = N - W + j;
+  if (K <= 0) return;
+  if (tid == 0) {
+    sc.prefix = 0u;
+    sc.remaining = K;
+  }
+  __syncthreads();
+  pick_bin<0, NT>(hist, kHistBins, sc, 20, tid);
+  // digits 2 (bits [19:8]) and 3 (bits [7:0]) over the keys of the chosen bin
+#pragma unroll 1
+  for (int level = 1; level <= 2; ++level) {
+    const int hi_shift = level == 1 ? 20 : 8;
+    const int sh = level == 1 ? 8 : 0;
+    const uint32_t dmask = level == 1 ? 0xfffu : 0xffu;
+    clear_words<NT>(hist, kHistBins, tid);
+    __syncthreads();
+    const uint32_t pre = sc.prefix >> hi_shift;
+    for (int c = tid; c < C; c += NT) {
+      const uint32_t k = keys[c];
+      if ((k >> hi_shift) == pre) atomicAdd(hist + ((k >> sh) & dmask), 1u);
+    }
+    __syncthreads();
+    pick_bin<0, NT>(hist, kHistBins, sc, sh, tid);
+  }
+  const uint32_t T = sc.prefix;
+  const int need = sc.remaining;  // keys equal to T to take, lowest slots first (>= 1)
+  // emission: warp w walks candidates [w * per_w, (w + 1) * per_w) 32 at a time
+  const int steps = (C + NT - 1) / NT;
+  const int cb = warp * steps * 32;
+  int gt = 0, eq = 0;
+  for (int e = 0; e < steps; ++e) {
+    const int c = cb + e * 32 + lane;
+    const uint32_t k = (c < C) ? keys[c] : 0u;
+    gt += __popc(__ballot_sync(kFull, c < C && k > T));
+    eq += __popc(__ballot_sync(kFull, c < C && k == T));
+  }
+  if (lane == 0) {
+    sc.warp_gt[warp] = gt;
+    sc.warp_eq[warp] = eq;
+  }
+  __syncthreads();
+  int gt_before = 0, eq_before = 0;
+  for (int i = 0; i < warp; ++i) {
+    gt_before += sc.warp_gt[i];
+    eq_before += sc.warp_eq[i];
+  }
+  int run_keep = gt_before + min(eq_before, need);
+  int run_eq = eq_before;
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int e = 0; e < steps; ++e) {
+    const int c = cb + e * 32 + lane;
+    const bool valid = c < C;
+    const uint32_t k = valid ? keys[c] : 0u;
+    const bool is_eq = valid && k == T;
+    const uint32_t beq = __ballot_sync(kFull, is_eq);
+    const bool keep = valid && (k > T || (is_eq && run_eq + __popc(beq & lt) < need));
+    const uint32_t bk = __ballot_sync(kFull, keep);
+    if (keep) {
+      const int pos = run_keep + __popc(bk & lt);
+      if (pos < K) kept[S + pos] = S + c;
+    }
+    run_eq += __popc(beq);
+    run_keep += __popc(bk);
   }
 }
 

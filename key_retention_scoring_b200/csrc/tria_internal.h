@@ -75,6 +75,8 @@ struct WsLayout {
 
 constexpr int kAggHistBins = 4096;
 constexpr int kAggChunk = 4096;   // candidates per block of the normalization kernel
+constexpr int kUnitTailMaxC = 49152;       // candidates per unit of the one-block-per-unit tail
+constexpr size_t kMaxDynSmem = 232448;     // opt-in shared memory per block (227 KB)
 
 WsLayout ws_layout(const Geom &g);
 
@@ -148,6 +150,10 @@ cudaError_t launch_coef(const CoefParams &p, cudaStream_t st);
 cudaError_t launch_score(const ScoreParams &p, cudaStream_t st);
 cudaError_t launch_tail(const TailParams &p, cudaStream_t st);
 cudaError_t launch_select(const SelectParams &p, cudaStream_t st);
+// Normalize-then-max + selection with one block per unit (kept != null);
+// only when unit_tail_fits(geo).
+bool unit_tail_fits(const Geom &g);
+cudaError_t launch_unit_tail(const TailParams &p, cudaStream_t st);
 cudaError_t launch_compact(const CompactParams &p, cudaStream_t st);
 
 }  // namespace tria

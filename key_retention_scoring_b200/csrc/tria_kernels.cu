@@ -202,6 +202,51 @@ __global__ void __launch_bounds__(kThreads) tail_kernel(const __grid_constant__ 
 }
 
 // ---------------------------------------------------------------------------
+// unit_tail_kernel: normalize-then-max and selection with one block of
+// kUnitThreads per unit (units strided over the grid), for passes whose
+// candidates' keys fit in shared memory.  The unit's raw scores are read
+// once; agg lives only as order keys in shared memory.
+// ---------------------------------------------------------------------------
+constexpr int kUnitThreads = 1024;
+
+size_t unit_tail_smem_bytes(int c_max) {
+  return sizeof(UnitScalars) + (size_t)kHistBins * 4 + (size_t)((c_max + 3) & ~3) * 4;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kUnitThreads, 1) unit_tail_kernel(const __grid_constant__ TailParams p) {
+  extern __shared__ __align__(16) uint8_t smem_ut[];
+  UnitScalars &sc = *reinterpret_cast<UnitScalars *>(smem_ut);
+  uint32_t *hist = reinterpret_cast<uint32_t *>(smem_ut + sizeof(UnitScalars));
+  uint32_t *keys = hist + kHistBins;
+  const Geom &geo = p.geo;
+  const int t = threadIdx.x;
+  const int K = geo.budget - geo.window - geo.sinks;
+  for (int64_t u = blockIdx.x; u < geo.n_units; u += gridDim.x) {
+    const int s = (int)(u / ((int64_t)geo.nl * geo.hkv));
+    const int N = p.seq_lens[s];
+    // invalid lengths and units within the budget: the coefficient kernel
+    // wrote their kept rows and flagged the former
+    if (N < 0 || N > geo.max_seq_len || N <= geo.budget) continue;
+    const int C = N - geo.window - geo.sinks;
+    unit_norm<G, 0, kUnitThreads>(p.moments + u * geo.tiles_max * kRowGroups * G * 2,
+                                  unit_tiles(N, geo.window, geo.sinks), C, t, sc);
+    clear_words<kUnitThreads>(hist, kHistBins, t);
+    __syncthreads();
+    const float *raw = p.raw + u * p.raw_stride;
+    unit_keys<G, kUnitThreads>(raw, C, sc.mean, sc.inv, keys, hist, t);
+    __syncthreads();
+    if (p.discard_raw) {
+      const int64_t lines = ((int64_t)C * G * 4 + 127) / 128;
+      for (int64_t i = t; i < lines; i += kUnitThreads) discard_line(raw + i * 32);
+    }
+    select_keys<kUnitThreads>(keys, C, K, N, geo.budget, geo.window, geo.sinks,
+                              p.kept + u * geo.budget, hist, sc, t);
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
 // select_kernel: one CTA per unit
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads) select_kernel(const __grid_constant__ SelectParams p) {
@@ -331,6 +376,38 @@ cudaError_t launch_tail(const TailParams &p, cudaStream_t st) {
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
+}
+
+template <int G>
+cudaError_t launch_unit_tail_g(const TailParams &p, size_t smem, cudaStream_t st) {
+  auto kern = unit_tail_kernel<G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0, per_sm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kUnitThreads, smem)) != cudaSuccess)
+    return e;
+  int64_t grid = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
+  if (grid > p.geo.n_units) grid = p.geo.n_units;
+  kern<<<(unsigned)grid, kUnitThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+bool unit_tail_fits(const Geom &g) {
+  return g.c_max <= kUnitTailMaxC && unit_tail_smem_bytes(g.c_max) <= kMaxDynSmem;
+}
+
+cudaError_t launch_unit_tail(const TailParams &p, cudaStream_t st) {
+  const size_t smem = unit_tail_smem_bytes(p.geo.c_max);
+  switch (p.geo.g) {
+    case 1: return launch_unit_tail_g<1>(p, smem, st);
+    case 2: return launch_unit_tail_g<2>(p, smem, st);
+    case 4: return launch_unit_tail_g<4>(p, smem, st);
+    case 8: return launch_unit_tail_g<8>(p, smem, st);
+    case 16: return launch_unit_tail_g<16>(p, smem, st);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_select(const SelectParams &p, cudaStream_t st) {

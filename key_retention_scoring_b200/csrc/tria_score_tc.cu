@@ -55,11 +55,21 @@ constexpr int kNB = 4;
 constexpr uint32_t kTmemCols = 512;         // [0, kNB*NCOL): accumulators; [128, 384): magnitude tiles
 constexpr uint32_t kTmemMag = 128;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint32_t kSuspendNs = 1000000;    // a blocked try_wait sleeps up to 1 ms per call
 
 struct SubRec {
+  float *raw;      // the unit's raw scores, candidate 0
+  double *mom;     // the item's moment partials
   long long u;
   int s, lrel, h, tile, N;
   int slot0, flags, bpar;  // first slot of the 128-row tile (a multiple of 128)
+};
+
+// What the epilogue of a tile needs from its record.
+struct EpRec {
+  float *raw;
+  double *mom;
+  int slot0, N, flags;
 };
 
 template <int G>
@@ -118,21 +128,32 @@ __device__ __forceinline__ uint64_t global_timer() {
   return t;
 }
 
-// Bounded wait for the phase of `parity`; false on expiry or abort.
+// try_wait that may suspend the thread (up to kSuspendNs) until the phase
+// completes, instead of returning at once.
+__device__ __forceinline__ bool mbar_try_sleep(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity), "n"(kSuspendNs)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait (one thread) for the phase of `parity`; false on expiry or abort.
 __device__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                           int32_t *status) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try(a, parity)) return true;
   const uint64_t t0 = global_timer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try(a, parity)) return true;
-    if ((it & 255u) == 0u) {
-      if (*abort_flag) return false;
-      if (global_timer() - t0 > kWaitLimitNs) {
-        *abort_flag = 1;
-        atomicOr(status, 2);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_sleep(a, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_timer() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicOr(status, 2);
+      return false;
     }
   }
 }
@@ -397,6 +418,8 @@ __device__ void producer(const ScoreParams &p, TcSmem<G> &sm, int n_items, int l
     if (lane == 0) {
       SubRec &r = sm.rec[stage];
       r.u = u; r.s = s; r.lrel = lrel; r.h = h; r.tile = tile; r.N = N; r.slot0 = slot0;
+      r.raw = p.raw + u * p.raw_stride;
+      r.mom = p.moments + (u * geo.tiles_max + tile) * kRowGroups * G * 2;
       r.flags = (first ? kFlagFirst : 0) | (sub == sub_end - 1 ? kFlagLast : 0);
       r.bpar = bpar;
       mbar_arrive_expect_tx(&sm.full[stage], bytes);
@@ -509,22 +532,31 @@ __device__ __forceinline__ void mags(const uint8_t *kt, uint32_t tcol, int r, in
   tmem_st8(tcol + (uint32_t)(32 + 8 * q), lo);
 }
 
-// Lane 0 waits on the barrier for the whole warp; __syncwarp orders the other
-// lanes after it.  Returns false (uniformly over the warp) on expiry/abort.
+// Bounded wait of a whole warp (every lane tests the barrier; the warp
+// leaves together).  Returns false, uniformly over the warp, on expiry/abort.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                           int32_t *status, int lane) {
-  bool ok = true;
-  if (lane == 0) ok = mbar_wait(bar, parity, abort_flag, status);
-  ok = __shfl_sync(kFull, ok, 0) != 0;
-  __syncwarp();
-  return ok;
+  const uint32_t a = smem_u32(bar);
+  if (__all_sync(kFull, mbar_try(a, parity))) return true;
+  const uint64_t t0 = global_timer();
+  for (;;) {
+    if (__all_sync(kFull, mbar_try_sleep(a, parity))) return true;
+    if (__any_sync(kFull, *abort_flag != 0)) return false;
+    if (__any_sync(kFull, global_timer() - t0 > kWaitLimitNs)) {
+      if (lane == 0) {
+        *abort_flag = 1;
+        atomicOr(status, 2);
+      }
+      return false;
+    }
+  }
 }
 
 // Epilogue of tile j (record pr): raw scores of this warp's 32 rows and GQ
 // heads, fp64 moment sums, and the item's moment partials after its last tile.
 template <int G>
 __device__ __forceinline__ bool epilogue(const ScoreParams &p, TcSmem<G> &sm, uint32_t tmem, int j,
-                                         const SubRec &pr, int q, int rg, int lane,
+                                         const EpRec &pr, int q, int rg, int lane,
                                          double (&msum)[TcCfg<G>::GQ], double (&msq)[TcCfg<G>::GQ]) {
   constexpr int NCOL = TcCfg<G>::NCOL, GQ = TcCfg<G>::GQ;
   const Geom &geo = p.geo;
@@ -547,7 +579,7 @@ __device__ __forceinline__ bool epilogue(const ScoreParams &p, TcSmem<G> &sm, ui
         msum[g] += (double)sc[g];
         msq[g] = fma((double)sc[g], (double)sc[g], msq[g]);
       }
-      float *dst = p.raw + pr.u * p.raw_stride + (int64_t)(slot - geo.sinks) * G + q * GQ;
+      float *dst = pr.raw + (slot - geo.sinks) * G + q * GQ;
       if constexpr (GQ == 4) {
         *reinterpret_cast<float4 *>(dst) = make_float4(sc[0], sc[1], sc[2], sc[3]);
       } else if constexpr (GQ == 2) {
@@ -568,7 +600,7 @@ __device__ __forceinline__ bool epilogue(const ScoreParams &p, TcSmem<G> &sm, ui
       }
     }
     if (lane == 0) {
-      double *m = p.moments + (((pr.u * geo.tiles_max + pr.tile) * kRowGroups + rg) * G + q * GQ) * 2;
+      double *m = pr.mom + (rg * G + q * GQ) * 2;
 #pragma unroll
       for (int g = 0; g < GQ; ++g) {
         m[2 * g] = msum[g];
@@ -588,26 +620,40 @@ __device__ void compute(const ScoreParams &p, TcSmem<G> &sm, uint32_t tmem, int 
   double msum[GQ], msq[GQ];
 #pragma unroll
   for (int g = 0; g < GQ; ++g) msum[g] = msq[g] = 0.0;
-  SubRec p0, p1;  // records of tiles i - 2 and i - 1
-  for (int i = 0;; ++i) {
+  // Tile i: magnitudes of tile i, then the epilogue of tile i - 2 (record
+  // `older`, replaced by tile i's record); after the end marker also the
+  // epilogue of tile i - 1 (record `other`).  0: go on, 1: done, -1: abort.
+  auto step = [&](int i, EpRec &older, EpRec &other) -> int {
     const int stage = i % ST;
-    if (!warp_wait(&sm.full[stage], (i / ST) & 1, &sm.abort_flag, p.status, lane)) return;
-    const SubRec rec = sm.rec[stage];
-    const bool end = (rec.flags & kFlagEnd) != 0;
+    if (!warp_wait(&sm.full[stage], (i / ST) & 1, &sm.abort_flag, p.status, lane)) return -1;
+    const SubRec &rc = sm.rec[stage];
+    const int flags = rc.flags;
+    const bool end = (flags & kFlagEnd) != 0;
+    EpRec cur;
     if (!end) {
+      cur.raw = rc.raw;
+      cur.mom = rc.mom;
+      cur.slot0 = rc.slot0;
+      cur.N = rc.N;
+      cur.flags = flags;
       mags<PAIR>(&sm.k[stage][0][0], mag_base + (uint32_t)((i % kNB) * 64), r, q);
       tmem_wait_st();
       tc_fence_before();
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.aready[i % kNB]);
-    if (i >= 2 && !epilogue<G>(p, sm, tmem, i - 2, p0, q, rg, lane, msum, msq)) return;
+    if (i >= 2 && !epilogue<G>(p, sm, tmem, i - 2, older, q, rg, lane, msum, msq)) return -1;
     if (end) {
-      if (i >= 1) epilogue<G>(p, sm, tmem, i - 1, p1, q, rg, lane, msum, msq);
-      return;
+      if (i >= 1 && !epilogue<G>(p, sm, tmem, i - 1, other, q, rg, lane, msum, msq)) return -1;
+      return 1;
     }
-    p0 = p1;
-    p1 = rec;
+    older = cur;
+    return 0;
+  };
+  EpRec ra{}, rb{};
+  for (int i = 0;; i += 2) {
+    if (step(i, ra, rb)) return;
+    if (step(i + 1, rb, ra)) return;
   }
 }
 
