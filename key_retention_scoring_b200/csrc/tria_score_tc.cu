@@ -21,7 +21,9 @@
 //   warp 17     one lane issues tcgen05.mma (M=128, N=16|32, K=16): 8 steps
 //               with A = the K tile in shared memory (then the K stage is
 //               released), 8 steps with A = the magnitude tile in tensor
-//               memory, and tcgen05.commit;
+//               memory, and tcgen05.commit.  Consecutive steps accumulate
+//               into NACC different partial accumulators (summed by the
+//               epilogue), so they do not wait on each other's results;
 //   warps 0-15  band magnitudes -> tensor memory (tcgen05.st; warp w takes
 //               rows 32(w%4).. and bands 16(w/4)..), then, kLag tiles later,
 //               the epilogue (tcgen05.ld, raw scores, fp64 moment partials).
@@ -52,8 +54,8 @@ constexpr int kFlagFirst = 1, kFlagLast = 2, kFlagEnd = 4;
 // whose previous user, tile i - kNB, finished its epilogue before the
 // magnitudes of tile i - 1).
 constexpr int kNB = 4;
-constexpr uint32_t kTmemCols = 512;         // [0, kNB*NCOL): accumulators; [128, 384): magnitude tiles
-constexpr uint32_t kTmemMag = 128;
+constexpr uint32_t kTmemCols = 512;         // [0, 256): accumulators; [256, 512): magnitude tiles
+constexpr uint32_t kTmemMag = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint32_t kSuspendNs = 1000000;    // a blocked try_wait sleeps up to 1 ms per call
 
@@ -78,6 +80,8 @@ struct TcCfg {
   static constexpr int STAGES = (G <= 8) ? 6 : 5;
   static constexpr int GQ = (G >= 4) ? G / 4 : 1;          // heads per band quarter
   static constexpr int BBLK = NCOL * 128;                  // bytes per 64-wide K block of B
+  static constexpr int NACC = (NCOL <= 16) ? 4 : 2;        // partial accumulators per tile
+  static_assert(kNB * NACC * NCOL <= 256, "accumulator columns");
 };
 
 template <int G>
@@ -264,9 +268,9 @@ __device__ __forceinline__ void mma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// Load N consecutive 32-bit columns of this thread's lane (no wait).
 template <int N>
-__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[N]) {
-  uint32_t r[N];
+__device__ __forceinline__ void tmem_ld_nowait(uint32_t taddr, uint32_t (&r)[N]) {
   if constexpr (N == 2) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];"
                  : "=r"(r[0]), "=r"(r[1])
@@ -275,68 +279,57 @@ __device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[N]) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                  : "r"(taddr));
-  } else if constexpr (N == 8) {
+  } else {
+    static_assert(N == 8, "tmem_ld_nowait width");
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
                    "=r"(r[6]), "=r"(r[7])
                  : "r"(taddr));
-  } else {
-    static_assert(N == 16, "tmem_ld width");
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-        "%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
   }
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < N; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ uint4 lds128(const uint8_t *p) { return *reinterpret_cast<const uint4 *>(p); }
 
-// Packed fp32 pairs (sm_100 f32x2 arithmetic).
-__device__ __forceinline__ uint64_t pk2(float a, float b) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+// Squared magnitude of a band from its bf16 parts (the low or high halves
+// of re_w / im_w): re^2 (exact in fp32) + im^2 with one rounding.
+template <bool HI>
+__device__ __forceinline__ float band_sq(uint32_t re_w, uint32_t im_w) {
+  float r;
+  if constexpr (HI) {
+    asm("{\n .reg .b16 a, b, c, d;\n mov.b32 {a, b}, %1;\n mov.b32 {c, d}, %2;\n"
+        " fma.rn.f32.bf16 %0, b, b, 0f00000000;\n fma.rn.f32.bf16 %0, d, d, %0;\n}"
+        : "=f"(r) : "r"(re_w), "r"(im_w));
+  } else {
+    asm("{\n .reg .b16 a, b, c, d;\n mov.b32 {a, b}, %1;\n mov.b32 {c, d}, %2;\n"
+        " fma.rn.f32.bf16 %0, a, a, 0f00000000;\n fma.rn.f32.bf16 %0, c, c, %0;\n}"
+        : "=f"(r) : "r"(re_w), "r"(im_w));
+  }
   return r;
 }
-__device__ __forceinline__ void up2(uint64_t v, float &a, float &b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
+
+// Squared magnitude of a band held in one word (re low half, im high half).
+__device__ __forceinline__ float band_sq_word(uint32_t w) {
+  float r;
+  asm("{\n .reg .b16 a, b;\n mov.b32 {a, b}, %1;\n"
+      " fma.rn.f32.bf16 %0, a, a, 0f00000000;\n fma.rn.f32.bf16 %0, b, b, %0;\n}"
+      : "=f"(r) : "r"(w));
+  return r;
 }
 
-// Magnitudes of two bands from their bf16 re/im parts, split into bf16
-// hi + lo parts: hi = the top halves of the fp32 bit patterns (truncation),
-// lo = bf16(x - hi) rounded to nearest.  |x - hi - lo| <= 2^-16 x.
-__device__ __forceinline__ void mag_pair(float ra, float rb, float ia, float ib, uint32_t &hi,
-                                         uint32_t &lo) {
-  const uint64_t sq = fma2(pk2(ia, ib), pk2(ia, ib), mul2(pk2(ra, rb), pk2(ra, rb)));
-  float sa, sb;
-  up2(sq, sa, sb);
+// Magnitudes of two bands from their squared magnitudes, split into bf16
+// hi + lo parts (packed two per word, first band in the low half): hi = the
+// top halves of the fp32 bit patterns (truncation), lo = bf16(x - hi)
+// rounded to nearest.  |x - hi - lo| <= 2^-16 x.
+__device__ __forceinline__ void mag_split(float sa, float sb, uint32_t &hi, uint32_t &lo) {
   const float ma = sqrt_approx(sa), mb = sqrt_approx(sb);
   const uint32_t ua = __float_as_uint(ma), ub = __float_as_uint(mb);
   hi = __byte_perm(ua, ub, 0x7632);
-  const uint64_t res = sub2(pk2(ma, mb), pk2(__uint_as_float(ua & 0xffff0000u),
-                                             __uint_as_float(ub & 0xffff0000u)));
-  float xa, xb;
-  up2(res, xa, xb);
+  const float xa = ma - __uint_as_float(ua & 0xffff0000u);
+  const float xb = mb - __uint_as_float(ub & 0xffff0000u);
   const __nv_bfloat162 l = __floats2bfloat162_rn(xa, xb);
   lo = *reinterpret_cast<const uint32_t *>(&l);
 }
@@ -464,34 +457,41 @@ __device__ void producer(const ScoreParams &p, TcSmem<G> &sm, int n_items, int l
 // ---------------------------------------------------------------------------
 template <int G>
 __device__ void mma_issuer(const ScoreParams &p, TcSmem<G> &sm, uint32_t tmem) {
-  constexpr int ST = TcCfg<G>::STAGES, NCOL = TcCfg<G>::NCOL, BBLK = TcCfg<G>::BBLK;
+  using Cfg = TcCfg<G>;
+  constexpr int ST = Cfg::STAGES, NCOL = Cfg::NCOL, BBLK = Cfg::BBLK, NACC = Cfg::NACC;
   constexpr uint32_t idesc = idesc_bf16_m128<NCOL>();
+  // descriptors of stage 0 / coefficient buffer 0; an operand at byte offset
+  // o from there is the descriptor plus o >> 4 (shared addresses < 256 KB)
+  const uint64_t da0 = sw128_desc(smem_u32(&sm.k[0][0][0]));
+  const uint64_t db0 = sw128_desc(smem_u32(&sm.b[0][0][0]));
+  constexpr uint32_t kStageBytes = 2 * kHalfBlock;
   int i = 0;
   for (;; ++i) {
     if (!mbar_wait(&sm.aready[i % kNB], (i / kNB) & 1, &sm.abort_flag, p.status)) break;
     tc_fence_after();
     const int stage = i % ST, ab = i % kNB;
     const SubRec &rec = sm.rec[stage];
-    if (rec.flags & kFlagEnd) break;
-    const uint32_t d = tmem + (uint32_t)(ab * NCOL);
-    const uint32_t ka = smem_u32(&sm.k[stage][0][0]);
+    const int flags = rec.flags, bpar = rec.bpar;
+    if (flags & kFlagEnd) break;
+    const uint32_t d = tmem + (uint32_t)(ab * NACC * NCOL);
     const uint32_t ta = tmem + kTmemMag + (uint32_t)(ab * 64);
-    const uint32_t bb = smem_u32(&sm.b[rec.bpar][0][0]);
-    const bool last = (rec.flags & kFlagLast) != 0;
-    const int bpar = rec.bpar;
+    const uint64_t da = da0 + (uint64_t)((stage * kStageBytes) >> 4);
+    const uint64_t db = db0 + (uint64_t)((bpar * 4 * BBLK) >> 4);
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
-      const uint32_t a_addr = ka + (s >> 2) * kHalfBlock + (s & 3) * 32;
-      const uint32_t b_addr = bb + (s >> 2) * BBLK + (s & 3) * 32;
-      mma_bf16(d, sw128_desc(a_addr), sw128_desc(b_addr), idesc, s > 0 ? 1u : 0u);
+      const uint32_t ao = (s >> 2) * kHalfBlock + (s & 3) * 32;
+      const uint32_t bo = (s >> 2) * BBLK + (s & 3) * 32;
+      mma_bf16(d + (uint32_t)((s % NACC) * NCOL), da + (ao >> 4), db + (bo >> 4), idesc,
+               s >= NACC ? 1u : 0u);
     }
     mma_commit(&sm.kempty[stage]);  // the K tile is consumed: the producer may refill it
 #pragma unroll
     for (int s = 8; s < 16; ++s) {
-      const uint32_t b_addr = bb + (s >> 2) * BBLK + (s & 3) * 32;
-      mma_bf16_ta(d, ta + (uint32_t)((s - 8) * 8), sw128_desc(b_addr), idesc, 1u);
+      const uint32_t bo = (s >> 2) * BBLK + (s & 3) * 32;
+      mma_bf16_ta(d + (uint32_t)((s % NACC) * NCOL), ta + (uint32_t)((s - 8) * 8), db + (bo >> 4),
+                  idesc, 1u);
     }
-    if (last) mma_commit(&sm.bempty[bpar]);
+    if (flags & kFlagLast) mma_commit(&sm.bempty[bpar]);
     mma_commit(&sm.accfull[ab]);  // issued last: the final wait below covers all
   }
   if (i > 0) mbar_wait(&sm.accfull[(i - 1) % kNB], ((i - 1) / kNB) & 1, &sm.abort_flag, p.status);
@@ -508,6 +508,7 @@ __device__ __forceinline__ void mags(const uint8_t *kt, uint32_t tcol, int r, in
   const int sw = r & 7;
   uint32_t hi[8], lo[8];
   if (PAIR == TRIA_PAIR_NEOX) {
+    // band f: re at dim f, im at dim 64 + f; a word holds bands (2k, 2k + 1)
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       const int cc = 2 * q + j;
@@ -516,16 +517,18 @@ __device__ __forceinline__ void mags(const uint8_t *kt, uint32_t tcol, int r, in
       const uint32_t rw[4] = {re.x, re.y, re.z, re.w}, iw[4] = {im.x, im.y, im.z, im.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        mag_pair(bf_lo(rw[e]), bf_hi(rw[e]), bf_lo(iw[e]), bf_hi(iw[e]), hi[4 * j + e], lo[4 * j + e]);
+        mag_split(band_sq<false>(rw[e], iw[e]), band_sq<true>(rw[e], iw[e]), hi[4 * j + e],
+                  lo[4 * j + e]);
     }
   } else {
+    // band f: re at dim 2f, im at dim 2f + 1; a word holds one band
     const uint8_t *kh = kt + (q >> 1) * kHalfBlock;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int cc = 4 * (q & 1) + j;
       const uint4 x = lds128(kh + r * 128 + ((cc ^ sw) << 4));
-      mag_pair(bf_lo(x.x), bf_lo(x.y), bf_hi(x.x), bf_hi(x.y), hi[2 * j], lo[2 * j]);
-      mag_pair(bf_lo(x.z), bf_lo(x.w), bf_hi(x.z), bf_hi(x.w), hi[2 * j + 1], lo[2 * j + 1]);
+      mag_split(band_sq_word(x.x), band_sq_word(x.y), hi[2 * j], lo[2 * j]);
+      mag_split(band_sq_word(x.z), band_sq_word(x.w), hi[2 * j + 1], lo[2 * j + 1]);
     }
   }
   tmem_st8(tcol + (uint32_t)(8 * q), hi);
@@ -568,8 +571,21 @@ __device__ __forceinline__ bool epilogue(const ScoreParams &p, TcSmem<G> &sm, ui
     for (int g = 0; g < GQ; ++g) msum[g] = msq[g] = 0.0;
   }
   if (active) {
+    // this thread's 2 GQ columns of each partial accumulator, summed in order
+    constexpr int NACC = TcCfg<G>::NACC;
+    uint32_t pa[NACC][2 * GQ];
+    const uint32_t col = tmem + ((uint32_t)(32 * rg) << 16) + (uint32_t)((j % kNB) * NACC * NCOL + q * 2 * GQ);
+#pragma unroll
+    for (int a = 0; a < NACC; ++a) tmem_ld_nowait<2 * GQ>(col + (uint32_t)(a * NCOL), pa[a]);
+    tmem_wait_ld();
     float v[2 * GQ];
-    tmem_ld<2 * GQ>(tmem + ((uint32_t)(32 * rg) << 16) + (uint32_t)((j % kNB) * NCOL + q * 2 * GQ), v);
+#pragma unroll
+    for (int c = 0; c < 2 * GQ; ++c) {
+      float x = __uint_as_float(pa[0][c]);
+#pragma unroll
+      for (int a = 1; a < NACC; ++a) x += __uint_as_float(pa[a][c]);
+      v[c] = x;
+    }
     const int slot = pr.slot0 + rg * 32 + lane;
     if (slot >= geo.sinks && slot < pr.N - geo.window) {
       float sc[GQ];
