@@ -24,11 +24,11 @@
 //               memory, and tcgen05.commit.  Consecutive steps accumulate
 //               into NACC different partial accumulators (summed by the
 //               epilogue), so they do not wait on each other's results;
-//   warps 0-15  band magnitudes -> tensor memory (tcgen05.st; warp w takes
-//               rows 32(w%4).. and bands 16(w/4)..), then, kLag tiles later,
+//   warps 0-7   band magnitudes -> tensor memory (tcgen05.st; warp w takes
+//               rows 32(w%4).. and bands 32(w/4)..), then, two tiles later,
 //               the epilogue (tcgen05.ld, raw scores, fp64 moment partials).
 //               Magnitude tiles and accumulators rotate through kNB
-//               tensor-memory buffers, so kLag MMA chains stay in flight.
+//               tensor-memory buffers, so two MMA chains stay in flight.
 // Normalize-then-max and the selection run in the next kernel (tail_kernel).
 // Every wait is bounded (2 s); on expiry the kernel flags status bit 1, lets
 // its own loads and MMAs land, frees its tensor memory and returns.
@@ -42,10 +42,12 @@ namespace {
 using namespace dev;
 
 constexpr int kRows = 128;                  // keys per MMA tile (M)
-constexpr int kComputeWarps = 16;
-constexpr int kProducerWarp = 16;
-constexpr int kMmaWarp = 17;
-constexpr int kTcThreads = 576;
+constexpr int kBandGroups = 2;              // compute warps per 32-row quadrant of a tile
+constexpr int kBandsPerThread = kBands / kBandGroups;
+constexpr int kComputeWarps = 4 * kBandGroups;
+constexpr int kProducerWarp = kComputeWarps;
+constexpr int kMmaWarp = kComputeWarps + 1;
+constexpr int kTcThreads = 32 * (kComputeWarps + 2);
 constexpr int kHalfBlock = kRows * 128;     // 128 rows x 64 bf16, swizzled
 constexpr int kFlagFirst = 1, kFlagLast = 2, kFlagEnd = 4;
 // The epilogue of tile i runs after the magnitudes of tile i + 2, so two MMA
@@ -78,7 +80,7 @@ template <int G>
 struct TcCfg {
   static constexpr int NCOL = (2 * G < 16) ? 16 : 2 * G;   // MMA N
   static constexpr int STAGES = (G <= 8) ? 6 : 5;
-  static constexpr int GQ = (G >= 4) ? G / 4 : 1;          // heads per band quarter
+  static constexpr int GQ = (G >= kBandGroups) ? G / kBandGroups : 1;  // heads per band group
   static constexpr int BBLK = NCOL * 128;                  // bytes per 64-wide K block of B
   static constexpr int NACC = (NCOL <= 16) ? 4 : 2;        // partial accumulators per tile
   static_assert(kNB * NACC * NCOL <= 256, "accumulator columns");
@@ -246,12 +248,23 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
       : "memory");
 }
 
-// Store 8 consecutive 32-bit columns of this thread's tensor-memory lane.
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-      : "memory");
+// Store N (8 or 16) consecutive 32-bit columns of this thread's tensor-memory lane.
+template <int N>
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&r)[N]) {
+  if constexpr (N == 8) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+        : "memory");
+  } else {
+    static_assert(N == 16, "tmem_st width");
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+        "%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+  }
 }
 
 __device__ __forceinline__ void tmem_wait_st() {
@@ -279,12 +292,20 @@ __device__ __forceinline__ void tmem_ld_nowait(uint32_t taddr, uint32_t (&r)[N])
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                  : "r"(taddr));
-  } else {
-    static_assert(N == 8, "tmem_ld_nowait width");
+  } else if constexpr (N == 8) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
                    "=r"(r[6]), "=r"(r[7])
                  : "r"(taddr));
+  } else {
+    static_assert(N == 16, "tmem_ld_nowait width");
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
   }
 }
 
@@ -500,18 +521,20 @@ __device__ void mma_issuer(const ScoreParams &p, TcSmem<G> &sm, uint32_t tmem) {
 // ---------------------------------------------------------------------------
 // compute warps
 // ---------------------------------------------------------------------------
-// Band magnitudes of row r, bands [16q, 16q + 16), stored to the row's
-// tensor-memory lane: hi parts at columns [8q, 8q + 8), lo parts at
-// [32 + 8q, ...) of the magnitude tile (two bf16 per column, band order).
+// Band magnitudes of row r, bands [B q, B q + B) with B = kBandsPerThread,
+// stored to the row's tensor-memory lane: hi parts at columns
+// [B q / 2, B q / 2 + B / 2), lo parts at 32 + the same (two bf16 per
+// column, band order).
 template <int PAIR>
 __device__ __forceinline__ void mags(const uint8_t *kt, uint32_t tcol, int r, int q) {
+  constexpr int B = kBandsPerThread, W = B / 2;
   const int sw = r & 7;
-  uint32_t hi[8], lo[8];
+  uint32_t hi[W], lo[W];
   if (PAIR == TRIA_PAIR_NEOX) {
     // band f: re at dim f, im at dim 64 + f; a word holds bands (2k, 2k + 1)
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int cc = 2 * q + j;
+    for (int j = 0; j < B / 8; ++j) {
+      const int cc = (B / 8) * q + j;
       const uint4 re = lds128(kt + r * 128 + ((cc ^ sw) << 4));
       const uint4 im = lds128(kt + kHalfBlock + r * 128 + ((cc ^ sw) << 4));
       const uint32_t rw[4] = {re.x, re.y, re.z, re.w}, iw[4] = {im.x, im.y, im.z, im.w};
@@ -521,18 +544,21 @@ __device__ __forceinline__ void mags(const uint8_t *kt, uint32_t tcol, int r, in
                   lo[4 * j + e]);
     }
   } else {
-    // band f: re at dim 2f, im at dim 2f + 1; a word holds one band
-    const uint8_t *kh = kt + (q >> 1) * kHalfBlock;
+    // band f: re at dim 2f, im at dim 2f + 1; a word holds one band; bands
+    // [32 h, 32 h + 32) are the half block h
+    const int f0 = B * q;
+    const uint8_t *kh = kt + (f0 / 32) * kHalfBlock;
+    const int c0 = (f0 % 32) / 4;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int cc = 4 * (q & 1) + j;
+    for (int j = 0; j < B / 4; ++j) {
+      const int cc = c0 + j;
       const uint4 x = lds128(kh + r * 128 + ((cc ^ sw) << 4));
       mag_split(band_sq_word(x.x), band_sq_word(x.y), hi[2 * j], lo[2 * j]);
       mag_split(band_sq_word(x.z), band_sq_word(x.w), hi[2 * j + 1], lo[2 * j + 1]);
     }
   }
-  tmem_st8(tcol + (uint32_t)(8 * q), hi);
-  tmem_st8(tcol + (uint32_t)(32 + 8 * q), lo);
+  tmem_st<W>(tcol + (uint32_t)(W * q), hi);
+  tmem_st<W>(tcol + (uint32_t)(32 + W * q), lo);
 }
 
 // Bounded wait of a whole warp (every lane tests the barrier; the warp
@@ -563,7 +589,7 @@ __device__ __forceinline__ bool epilogue(const ScoreParams &p, TcSmem<G> &sm, ui
                                          double (&msum)[TcCfg<G>::GQ], double (&msq)[TcCfg<G>::GQ]) {
   constexpr int NCOL = TcCfg<G>::NCOL, GQ = TcCfg<G>::GQ;
   const Geom &geo = p.geo;
-  const bool active = (G >= 4) || q < G;  // quarter q scores heads [q GQ, (q + 1) GQ)
+  const bool active = (G >= kBandGroups) || q < G;  // group q scores heads [q GQ, (q + 1) GQ)
   if (!warp_wait(&sm.accfull[j % kNB], (j / kNB) & 1, &sm.abort_flag, p.status, lane)) return false;
   tc_fence_after();
   if (pr.flags & kFlagFirst) {
@@ -596,7 +622,10 @@ __device__ __forceinline__ bool epilogue(const ScoreParams &p, TcSmem<G> &sm, ui
         msq[g] = fma((double)sc[g], (double)sc[g], msq[g]);
       }
       float *dst = pr.raw + (slot - geo.sinks) * G + q * GQ;
-      if constexpr (GQ == 4) {
+      if constexpr (GQ == 8) {
+        reinterpret_cast<float4 *>(dst)[0] = make_float4(sc[0], sc[1], sc[2], sc[3]);
+        reinterpret_cast<float4 *>(dst)[1] = make_float4(sc[4], sc[5], sc[6], sc[7]);
+      } else if constexpr (GQ == 4) {
         *reinterpret_cast<float4 *>(dst) = make_float4(sc[0], sc[1], sc[2], sc[3]);
       } else if constexpr (GQ == 2) {
         *reinterpret_cast<float2 *>(dst) = make_float2(sc[0], sc[1]);
@@ -631,7 +660,7 @@ template <int G, int PAIR>
 __device__ void compute(const ScoreParams &p, TcSmem<G> &sm, uint32_t tmem, int tid) {
   constexpr int ST = TcCfg<G>::STAGES, GQ = TcCfg<G>::GQ;
   const int warp = tid >> 5, lane = tid & 31;
-  const int q = warp >> 2, rg = warp & 3, r = rg * 32 + lane;
+  const int q = warp >> 2, rg = warp & 3, r = rg * 32 + lane;  // band group, quadrant, row
   const uint32_t mag_base = tmem + ((uint32_t)(32 * rg) << 16) + kTmemMag;
   double msum[GQ], msq[GQ];
 #pragma unroll
