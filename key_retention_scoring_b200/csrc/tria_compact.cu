@@ -1,0 +1,217 @@
+// compact_kernel: in-place gather of the kept K/V rows of every unit (and of
+// the K positions), then the sequence lengths and freed paged blocks.
+//
+// The kept list of a unit is ascending with kept[j] >= j, so destination j
+// never lies above its source.  Rows move in chunks of kCpRows destination
+// rows, in ascending order, through a ring of shared-memory chunk buffers
+// filled by cp.async (16 bytes per copy, no registers held while in flight):
+//   * every row of chunk c is read before any row of chunk c is written, as a
+//     destination of chunk c can be the source of another row of chunk c or
+//     of an earlier chunk (one __syncthreads per chunk);
+//   * chunk c + A is read before chunk c is written: its sources are at or
+//     above its first destination, above every destination of chunk c.
+// One block per SM walks the chunks of its items (unit, K or V) as one
+// stream, reading A = 2 chunks ahead of the chunk it writes.  A thread always
+// handles the same rows and 16-byte pieces of a chunk: it loads their kept
+// entries one chunk before it starts their copies, keeps their sources in
+// shared memory for the write-back, and writes back exactly the pieces it
+// read, so the only wait on the path is for copies started two chunks ago.
+#include "tria_device.cuh"
+
+namespace tria {
+namespace {
+
+using namespace dev;
+
+constexpr int kCpThreads = 512;
+constexpr int kCpRows = 256;                              // destination rows per chunk
+constexpr int kCpDepth = 3;                               // chunk buffers
+constexpr int kCpAhead = 2;                               // chunks read ahead
+constexpr int kRowBytes = kHeadDim * 2;                   // 256
+constexpr int kPieces = kRowBytes / 16;                   // 16-byte pieces per row
+constexpr int kRowStep = kCpThreads / kPieces;            // rows covered by one pass of the block
+constexpr int kRowsPerThread = kCpRows / kRowStep;        // 8
+
+struct CpSmem {
+  alignas(16) uint8_t buf[kCpDepth][kCpRows][kRowBytes];
+  int32_t pos[kCpDepth][kCpRows];
+  int32_t src[kCpDepth][kCpRows];   // source of each destination row (-1: stays)
+};
+
+struct ItemGeo {
+  unsigned char *base;  // K or V of the layer
+  int32_t *pos;         // positions of the unit (K items only; may be null)
+  const int32_t *kept;
+  int s, h, ul, part;
+};
+
+__device__ __forceinline__ ItemGeo item_geo(const CompactParams &p, int64_t it) {
+  const Geom &geo = p.geo;
+  ItemGeo g;
+  const int64_t u = it >> 1;
+  g.part = (int)(it & 1);
+  g.s = (int)(u / ((int64_t)geo.nl * geo.hkv));
+  g.ul = (int)(u % ((int64_t)geo.nl * geo.hkv));
+  const int lrel = g.ul / geo.hkv;
+  g.h = g.ul % geo.hkv;
+  g.kept = p.kept + u * geo.budget;
+  g.base = reinterpret_cast<unsigned char *>(g.part == 0 ? const_cast<uint16_t *>(p.cache.k[lrel])
+                                                         : p.cache.v[lrel]);
+  const int64_t pu = ((int64_t)g.s * geo.n_layers + geo.layer0 + lrel) * geo.hkv + g.h;
+  g.pos = (g.part == 0 && p.cache.positions != nullptr)
+              ? p.cache.positions + pu * p.cache.pos_unit_stride
+              : nullptr;
+  return g;
+}
+
+__device__ __forceinline__ void cp16(void *sdst, const void *gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(sdst)),
+               "l"(gsrc)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp4(void *sdst, const void *gsrc) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(sdst)),
+               "l"(gsrc)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Length and freed blocks of sequence s, from the kept list of its unit 0.
+__device__ void update_len(const CompactParams &p, const ItemGeo &g) {
+  const Geom &geo = p.geo;
+  const int s = g.s;
+  const int N = p.cache.seq_lens[s];
+  int newlen = geo.budget;
+  if (g.kept[geo.budget - 1] < 0) {
+    newlen = 0;
+    while (newlen < geo.budget && g.kept[newlen] >= 0) ++newlen;
+  }
+  if (N > geo.budget && N <= geo.max_seq_len) {
+    if (p.cache.layout == TRIA_LAYOUT_PAGED && p.n_freed != nullptr) {
+      const int bs = p.cache.block_size;
+      const int keep_blocks = (newlen + bs - 1) / bs;
+      const int old_blocks = (N + bs - 1) / bs;
+      int nf = 0;
+      for (int b = keep_blocks; b < old_blocks; ++b) {
+        if (p.freed_blocks != nullptr)
+          p.freed_blocks[(int64_t)s * p.cache.max_blocks + nf] =
+              p.cache.block_table[(int64_t)s * p.cache.max_blocks + b];
+        ++nf;
+      }
+      p.n_freed[s] = nf;
+    }
+    p.cache.seq_lens[s] = newlen;
+  } else if (p.cache.layout == TRIA_LAYOUT_PAGED && p.n_freed != nullptr) {
+    p.n_freed[s] = 0;
+  }
+}
+
+__global__ void __launch_bounds__(kCpThreads, 1) compact_kernel(const __grid_constant__ CompactParams p) {
+  extern __shared__ __align__(16) uint8_t smem_cp[];
+  CpSmem &sm = *reinterpret_cast<CpSmem *>(smem_cp);
+  const Geom &geo = p.geo;
+  const int t = threadIdx.x;
+  const int piece = t % kPieces, rr = t / kPieces;
+  const int cap = geo.max_seq_len;
+  const int nch = (geo.budget + kCpRows - 1) / kCpRows;
+  const int64_t n_items = geo.n_units * 2;
+  const int64_t my_items =
+      (blockIdx.x < n_items) ? (n_items - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const int64_t total = my_items * nch;  // chunks of this block, item-major
+
+  // kept entries (raw) of this thread's rows of stream chunk k
+  auto fetch = [&](int64_t k, int (&kv)[kRowsPerThread]) {
+    if (k < total) {
+      const int64_t it = blockIdx.x + (k / nch) * gridDim.x;
+      const int c = (int)(k % nch);
+      const int32_t *kept = p.kept + (it >> 1) * geo.budget;
+#pragma unroll
+      for (int e = 0; e < kRowsPerThread; ++e) {
+        const int j = c * kCpRows + rr + e * kRowStep;
+        kv[e] = (j < geo.budget) ? __ldg(kept + j) : -1;
+      }
+    }
+  };
+  // copies of this thread's pieces of stream chunk k into buffer k % depth
+  // (one commit group per chunk, empty past the end)
+  auto issue = [&](int64_t k, const int (&kv)[kRowsPerThread]) {
+    if (k < total) {
+      const int64_t it = blockIdx.x + (k / nch) * gridDim.x;
+      const int c = (int)(k % nch);
+      const ItemGeo g = item_geo(p, it);
+      const int b = (int)(k % kCpDepth);
+#pragma unroll
+      for (int e = 0; e < kRowsPerThread; ++e) {
+        const int r = rr + e * kRowStep, j = c * kCpRows + r;
+        const int v = kv[e];
+        const int src = (j >= geo.budget || v == j || v < 0 || v >= cap || j >= cap) ? -1 : v;
+        if (piece == 0) sm.src[b][r] = src;
+        if (src >= 0) {
+          cp16(&sm.buf[b][r][piece * 16], g.base + row_off(p.cache, g.s, g.h, src) * 2 + piece * 16);
+          if (g.pos != nullptr && piece == 0) cp4(&sm.pos[b][r], g.pos + src);
+        }
+      }
+    }
+    cp_commit();
+  };
+
+  int kv[kRowsPerThread];
+  for (int k = 0; k < kCpAhead; ++k) {
+    fetch(k, kv);
+    issue(k, kv);
+  }
+  fetch(kCpAhead, kv);
+  for (int64_t k = 0; k < total; ++k) {
+    issue(k + kCpAhead, kv);
+    fetch(k + kCpAhead + 1, kv);  // used at the next iteration
+    cp_wait<kCpAhead>();  // this thread's copies of chunk k have landed
+    __syncthreads();      // ... and every other thread's
+    const int64_t it = blockIdx.x + (k / nch) * gridDim.x;
+    const int c = (int)(k % nch);
+    const ItemGeo g = item_geo(p, it);
+    const int b = (int)(k % kCpDepth);
+#pragma unroll
+    for (int e = 0; e < kRowsPerThread; ++e) {
+      const int r = rr + e * kRowStep, j = c * kCpRows + r;
+      // the row's source, recorded (and now read) by the row's piece-0 thread
+      const int mine = (piece == 0) ? sm.src[b][r] : 0;
+      const int src = __shfl_sync(kFull, mine, (threadIdx.x & 31) & ~(kPieces - 1));
+      if (src >= 0) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(&sm.buf[b][r][piece * 16]);
+        *reinterpret_cast<uint4 *>(g.base + row_off(p.cache, g.s, g.h, j) * 2 + piece * 16) = v;
+        if (g.pos != nullptr && piece == 0) g.pos[j] = sm.pos[b][r];
+      }
+    }
+    // sequence length / freed blocks: once per sequence, after the last layer
+    if (c == nch - 1 && p.update_lens && g.part == 0 && g.ul == 0 && t == 0) update_len(p, g);
+  }
+  cp_wait<0>();
+}
+
+}  // namespace
+
+cudaError_t launch_compact(const CompactParams &p, cudaStream_t st) {
+  const int smem = (int)sizeof(CpSmem);
+  cudaError_t e = cudaFuncSetAttribute(compact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  int64_t grid = p.geo.n_units * 2;
+  if (grid > sms) grid = sms;
+  compact_kernel<<<(unsigned)grid, kCpThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+static_assert(sizeof(CpSmem) <= 232448, "shared memory of the compaction kernel");
+
+}  // namespace tria

@@ -8,7 +8,7 @@
 //   tail_kernel     blocks over (unit, candidate chunk): normalize-then-max,
 //                   histogram of the agg keys, selection by the last block.
 //   select_kernel   one CTA per unit: radix top-K of agg + ascending kept list.
-//   compact_kernel  in-place gather of kept K/V rows (and positions).
+//   (the compaction kernel is in tria_compact.cu)
 //
 // Sources: academ.us article 2607.13051 (Eqs. 2, 3, 4, 6, 7 and sec. 4),
 // ghidav.me "TriAttention, or: what a rotating query already knows" ("The
@@ -270,94 +270,6 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const __grid_constant_
                            kept, ts, sc, false, t);
 }
 
-// ---------------------------------------------------------------------------
-// compact_kernel: items (unit, part) with part 0/1 = K bytes [0,128)/[128,256),
-// part 2/3 = V.  Destination chunks are walked in ascending order; a chunk's
-// sources are all read before any of its rows is written.  Because the kept
-// list is ascending with kept[j] >= j, a chunk never overwrites a row that a
-// later chunk still has to read.
-// ---------------------------------------------------------------------------
-constexpr int kCompactRowsPerChunk = 256;  // 8 threads x 16 B per half row
-
-__global__ void __launch_bounds__(kThreads) compact_kernel(const __grid_constant__ CompactParams p) {
-  const Geom &geo = p.geo;
-  const int t = threadIdx.x;
-  const int sub = t & 7;         // 16-byte piece of the 128-byte half row
-  const int rsub = t >> 3;       // 0..31
-  const int64_t n_items = geo.n_units * 4;
-  for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x) {
-    const int64_t u = it >> 2;
-    const int part = (int)(it & 3);
-    const int s = (int)(u / ((int64_t)geo.nl * geo.hkv));
-    const int ul = (int)(u % ((int64_t)geo.nl * geo.hkv));
-    const int lrel = ul / geo.hkv, h = ul % geo.hkv;
-    const int32_t *kept = p.kept + u * geo.budget;
-    uint16_t *base = (part < 2) ? const_cast<uint16_t *>(p.cache.k[lrel]) : p.cache.v[lrel];
-    const int byte_off = (part & 1) * 128 + sub * 16;
-    // positions are laid out over all layers of the model
-    const int64_t pu = ((int64_t)s * geo.n_layers + geo.layer0 + lrel) * geo.hkv + h;
-    int32_t *pos = (part == 0 && p.cache.positions != nullptr)
-                       ? p.cache.positions + pu * p.cache.pos_unit_stride
-                       : nullptr;
-    for (int j0 = 0; j0 < geo.budget; j0 += kCompactRowsPerChunk) {
-      uint4 vals[kCompactRowsPerChunk / 32];
-      int32_t pv[kCompactRowsPerChunk / 32];
-      int srcs[kCompactRowsPerChunk / 32];
-#pragma unroll
-      for (int r = 0; r < kCompactRowsPerChunk / 32; ++r) {
-        const int j = j0 + r * 32 + rsub;
-        int src = (j < geo.budget) ? kept[j] : -1;
-        // only well-formed moves inside the cache capacity
-        if (src == j || src < 0 || src >= geo.max_seq_len || j >= geo.max_seq_len) src = -1;
-        srcs[r] = src;
-        if (src >= 0) {
-          const uint16_t *row = base + row_off(p.cache, s, h, src);
-          vals[r] = *reinterpret_cast<const uint4 *>(reinterpret_cast<const unsigned char *>(row) + byte_off);
-          if (pos != nullptr && sub == 0) pv[r] = pos[src];
-        }
-      }
-      __syncthreads();
-#pragma unroll
-      for (int r = 0; r < kCompactRowsPerChunk / 32; ++r) {
-        const int j = j0 + r * 32 + rsub;
-        if (srcs[r] >= 0) {
-          uint16_t *row = base + row_off(p.cache, s, h, j);
-          *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(row) + byte_off) = vals[r];
-          if (pos != nullptr && sub == 0) pos[j] = pv[r];
-        }
-      }
-      __syncthreads();
-    }
-    // sequence length / freed blocks: once per sequence, after the last layer
-    if (p.update_lens && part == 0 && ul == 0 && t == 0) {
-      const int N = p.cache.seq_lens[s];
-      int newlen = geo.budget;
-      if (kept[geo.budget - 1] < 0) {
-        newlen = 0;
-        while (newlen < geo.budget && kept[newlen] >= 0) ++newlen;
-      }
-      if (N > geo.budget && N <= geo.max_seq_len) {
-        if (p.cache.layout == TRIA_LAYOUT_PAGED && p.n_freed != nullptr) {
-          const int bs = p.cache.block_size;
-          const int keep_blocks = (newlen + bs - 1) / bs;
-          const int old_blocks = (N + bs - 1) / bs;
-          int nf = 0;
-          for (int b = keep_blocks; b < old_blocks; ++b) {
-            if (p.freed_blocks != nullptr)
-              p.freed_blocks[(int64_t)s * p.cache.max_blocks + nf] =
-                  p.cache.block_table[(int64_t)s * p.cache.max_blocks + b];
-            ++nf;
-          }
-          p.n_freed[s] = nf;
-        }
-        p.cache.seq_lens[s] = newlen;
-      } else if (p.cache.layout == TRIA_LAYOUT_PAGED && p.n_freed != nullptr) {
-        p.n_freed[s] = 0;
-      }
-    }
-  }
-}
-
 }  // namespace
 
 cudaError_t launch_coef(const CoefParams &p, cudaStream_t st) {
@@ -415,15 +327,5 @@ cudaError_t launch_select(const SelectParams &p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_compact(const CompactParams &p, cudaStream_t st) {
-  int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t items = p.geo.n_units * 4;
-  int64_t grid = (int64_t)sms * 8;
-  if (grid > items) grid = items;
-  compact_kernel<<<(unsigned)grid, kThreads, 0, st>>>(p);
-  return cudaGetLastError();
-}
 
 }  // namespace tria
