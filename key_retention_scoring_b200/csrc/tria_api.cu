@@ -260,8 +260,11 @@ TailParams make_tail(const Geom &g, const tria_cache_view *c, void *ws, const Ws
   tp.kept = nullptr;
   tp.hist = at<uint32_t>(ws, wl.hist);
   tp.unit_done = at<uint32_t>(ws, wl.unit_done);
-  tp.discard_raw = 1;
-  tp.discard_agg = 1;
+  // dropping dead scratch lines from L2 saves their write-back only while the
+  // scratch still fits in L2; beyond that they are long written back
+  const bool small = (int64_t)g.n_units * wl.raw_stride * 4 <= (int64_t)48 << 20;
+  tp.discard_raw = small ? 1 : 0;
+  tp.discard_agg = small ? 1 : 0;
   return tp;
 }
 

@@ -470,7 +470,13 @@ __device__ void agg_range(const float *__restrict__ raw, float *agg, int c0, int
 // scores [C][G]; adds the top 12 key bits of every candidate to hist.
 // select_keys: radix top-K over the keys (digits of 12, 12 and 8 bits), then
 // the ascending kept list: sinks, the K candidates above the threshold key T
-// plus the lowest-slot keys equal to T, the window.
+// plus the lowest-slot keys equal to T, the window.  After the first digit
+// (histogram of unit_keys), one pass over the keys counts, per warp range,
+// the keys above the chosen bin, histograms the bin's keys on the second
+// digit and gathers them into a list; the third digit and the per-warp
+// counts of keys above / equal to T inside the bin come from the list.  A bin
+// larger than the list falls back to passes over all keys.  The emission is
+// one more pass.
 // ---------------------------------------------------------------------------
 struct UnitScalars {
   int warp_tmp[32];
@@ -479,6 +485,7 @@ struct UnitScalars {
   int digit;
   int above;
   int bin_count;
+  int list_n;
   int warp_gt[32];
   int warp_eq[32];
   float mean[TRIA_MAX_GROUP];
@@ -490,7 +497,7 @@ template <int G, int NT>
 __device__ void unit_keys(const float *raw, int C, const float *s_mean, const float *s_inv,
                           uint32_t *keys, uint32_t *hist, int tid) {
   const int lane = tid & 31;
-  constexpr int U = 4;  // float4 loads in flight per thread
+  constexpr int U = 8;  // float4 loads in flight per thread
   const float4 *src = reinterpret_cast<const float4 *>(raw);
   if constexpr (G >= 4) {
     // LPC lanes per candidate, each with 4 of its G heads
@@ -574,48 +581,94 @@ __device__ void unit_keys(const float *raw, int C, const float *s_mean, const fl
 
 template <int NT>
 __device__ void select_keys(const uint32_t *keys, int C, int K, int N, int B, int W, int S,
-                            int32_t *kept, uint32_t *hist, UnitScalars &sc, int tid) {
+                            int32_t *kept, uint32_t *hist, uint2 *list, UnitScalars &sc, int tid) {
   const int lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
   for (int j = tid; j < S; j += NT) kept[j] = j;
   for (int j = tid; j < W; j += NT) kept[B - W + j] = N - W + j;
   if (K <= 0) return;
   if (tid == 0) {
     sc.prefix = 0u;
     sc.remaining = K;
+    sc.list_n = 0;
   }
   __syncthreads();
   pick_bin<0, NT>(hist, kHistBins, sc, 20, tid);
-  // digits 2 (bits [19:8]) and 3 (bits [7:0]) over the keys of the chosen bin
-#pragma unroll 1
-  for (int level = 1; level <= 2; ++level) {
-    const int hi_shift = level == 1 ? 20 : 8;
-    const int sh = level == 1 ? 8 : 0;
-    const uint32_t dmask = level == 1 ? 0xfffu : 0xffu;
-    clear_words<NT>(hist, kHistBins, tid);
-    __syncthreads();
-    const uint32_t pre = sc.prefix >> hi_shift;
-    for (int c = tid; c < C; c += NT) {
-      const uint32_t k = keys[c];
-      if ((k >> hi_shift) == pre) atomicAdd(hist + ((k >> sh) & dmask), 1u);
-    }
-    __syncthreads();
-    pick_bin<0, NT>(hist, kHistBins, sc, sh, tid);
-  }
-  const uint32_t T = sc.prefix;
-  const int need = sc.remaining;  // keys equal to T to take, lowest slots first (>= 1)
-  // emission: warp w walks candidates [w * per_w, (w + 1) * per_w) 32 at a time
+  // warp w owns candidates [w R, (w + 1) R), R = 32 steps
   const int steps = (C + NT - 1) / NT;
   const int cb = warp * steps * 32;
-  int gt = 0, eq = 0;
-  for (int e = 0; e < steps; ++e) {
-    const int c = cb + e * 32 + lane;
-    const uint32_t k = (c < C) ? keys[c] : 0u;
-    gt += __popc(__ballot_sync(kFull, c < C && k > T));
-    eq += __popc(__ballot_sync(kFull, c < C && k == T));
+  clear_words<NT>(hist, kHistBins, tid);
+  __syncthreads();
+  const uint32_t d1 = sc.prefix >> 20;
+  {
+    int above = 0;
+    for (int e = 0; e < steps; ++e) {
+      const int c = cb + e * 32 + lane;
+      const bool valid = c < C;
+      const uint32_t k = valid ? keys[c] : 0u;
+      above += __popc(__ballot_sync(kFull, valid && (k >> 20) > d1));
+      const bool in = valid && (k >> 20) == d1;
+      const uint32_t bal = __ballot_sync(kFull, in);
+      if (bal) {
+        int base = 0;
+        if (lane == 0) base = atomicAdd(&sc.list_n, __popc(bal));
+        base = __shfl_sync(kFull, base, 0);
+        if (in) {
+          atomicAdd(hist + ((k >> 8) & 0xfffu), 1u);
+          const int idx = base + __popc(bal & lt);
+          if (idx < kListCap) list[idx] = make_uint2(k, (uint32_t)c);
+        }
+      }
+    }
+    if (lane == 0) {
+      sc.warp_gt[warp] = above;
+      sc.warp_eq[warp] = 0;
+    }
   }
-  if (lane == 0) {
-    sc.warp_gt[warp] = gt;
-    sc.warp_eq[warp] = eq;
+  __syncthreads();
+  pick_bin<0, NT>(hist, kHistBins, sc, 8, tid);
+  const int ln = sc.list_n;
+  const bool use_list = ln <= kListCap;
+  clear_words<NT>(hist, kHistBins, tid);
+  __syncthreads();
+  {
+    const uint32_t d12 = sc.prefix >> 8;
+    if (use_list) {
+      for (int i = tid; i < ln; i += NT) {
+        const uint32_t k = list[i].x;
+        if ((k >> 8) == d12) atomicAdd(hist + (k & 0xffu), 1u);
+      }
+    } else {
+      for (int c = tid; c < C; c += NT) {
+        const uint32_t k = keys[c];
+        if ((k >> 8) == d12) atomicAdd(hist + (k & 0xffu), 1u);
+      }
+    }
+  }
+  __syncthreads();
+  pick_bin<0, NT>(hist, kHistBins, sc, 0, tid);
+  const uint32_t T = sc.prefix;
+  const int need = sc.remaining;  // keys equal to T to take, lowest slots first (>= 1)
+  // per-warp counts of the keys of the first-digit bin above / equal to T
+  if (use_list) {
+    for (int i = tid; i < ln; i += NT) {
+      const uint2 e = list[i];
+      const int w = (int)e.y / (steps * 32);
+      if (e.x > T) atomicAdd(&sc.warp_gt[w], 1);
+      else if (e.x == T) atomicAdd(&sc.warp_eq[w], 1);
+    }
+  } else {
+    int gt = 0, eq = 0;
+    for (int e = 0; e < steps; ++e) {
+      const int c = cb + e * 32 + lane;
+      const uint32_t k = (c < C) ? keys[c] : 0u;
+      gt += __popc(__ballot_sync(kFull, c < C && (k >> 20) == d1 && k > T));
+      eq += __popc(__ballot_sync(kFull, c < C && k == T));
+    }
+    if (lane == 0) {
+      atomicAdd(&sc.warp_gt[warp], gt);
+      atomicAdd(&sc.warp_eq[warp], eq);
+    }
   }
   __syncthreads();
   int gt_before = 0, eq_before = 0;
@@ -623,9 +676,9 @@ __device__ void select_keys(const uint32_t *keys, int C, int K, int N, int B, in
     gt_before += sc.warp_gt[i];
     eq_before += sc.warp_eq[i];
   }
+  // emission in slot order
   int run_keep = gt_before + min(eq_before, need);
   int run_eq = eq_before;
-  const uint32_t lt = (1u << lane) - 1u;
   for (int e = 0; e < steps; ++e) {
     const int c = cb + e * 32 + lane;
     const bool valid = c < C;

@@ -75,7 +75,7 @@ struct WsLayout {
 
 constexpr int kAggHistBins = 4096;
 constexpr int kAggChunk = 4096;   // candidates per block of the normalization kernel
-constexpr int kUnitTailMaxC = 49152;       // candidates per unit of the one-block-per-unit tail
+constexpr int kUnitTailMaxC = 45056;       // candidates per unit of the one-block-per-unit tail
 constexpr size_t kMaxDynSmem = 232448;     // opt-in shared memory per block (227 KB)
 
 WsLayout ws_layout(const Geom &g);

@@ -210,7 +210,8 @@ __global__ void __launch_bounds__(kThreads) tail_kernel(const __grid_constant__ 
 constexpr int kUnitThreads = 1024;
 
 size_t unit_tail_smem_bytes(int c_max) {
-  return sizeof(UnitScalars) + (size_t)kHistBins * 4 + (size_t)((c_max + 3) & ~3) * 4;
+  return sizeof(UnitScalars) + (size_t)kHistBins * 4 + (size_t)kListCap * 8 +
+         (size_t)((c_max + 3) & ~3) * 4;
 }
 
 template <int G>
@@ -218,7 +219,8 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_tail_kernel(const __grid
   extern __shared__ __align__(16) uint8_t smem_ut[];
   UnitScalars &sc = *reinterpret_cast<UnitScalars *>(smem_ut);
   uint32_t *hist = reinterpret_cast<uint32_t *>(smem_ut + sizeof(UnitScalars));
-  uint32_t *keys = hist + kHistBins;
+  uint2 *list = reinterpret_cast<uint2 *>(hist + kHistBins);
+  uint32_t *keys = reinterpret_cast<uint32_t *>(list + kListCap);
   const Geom &geo = p.geo;
   const int t = threadIdx.x;
   const int K = geo.budget - geo.window - geo.sinks;
@@ -241,7 +243,7 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_tail_kernel(const __grid
       for (int64_t i = t; i < lines; i += kUnitThreads) discard_line(raw + i * 32);
     }
     select_keys<kUnitThreads>(keys, C, K, N, geo.budget, geo.window, geo.sinks,
-                              p.kept + u * geo.budget, hist, sc, t);
+                              p.kept + u * geo.budget, hist, list, sc, t);
     __syncthreads();
   }
 }
