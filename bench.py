@@ -383,6 +383,7 @@ def main():
 
     if not args.no_extras:
         line["run16"] = run16(T, w, st, cache, prm, ws, kept, restore)
+        line["calibration"] = calibration(T, torch, hbm)
         line["e2e"] = e2e(T, torch, w, st, cache, prm, ws, kept, restore, args.e2e_steps, keys, world)
         if rank == 0 and world == 1:
             v, n_units, spent = oracle_unit_keys_per_s(cfg, args.cpu_seconds)
@@ -398,6 +399,34 @@ def main():
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def calibration(T, torch, hbm, reps=5):
+    """Calibration reduction (tria_calib_accumulate) of one Qwen3-32B-shape
+    layer: 32768 pre-RoPE query tokens x 64 heads x 128 bf16 = 512 MB, larger
+    than L2, generated on the device (seeded)."""
+    hq, n = 64, 32768
+    g = torch.Generator(device="cuda")
+    g.manual_seed(3)
+    q = (torch.randn((n, hq, 128), generator=g, device="cuda") + 0.5).to(torch.bfloat16)
+    acc = torch.zeros((hq, 64, 3), dtype=torch.float64, device="cuda")
+    desc = T.model_desc(1, hq, 8, T.PAIR_NEOX, 1e4)
+    for _ in range(2):
+        T.tria_calib_accumulate(desc, q, acc)
+    ts = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        T.tria_calib_accumulate(desc, q, acc)
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    ms = statistics.mean(ts)
+    nbytes = n * hq * 128 * 2
+    del q
+    return {"workload": "one layer, 32768 tokens x 64 query heads x 128 (bf16, 512 MB)",
+            "ms": ms, "tokens_per_s": n / (ms * 1e-3), "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
+            "frac": nbytes / (ms * 1e-3) / 1e9 / hbm, "reps": reps}
 
 
 def run16(T, w, st, cache, prm, ws, kept, restore):

@@ -294,6 +294,39 @@ tria_status tria_compress_pass_static(const tria_stats *stats, const tria_cache_
                                       int32_t *device_status, tria_stream_t stream);
 
 /*
+ * tria_calib_accumulate - the calibration reduction that produces the query
+ * statistics tria_load_stats takes (GitHub issue #10 of the llama.cpp
+ * TurboQuant HIP fork, "Working calibration tool": q_mean_real[f] =
+ * E[Re q_f], q_mean_imag[f] = E[Im q_f], q_abs_mean[f] = E[|q_f|] over the
+ * post-norm, pre-RoPE queries, with the model's complex pairing; academ.us
+ * article 2607.13051 sec. 2: E[q_f] is the average of band-f queries over a
+ * calibration set).  One layer per call; batches of one layer add up.
+ *   q    device bf16 pre-RoPE queries of one layer, element (t, h, i) at
+ *        q[t * stride_token + h * stride_head + i], i < 128 contiguous;
+ *        8-byte aligned, strides multiples of 4 elements;
+ *   acc  device fp64 [n_q_heads][64][3] = (sum Re q_f, sum Im q_f,
+ *        sum |q_f|) per (head, band); the caller zeroes it before the first
+ *        batch and keeps it between batches.  The sums are added with fp64
+ *        atomics (the order of additions, so the last bits, may vary).
+ * Reads desc->n_q_heads, head_dim (128) and pairing.  Stream-ordered, no
+ * allocation.  Errors: INVALID_ARG, UNSUPPORTED (head_dim), CUDA.
+ */
+tria_status tria_calib_accumulate(const tria_model_desc *desc, const void *q, int64_t n_tokens,
+                                  int64_t stride_token, int64_t stride_head, double *acc,
+                                  tria_stream_t stream);
+
+/*
+ * tria_calib_finalize - statistics from the sums of tria_calib_accumulate
+ * over n_tokens tokens in total: device fp32 [n_q_heads][64] arrays
+ * q_mean_re = sum Re / n_tokens, q_mean_im = sum Im / n_tokens,
+ * q_abs_mean = sum |q_f| / n_tokens (one layer's slice of the host arrays
+ * tria_load_stats takes).  Errors: INVALID_ARG (n_tokens <= 0), CUDA.
+ */
+tria_status tria_calib_finalize(const tria_model_desc *desc, const double *acc, int64_t n_tokens,
+                                float *q_mean_re, float *q_mean_im, float *q_abs_mean,
+                                tria_stream_t stream);
+
+/*
  * tria_read_device_status - errors the kernels found in device-resident
  * inputs during the calls that used this workspace (bit 0: a seq_lens entry
  * outside [0, max_seq_len]; such a unit is skipped and its kept row is all

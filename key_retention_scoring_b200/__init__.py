@@ -28,7 +28,7 @@ MAX_LAYERS = 128
 EXPORTS = ["tria_status_string", "tria_version", "tria_load_stats", "tria_free_stats",
            "tria_stats_desc", "tria_workspace_size", "tria_score", "tria_select", "tria_compact",
            "tria_compress_pass", "tria_read_device_status", "tria_set_pass_events",
-           "tria_compress_pass_static"]
+           "tria_compress_pass_static", "tria_calib_accumulate", "tria_calib_finalize"]
 STATIC_SCRATCH_BYTES = 32 * 1024 * 1024   # TRIA_STATIC_SCRATCH_BYTES
 
 
@@ -96,6 +96,10 @@ def lib() -> ctypes.CDLL:
     L.tria_set_pass_events.argtypes = [ctypes.POINTER(_VP)]
     L.tria_compress_pass_static.argtypes = [_VP, ctypes.POINTER(CacheView),
                                             ctypes.POINTER(Params), _VP, _VP, _VP, _VP, _VP]
+    L.tria_calib_accumulate.argtypes = [ctypes.POINTER(ModelDesc), _VP, ctypes.c_int64,
+                                        ctypes.c_int64, ctypes.c_int64, _VP, _VP]
+    L.tria_calib_finalize.argtypes = [ctypes.POINTER(ModelDesc), _VP, ctypes.c_int64, _VP, _VP,
+                                      _VP, _VP]
     for name in EXPORTS:
         if name not in ("tria_status_string", "tria_version"):
             getattr(L, name).restype = _I
@@ -263,6 +267,27 @@ def tria_compress_pass_static(stats, cache, prm, kept_idx=None, freed_blocks=Non
                             f"the static scratch holds {STATIC_SCRATCH_BYTES}; use "
                             f"tria_compress_pass with a workspace")
     _check(rc, "tria_compress_pass_static")
+
+
+def tria_calib_accumulate(desc, q, acc, stream=None):
+    """Add one batch of pre-RoPE queries q (bf16 tensor [tokens, n_q_heads,
+    128], any token/head strides, unit stride inside a head) to the fp64 sums
+    acc [n_q_heads, 64, 3] (zeroed by the caller before the first batch)."""
+    import torch
+
+    if q.dtype != torch.bfloat16 or q.dim() != 3 or q.stride(2) != 1:
+        raise TriaError(1, "tria_calib_accumulate: q must be bf16 [tokens, heads, 128] "
+                           "with unit stride inside a head")
+    _check(lib().tria_calib_accumulate(ctypes.byref(desc), _ptr(q), q.shape[0], q.stride(0),
+                                       q.stride(1), _ptr(acc), _stream(stream)),
+           "tria_calib_accumulate")
+
+
+def tria_calib_finalize(desc, acc, n_tokens, q_mean_re, q_mean_im, q_abs_mean, stream=None):
+    """E[Re q_f], E[Im q_f], E|q_f| (fp32 [n_q_heads, 64] outputs) from the sums."""
+    _check(lib().tria_calib_finalize(ctypes.byref(desc), _ptr(acc), int(n_tokens), _ptr(q_mean_re),
+                                     _ptr(q_mean_im), _ptr(q_abs_mean), _stream(stream)),
+           "tria_calib_finalize")
 
 
 def tria_read_device_status(workspace, stream=None) -> int:

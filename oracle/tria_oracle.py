@@ -317,6 +317,19 @@ def score_l1_scale(k_post, positions, q_center, q_abs_mean, omega, pairing,
     return np.stack(out)
 
 
+def calibration_stats(q_pre: np.ndarray, pairing: int):
+    """Query statistics of the calibration step, from pre-RoPE queries
+    q_pre [tokens..., Hq, d] (every axis before the head axis is averaged
+    over): per (head, band) E[Re q_f], E[Im q_f] and E|q_f| ([P4]
+    calibration-tool comment: q_mean_real, q_mean_imag and q_abs_mean over
+    the post-norm, pre-RoPE queries, with the model's complex pairing; [P5]
+    sec. 2: E[q_f] is the average of band-f queries over a calibration set).
+    Returns three [Hq, d/2] float64 arrays."""
+    z = to_bands(q_pre, pairing)
+    z = z.reshape((-1,) + z.shape[-2:])
+    return z.real.mean(axis=0), z.imag.mean(axis=0), np.abs(z).mean(axis=0)
+
+
 def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
     """Exact value of bfloat16 numbers given as their uint16 bit patterns."""
     b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16

@@ -106,6 +106,21 @@ def make_stats(cfg: Config):
     return re.astype(np.float32), im.astype(np.float32), am.astype(np.float32)
 
 
+def calib_queries(n_tokens: int, n_q_heads: int, seed: int, layer: int = 0,
+                  center_sigma: float = 1.0, noise_sigma: float = 0.7) -> np.ndarray:
+    """Synthetic pre-RoPE calibration queries of one layer as bf16 bits
+    [n_tokens][n_q_heads][128]: a per-(layer, head) center ~ N(0, sigma_c^2)
+    per dimension plus per-token noise N(0, sigma_n^2) (concentrated bands,
+    as calibrated queries are)."""
+    h, j4 = np.meshgrid(np.arange(n_q_heads), np.arange(32), indexing="ij")
+    c = np.stack(P.normals4(j4, h, layer, P.STREAM_QCAL_CENTER, seed), axis=-1)
+    c = c.reshape(n_q_heads, 128) * center_sigma
+    t, h2, j4b = np.meshgrid(np.arange(n_tokens), np.arange(n_q_heads), np.arange(32), indexing="ij")
+    nz = np.stack(P.normals4(j4b, h2, t + (layer << 24), P.STREAM_QCAL_NOISE, seed), axis=-1)
+    q = c[None] + nz.reshape(n_tokens, n_q_heads, 128) * noise_sigma
+    return P.f32_to_bf16_bits(q.astype(np.float32))
+
+
 def near_zero_heads(cfg: Config) -> np.ndarray:
     """Boolean [L][Hkv]: the (layer, KV head) pairs with near-zero centers."""
     L, Hk = cfg.n_layers, cfg.n_kv_heads

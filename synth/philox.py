@@ -25,6 +25,8 @@ STREAM_V = 5
 STREAM_HEADPICK = 6
 STREAM_LENGTHS = 7
 STREAM_BLOCKS = 8
+STREAM_QCAL_CENTER = 9
+STREAM_QCAL_NOISE = 10
 
 
 def philox4x32_10(c0, c1, c2, c3, k0, k1=KEY_TAG):

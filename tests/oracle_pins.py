@@ -365,6 +365,42 @@ def pin_p4_candidate_count():
         raise AssertionError("candidate count other than n_kv - window accepted")
 
 
+def pin_calibration_golden():
+    """Two hand-worked tokens, both pairings (tests/golden/calib_two_tokens_d4.txt)."""
+    g = _golden_kv("calib_two_tokens_d4.txt")
+    toks = np.array([[float(t) for t in row.split()] for row in g["tokens"].split(";")])
+    q = toks[:, None, :]  # [2 tokens][1 head][4]
+    for pairing, tag in ((O.PAIR_NEOX, "neox"), (O.PAIR_INTERLEAVED, "inter")):
+        re, im, ab = O.calibration_stats(q, pairing)
+        for got, key in ((re, "re"), (im, "im"), (ab, "abs")):
+            want = np.array([float(t) for t in g[f"{tag}_{key}"].split()])
+            assert np.allclose(got[0], want, rtol=0, atol=1e-12), (tag, key, got[0], want)
+
+
+def pin_calibration_invariants():
+    """E|q_f| >= |E q_f| (triangle inequality); token order does not matter;
+    constant queries give their own bands; means scale with the queries."""
+    rng = np.random.default_rng(11)
+    q = rng.normal(size=(50, 3, 16)) + rng.normal(size=(1, 3, 16))
+    for pairing in (O.PAIR_NEOX, O.PAIR_INTERLEAVED):
+        re, im, ab = O.calibration_stats(q, pairing)
+        assert np.all(ab + 1e-12 >= np.hypot(re, im))
+        re2, im2, ab2 = O.calibration_stats(q[rng.permutation(50)], pairing)
+        assert np.allclose(re, re2) and np.allclose(im, im2) and np.allclose(ab, ab2)
+        re3, im3, ab3 = O.calibration_stats(-2.5 * q, pairing)
+        assert np.allclose(re3, -2.5 * re) and np.allclose(im3, -2.5 * im)
+        assert np.allclose(ab3, 2.5 * ab)
+        one = np.repeat(q[:1], 7, axis=0)
+        z = O.to_bands(q[0], pairing)
+        re4, im4, ab4 = O.calibration_stats(one, pairing)
+        assert np.allclose(re4, z.real) and np.allclose(im4, z.imag)
+        assert np.allclose(ab4, np.abs(z))
+        # strongly concentrated queries: E|q| and |E q| nearly agree (R -> 1)
+        tight = q[:1] + 1e-6 * rng.normal(size=(50, 3, 16))
+        re5, im5, ab5 = O.calibration_stats(tight, pairing)
+        assert np.allclose(ab5, np.hypot(re5, im5), rtol=1e-5)
+
+
 def pin_compaction():
     rng = np.random.default_rng(23)
     rows = rng.integers(0, 2 ** 16, size=(20, 4), dtype=np.uint16)

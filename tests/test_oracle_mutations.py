@@ -133,6 +133,21 @@ def _compact_off_by_one(rows, kept):
     return np.asarray(rows)[np.minimum(np.asarray(kept) + 1, len(rows) - 1)]
 
 
+def _calib_abs_of_mean(q_pre, pairing):
+    z = O.to_bands(q_pre, pairing).reshape((-1,) + O.to_bands(q_pre, pairing).shape[-2:])
+    return z.real.mean(axis=0), z.imag.mean(axis=0), np.abs(z.mean(axis=0))
+
+
+def _calib_sum_not_mean(q_pre, pairing):
+    z = O.to_bands(q_pre, pairing).reshape((-1,) + O.to_bands(q_pre, pairing).shape[-2:])
+    return z.real.sum(axis=0), z.imag.sum(axis=0), np.abs(z).sum(axis=0)
+
+
+def _calib_re_im_swapped(q_pre, pairing):
+    re, im, ab = _orig["calibration_stats"](q_pre, pairing)
+    return im, re, ab
+
+
 _orig = {name: getattr(O, name) for name in dir(O) if callable(getattr(O, name))}
 
 MUTATIONS = {
@@ -159,6 +174,9 @@ MUTATIONS = {
     "keeps the lowest scores": ("rank_order", _rank_ascending),
     "window not forced in": ("select_kept", _select_no_window),
     "compaction off by one": ("compact_rows", _compact_off_by_one),
+    "calibration |E q| for E|q|": ("calibration_stats", _calib_abs_of_mean),
+    "calibration sums not means": ("calibration_stats", _calib_sum_not_mean),
+    "calibration Re and Im swapped": ("calibration_stats", _calib_re_im_swapped),
 }
 
 
