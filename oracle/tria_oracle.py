@@ -142,6 +142,21 @@ def s_trig_direct_average(q_center: np.ndarray, k_pre: np.ndarray, omega: np.nda
     return np.mean(np.sum(table, axis=-1), axis=-1)
 
 
+def s_trig_direct_max(q_center: np.ndarray, k_pre: np.ndarray, omega: np.ndarray,
+                      delta, offsets: np.ndarray) -> np.ndarray:
+    """The non-default variant named at the end of [P5] sec. 4: the maximum of
+    Eq. (2) over the future offsets delta in D instead of their mean.  It is
+    not linear in the phasors, so it does not fold (Eqs. 6-7 do not apply);
+    it is evaluated offset by offset on the same [keys x offsets x bands]
+    table as :func:`s_trig_direct_average`."""
+    mag = np.abs(q_center) * np.abs(k_pre)
+    phi = np.angle(q_center) - np.angle(k_pre)
+    d = np.asarray(delta, dtype=np.float64)[..., None, None]
+    ang = omega * (d + offsets[:, None]) + phi[..., None, :]
+    table = mag[..., None, :] * np.cos(ang)
+    return np.max(np.sum(table, axis=-1), axis=-1)
+
+
 def offset_weight(omega: np.ndarray, offsets: np.ndarray) -> np.ndarray:
     """W_f = (1/|D|) sum_{delta in D} e^{i omega_f delta} ([P5] Eq. 6)."""
     return np.mean(np.exp(1j * np.outer(offsets, omega)), axis=0)
@@ -206,7 +221,9 @@ def unit_scores(k_post: np.ndarray, positions: np.ndarray, p_q: int,
 
     k_post: [N, d] post-RoPE keys; positions: [N] token positions p_k;
     q_center: [G, F] complex E[q_f]; q_abs_mean: [G, F] E|q_f|.
-    form: "folded" (Eq. 7) or "direct" (Eq. 4, the 17-offset table).
+    form: "folded" (Eq. 7), "direct" (Eq. 4, the 17-offset table) or "max"
+    (the maximum over the offsets instead of the mean, see
+    :func:`s_trig_direct_max`).
     Returns [G, N] float64."""
     kb = to_bands(k_post, pairing)
     k_pre = derotate(kb, positions, omega)
@@ -218,13 +235,13 @@ def unit_scores(k_post: np.ndarray, positions: np.ndarray, p_q: int,
     for h in range(G):
         if form == "folded":
             trig = s_trig_folded(folded_center(q_center[h], W, band_mask), k_pre, omega, delta)
-        elif form == "direct":
+        elif form in ("direct", "max"):
             qc = q_center[h] if band_mask is None else q_center[h] * np.asarray(band_mask)
+            fn = s_trig_direct_average if form == "direct" else s_trig_direct_max
             trig = np.empty(k_pre.shape[0])
             step = 4096
             for s in range(0, k_pre.shape[0], step):
-                trig[s:s + step] = s_trig_direct_average(qc, k_pre[s:s + step], omega,
-                                                         delta[s:s + step], D)
+                trig[s:s + step] = fn(qc, k_pre[s:s + step], omega, delta[s:s + step], D)
         else:
             raise ValueError(form)
         out[h] = trig + s_norm(q_center[h], q_abs_mean[h], k_pre)
@@ -301,17 +318,21 @@ def compress_unit(k_post, positions, p_q, q_center, q_abs_mean, omega, pairing,
 # Helpers used by the parity tests
 # ----------------------------------------------------------------------------
 def score_l1_scale(k_post, positions, q_center, q_abs_mean, omega, pairing,
-                   log2_max=16, band_mask=None) -> np.ndarray:
+                   log2_max=16, band_mask=None, form="folded") -> np.ndarray:
     """Sum of the absolute sizes of the terms of the score of every key,
-    sum_f (|mu'_f| + E|q_f| - |E q_f|) |k_f|, per head: [G, N].  Used to
-    scale the score tolerance (a plain relative error is meaningless where the
-    score crosses zero)."""
+    sum_f (|mu'_f| + E|q_f| - |E q_f|) |k_f|, per head: [G, N] (with
+    form="max", |E q_f| (masked) in place of |mu'_f|: the terms of one
+    offset).  Used to scale the score tolerance (a plain relative error is
+    meaningless where the score crosses zero)."""
     kb = to_bands(k_post, pairing)
     k_abs = np.abs(kb)
     W = offset_weight(omega, offset_set(log2_max))
     out = []
     for h in range(q_center.shape[0]):
-        mu = folded_center(q_center[h], W, band_mask)
+        if form == "max":
+            mu = q_center[h] if band_mask is None else q_center[h] * np.asarray(band_mask)
+        else:
+            mu = folded_center(q_center[h], W, band_mask)
         w = np.asarray(q_abs_mean[h]) - np.abs(q_center[h])
         out.append(np.sum((np.abs(mu) + w) * k_abs, axis=-1))
     return np.stack(out)

@@ -170,6 +170,32 @@ def pin_brute_force_rope():
                     assert abs(got_d[h, i] - ref) < 1e-9 * scale, (pairing, theta, h, i, got_d[h, i], ref)
 
 
+def pin_offset_max_brute_force():
+    """The max-over-offsets variant equals the largest textbook RoPE logit of
+    the query center rotated at p_q + delta, delta in D, with the cached key;
+    it bounds the offset average from above, and with D = {1} all forms agree
+    with the single distance Delta + 1."""
+    rng = np.random.default_rng(23)
+    for pairing in (O.PAIR_NEOX, O.PAIR_INTERLEAVED):
+        for theta, m in ((1e4, 16), (5e5, 5)):
+            d, G, N = 16, 2, 10
+            qc, _, k_pre, k_post, pos, p_q = _random_unit(rng, d, G, N, pairing, theta)
+            omega = O.band_frequencies(d, theta)
+            got = O.unit_scores(k_post, pos, p_q, qc, np.abs(qc), omega, pairing, m, form="max")
+            avg = O.unit_scores(k_post, pos, p_q, qc, np.abs(qc), omega, pairing, m, form="direct")
+            for h in range(G):
+                qv = _vec_from_pairs(qc[h].real, qc[h].imag, pairing)
+                for i in range(N):
+                    vals = [float(np.dot(_rope_rotate(qv, p_q + dl, theta, pairing), k_post[i]))
+                            for dl in _offsets_by_hand(m)]
+                    scale = np.sum(np.abs(qv)) * np.sum(np.abs(k_post[i]))
+                    assert abs(got[h, i] - max(vals)) < 1e-9 * scale, (pairing, theta, h, i)
+                    assert got[h, i] >= avg[h, i] - 1e-9 * scale
+            one_max = O.unit_scores(k_post, pos, p_q, qc, np.abs(qc), omega, pairing, 0, form="max")
+            one_avg = O.unit_scores(k_post, pos, p_q, qc, np.abs(qc), omega, pairing, 0, form="folded")
+            assert np.allclose(one_max, one_avg, atol=1e-9)
+
+
 def pin_single_distance_brute_force():
     """Eq. 2 and Eq. 3 at one distance equal the plain RoPE dot product."""
     rng = np.random.default_rng(5)

@@ -148,6 +148,18 @@ def _calib_re_im_swapped(q_pre, pairing):
     return im, re, ab
 
 
+def _max_is_mean(q_center, k_pre, omega, delta, offsets):
+    return _orig["s_trig_direct_average"](q_center, k_pre, omega, delta, offsets)
+
+
+def _max_is_min(q_center, k_pre, omega, delta, offsets):
+    mag = np.abs(q_center) * np.abs(k_pre)
+    phi = np.angle(q_center) - np.angle(k_pre)
+    d = np.asarray(delta, dtype=np.float64)[..., None, None]
+    ang = omega * (d + offsets[:, None]) + phi[..., None, :]
+    return np.min(np.sum(mag[..., None, :] * np.cos(ang), axis=-1), axis=-1)
+
+
 _orig = {name: getattr(O, name) for name in dir(O) if callable(getattr(O, name))}
 
 MUTATIONS = {
@@ -177,6 +189,8 @@ MUTATIONS = {
     "calibration |E q| for E|q|": ("calibration_stats", _calib_abs_of_mean),
     "calibration sums not means": ("calibration_stats", _calib_sum_not_mean),
     "calibration Re and Im swapped": ("calibration_stats", _calib_re_im_swapped),
+    "offset max taken as the mean": ("s_trig_direct_max", _max_is_mean),
+    "offset max taken as the min": ("s_trig_direct_max", _max_is_min),
 }
 
 
