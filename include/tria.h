@@ -132,11 +132,22 @@ typedef struct {
                                 post-RoPE key already carries its position.          */
 } tria_cache_view;
 
+/* How the trigonometric term combines the future offsets delta in D. */
+typedef enum {
+  TRIA_OFFSET_MEAN = 0, /* the mean over D (academ.us article 2607.13051 Eq. 4), the
+                           published default; computed folded (Eq. 7)               */
+  TRIA_OFFSET_MAX = 1   /* the maximum over D instead (the non-default variant named
+                           at the end of sec. 4 of the same article); not foldable:
+                           |D| scores per head per key.  Needs |D| <= 17 and
+                           G * |D| <= 136 (G <= 8 at |D| = 17), else UNSUPPORTED    */
+} tria_offset_reduce;
+
 /* Retention parameters (one set for all units of a call). */
 typedef struct {
   int budget;  /* B: rows kept per unit, window and sinks included; >= window + sinks */
   int window;  /* W: the newest W slots are always kept                               */
   int sinks;   /* S: the oldest S slots are always kept                               */
+  int offset_reduce;  /* tria_offset_reduce; 0 (mean) when zero-initialised           */
 } tria_params;
 
 /* Human-readable name of a status code (static string). */

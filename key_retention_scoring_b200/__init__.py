@@ -23,6 +23,8 @@ PAIR_NEOX = 0
 PAIR_INTERLEAVED = 1
 LAYOUT_CONTIGUOUS = 0
 LAYOUT_PAGED = 1
+OFFSET_MEAN = 0
+OFFSET_MAX = 1
 MAX_LAYERS = 128
 
 EXPORTS = ["tria_status_string", "tria_version", "tria_load_stats", "tria_free_stats",
@@ -58,7 +60,8 @@ class CacheView(ctypes.Structure):
 
 
 class Params(ctypes.Structure):
-    _fields_ = [("budget", ctypes.c_int), ("window", ctypes.c_int), ("sinks", ctypes.c_int)]
+    _fields_ = [("budget", ctypes.c_int), ("window", ctypes.c_int), ("sinks", ctypes.c_int),
+                ("offset_reduce", ctypes.c_int)]
 
 
 _lib = None
@@ -209,8 +212,9 @@ class Cache:
                    num_blocks=getattr(w, "n_blocks", 0), positions=w.positions)
 
 
-def params(budget, window, sinks) -> Params:
-    return Params(budget, window, sinks)
+def params(budget, window, sinks, offset_reduce=0) -> Params:
+    """offset_reduce: OFFSET_MEAN (the published average over D) or OFFSET_MAX."""
+    return Params(budget, window, sinks, offset_reduce)
 
 
 def tria_workspace_size(stats: Stats, cache: Cache, prm: Params, layer0=0, layer1=None) -> int:

@@ -92,6 +92,17 @@ tria_status make_geom(const tria_stats *stats, const tria_cache_view *cache,
   g.pairing = d.pairing;
   g.ncol = (2 * g.g < 16) ? 16 : 2 * g.g;
   g.n_units = (int64_t)g.n_seq * g.nl * g.hkv;
+  g.mode = params->offset_reduce;
+  if (g.mode != TRIA_OFFSET_MEAN && g.mode != TRIA_OFFSET_MAX) return TRIA_ERR_INVALID_ARG;
+  g.n_off = d.offset_log2_max + 1;
+  g.ncol_t = ((2 * g.n_off * g.g + 15) / 16) * 16;
+  g.ncol_n = g.ncol;
+  if (g.mode == TRIA_OFFSET_MAX) {
+    if (g.n_off > 17 || 2 * g.n_off * g.g > kMaxOffCols) return TRIA_ERR_UNSUPPORTED;
+    g.b_bytes = (g.ncol_t + g.ncol_n) * 256;  // two 64-wide K blocks of 128-byte rows each
+  } else {
+    g.b_bytes = g.ncol * kCoefK * 2;
+  }
   if (g.n_units * (int64_t)g.tiles_max > INT32_MAX) return TRIA_ERR_UNSUPPORTED;
   *geo = g;
   return TRIA_OK;
@@ -214,6 +225,7 @@ CoefParams make_coef(const tria_stats *st, const Geom &g, const tria_cache_view 
   CoefParams cp{};
   cp.geo = g;
   cp.mu_fold = st->dev.mu_fold;
+  cp.mu_raw = st->dev.mu_raw;
   cp.w_norm = st->dev.w_norm;
   cp.omega = st->dev.omega;
   cp.query_pos = c->query_pos;
@@ -283,7 +295,7 @@ WsLayout ws_layout(const Geom &g) {
   w.hdr = take(256);
   w.unit_done = take((size_t)g.n_units * 4);
   w.seq_items = take((size_t)(g.n_seq + 1) * 4);
-  w.btile = take((size_t)g.n_units * g.ncol * kCoefK * 2);
+  w.btile = take((size_t)g.n_units * g.b_bytes);
   w.moments = take((size_t)g.n_units * g.tiles_max * kRowGroups * g.g * 2 * 8);
   w.hist = take((size_t)g.n_units * kAggHistBins * 4);
   w.raw = take((size_t)g.n_units * w.raw_stride * 4);
@@ -348,7 +360,7 @@ tria_status tria_load_stats(const tria_model_desc *desc, const float *q_mean_re,
     wre[f] = sr / nd;
     wim[f] = si / nd;
   }
-  std::vector<double2> mu(n);
+  std::vector<double2> mu(n), mu_raw(n);
   std::vector<double> wn(n);
   for (size_t i = 0; i < n; ++i) {
     const int f = (int)(i % F);
@@ -361,6 +373,8 @@ tria_status tria_load_stats(const tria_model_desc *desc, const float *q_mean_re,
     }
     mu[i].x = (re * wre[f] - im * wim[f]) * m;
     mu[i].y = (re * wim[f] + im * wre[f]) * m;
+    mu_raw[i].x = re * m;
+    mu_raw[i].y = im * m;
     wn[i] = am - std::hypot(re, im);
   }
 
@@ -369,9 +383,11 @@ tria_status tria_load_stats(const tria_model_desc *desc, const float *q_mean_re,
   st->dev.desc = d;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMalloc(&st->dev.mu_fold, n * sizeof(double2)) != cudaSuccess ||
+      cudaMalloc(&st->dev.mu_raw, n * sizeof(double2)) != cudaSuccess ||
       cudaMalloc(&st->dev.w_norm, n * sizeof(double)) != cudaSuccess ||
       cudaMalloc(&st->dev.omega, F * sizeof(double)) != cudaSuccess) {
     cudaFree(st->dev.mu_fold);
+    cudaFree(st->dev.mu_raw);
     cudaFree(st->dev.w_norm);
     cudaFree(st->dev.omega);
     delete st;
@@ -380,6 +396,8 @@ tria_status tria_load_stats(const tria_model_desc *desc, const float *q_mean_re,
   }
   cudaError_t e = cudaMemcpyAsync(st->dev.mu_fold, mu.data(), n * sizeof(double2),
                                   cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(st->dev.mu_raw, mu_raw.data(), n * sizeof(double2), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(st->dev.w_norm, wn.data(), n * sizeof(double), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess)
@@ -397,6 +415,7 @@ tria_status tria_free_stats(tria_stats *st) {
   if (st == nullptr) return TRIA_OK;
   cudaError_t e = cudaDeviceSynchronize();
   cudaFree(st->dev.mu_fold);
+  cudaFree(st->dev.mu_raw);
   cudaFree(st->dev.w_norm);
   cudaFree(st->dev.omega);
   delete st;

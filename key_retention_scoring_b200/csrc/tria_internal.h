@@ -22,6 +22,7 @@ constexpr int kMaxSeqTable = TRIA_MAX_SEQS + 1;
 struct StatsDev {
   tria_model_desc desc;
   double2 *mu_fold;   // [L][Hq][F]  mu'_f = E[q_f] W_f mask_f   (complex, fp64)
+  double2 *mu_raw;    // [L][Hq][F]  E[q_f] mask_f (unfolded: the max-over-offsets form)
   double *w_norm;     // [L][Hq][F]  E|q_f| - |E q_f|            (fp64)
   double *omega;      // [F]         theta^(-2f/d)               (fp64)
 };
@@ -40,6 +41,11 @@ struct Geom {
   int tiles_max; // upper bound of the scheduling tiles of one unit
   int pairing;
   int64_t n_units;  // n_seq * nl * hkv
+  int mode;      // TRIA_OFFSET_MEAN / TRIA_OFFSET_MAX
+  int n_off;     // |D| = offset_log2_max + 1
+  int ncol_t;    // max mode: trig operand rows, 2 |D| G rounded up to 16
+  int ncol_n;    // max mode: norm operand rows, max(16, 2G)
+  int b_bytes;   // bytes of one unit's coefficient image
 };
 
 // Cache addressing (pointers indexed by layer - layer0).
@@ -80,6 +86,9 @@ constexpr size_t kMaxDynSmem = 232448;     // opt-in shared memory per block (22
 
 WsLayout ws_layout(const Geom &g);
 
+// Max-over-offsets mode: columns of the trig accumulator and B-image rows.
+constexpr int kMaxOffCols = 272;   // 2 |D| G <= 272 (|D| G <= 136)
+
 // Score-kernel parameters.
 struct ScoreParams {
   CUtensorMap kmap[TRIA_MAX_LAYERS];  // K of each layer in [layer0, layer1): 128B-swizzled boxes
@@ -114,6 +123,7 @@ struct TailParams {
 struct CoefParams {
   Geom geo;
   const double2 *mu_fold;
+  const double2 *mu_raw;
   const double *w_norm;
   const double *omega;
   const int64_t *query_pos;

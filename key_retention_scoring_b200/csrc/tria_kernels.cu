@@ -95,6 +95,70 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
   }
   if (bad || N <= g.budget) return;
 
+  if (g.mode == TRIA_OFFSET_MAX) {
+    // max over the offsets: one coefficient vector per (head, offset delta_j)
+    // with the unfolded center, c_gfj = E[q_gf] mask_f e^{i omega_f (p_q + delta_j)}
+    __shared__ double2 rotj[kBands][17];
+    const int nd = g.n_off;
+    for (int i = t; i < kBands * nd; i += kThreads) {
+      const int f = i / nd, j = i % nd;
+      double sn, cs;
+      sincos(p.omega[f] * ((double)p.query_pos[s] + (double)(1ll << j)), &sn, &cs);
+      rotj[f][j] = make_double2(cs, sn);
+    }
+    __syncthreads();
+    unsigned char *dst = reinterpret_cast<unsigned char *>(p.btile) + u * (int64_t)g.b_bytes;
+    // trig rows n = 2 (gg nd + j) + part over the 128 key dims (two 64-wide blocks)
+    for (int i = t; i < g.ncol_t * 16; i += kThreads) {
+      const int n = i >> 4, ch = i & 15, kb = ch >> 3, c8 = ch & 7;
+      const int col = n >> 1, part = n & 1, gg = col / nd, j = col % nd;
+      uint32_t w[4];
+      for (int e = 0; e < 8; e += 2) {
+        uint16_t b2[2];
+        for (int q2 = 0; q2 < 2; ++q2) {
+          const int k = ch * 8 + e + q2;  // key dim
+          float x = 0.0f;
+          if (gg < g.g) {
+            const int f = (g.pairing == TRIA_PAIR_NEOX) ? (k & 63) : (k >> 1);
+            const bool im = (g.pairing == TRIA_PAIR_NEOX) ? (k >= 64) : (k & 1);
+            const double2 mu = p.mu_raw[((int64_t)l * g.hq + h * g.g + gg) * kBands + f];
+            const double2 r = rotj[f][j];
+            x = im ? (float)(mu.x * r.y + mu.y * r.x) : (float)(mu.x * r.x - mu.y * r.y);
+          }
+          const uint16_t hi = bf16_rn_bits(x);
+          const uint16_t lo = bf16_rn_bits(x - __uint_as_float((uint32_t)hi << 16));
+          b2[q2] = (part == 0) ? hi : lo;
+        }
+        w[e >> 1] = (uint32_t)b2[0] | ((uint32_t)b2[1] << 16);
+      }
+      *reinterpret_cast<uint4 *>(dst + kb * (g.ncol_t * 128) + n * 128 + ((c8 ^ (n & 7)) << 4)) =
+          make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    // norm rows n = 2 gg + part over the magnitude dims: block 0 multiplies
+    // |k_f| hi (w_f split hi/lo over the rows), block 1 |k_f| lo (w_f hi, 0)
+    unsigned char *dn = dst + 2 * g.ncol_t * 128;
+    for (int i = t; i < g.ncol_n * 16; i += kThreads) {
+      const int n = i >> 4, ch = i & 15, kb = ch >> 3, c8 = ch & 7;
+      const int gg = n >> 1, part = n & 1;
+      uint32_t w[4];
+      for (int e = 0; e < 8; e += 2) {
+        uint16_t b2[2];
+        for (int q2 = 0; q2 < 2; ++q2) {
+          const int f = (ch & 7) * 8 + e + q2;
+          float x = 0.0f;
+          if (gg < g.g) x = (float)p.w_norm[((int64_t)l * g.hq + h * g.g + gg) * kBands + f];
+          const uint16_t hi = bf16_rn_bits(x);
+          const uint16_t lo = bf16_rn_bits(x - __uint_as_float((uint32_t)hi << 16));
+          b2[q2] = (kb == 0) ? (part == 0 ? hi : lo) : (part == 0 ? hi : (uint16_t)0);
+        }
+        w[e >> 1] = (uint32_t)b2[0] | ((uint32_t)b2[1] << 16);
+      }
+      *reinterpret_cast<uint4 *>(dn + kb * (g.ncol_n * 128) + n * 128 + ((c8 ^ (n & 7)) << 4)) =
+          make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    return;
+  }
+
   if (t < kBands) {
     double sn, cs;
     sincos(p.omega[t] * (double)p.query_pos[s], &sn, &cs);
@@ -111,7 +175,7 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
     cf[gg][2 * kBands + f] = (float)p.w_norm[qi];
   }
   __syncthreads();
-  unsigned char *dst = reinterpret_cast<unsigned char *>(p.btile + u * g.ncol * kCoefK);
+  unsigned char *dst = reinterpret_cast<unsigned char *>(p.btile) + u * (int64_t)g.b_bytes;
   for (int i = t; i < g.ncol * (kCoefK / 8); i += kThreads) {
     const int n = i / (kCoefK / 8), ch = i % (kCoefK / 8), k0 = ch * 8;
     const int gg = n >> 1, part = n & 1;

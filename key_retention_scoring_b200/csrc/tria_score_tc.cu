@@ -100,6 +100,7 @@ struct TcSmem {
   int seq_len[kMaxSeqTable];
   uint32_t tmem_base;
   volatile int abort_flag;
+  __device__ __forceinline__ uint8_t *bbuf(int i) { return &b[i][0][0]; }
 };
 
 // ---------------------------------------------------------------------------
@@ -358,10 +359,9 @@ __device__ __forceinline__ void mag_split(float sa, float sb, uint32_t &hi, uint
 // ---------------------------------------------------------------------------
 // producer warp
 // ---------------------------------------------------------------------------
-template <int G, int LAYOUT>
-__device__ void producer(const ScoreParams &p, TcSmem<G> &sm, int n_items, int lane) {
-  constexpr int ST = TcCfg<G>::STAGES, NCOL = TcCfg<G>::NCOL;
-  constexpr uint32_t kBBytes = NCOL * kCoefK * 2;
+template <int ST, int LAYOUT, class Smem>
+__device__ void producer(const ScoreParams &p, Smem &sm, int n_items, int lane) {
+  const uint32_t kBBytes = (uint32_t)p.geo.b_bytes;  // one unit's coefficient image
   const Geom &geo = p.geo;
   const uint64_t pol = evict_first_policy();
   const int units_per_seq = geo.nl * geo.hkv;
@@ -433,12 +433,13 @@ __device__ void producer(const ScoreParams &p, TcSmem<G> &sm, int n_items, int l
       SubRec &r = sm.rec[stage];
       r.u = u; r.s = s; r.lrel = lrel; r.h = h; r.tile = tile; r.N = N; r.slot0 = slot0;
       r.raw = p.raw + u * p.raw_stride;
-      r.mom = p.moments + (u * geo.tiles_max + tile) * kRowGroups * G * 2;
+      r.mom = p.moments + (u * geo.tiles_max + tile) * kRowGroups * geo.g * 2;
       r.flags = (first ? kFlagFirst : 0) | (sub == sub_end - 1 ? kFlagLast : 0);
       r.bpar = bpar;
       mbar_arrive_expect_tx(&sm.full[stage], bytes);
       if (first)
-        bulk_load(smem_u32(&sm.b[bpar][0][0]), p.btile + u * NCOL * kCoefK, kBBytes, &sm.full[stage]);
+        bulk_load(smem_u32(sm.bbuf(bpar)), reinterpret_cast<const uint8_t *>(p.btile) + u * kBBytes,
+                  kBBytes, &sm.full[stage]);
     }
     const CUtensorMap *map = &p.kmap[lrel];
     if (LAYOUT == TRIA_LAYOUT_CONTIGUOUS) {
@@ -526,10 +527,11 @@ __device__ void mma_issuer(const ScoreParams &p, TcSmem<G> &sm, uint32_t tmem) {
 // [B q / 2, B q / 2 + B / 2), lo parts at 32 + the same (two bf16 per
 // column, band order).
 template <int PAIR>
-__device__ __forceinline__ void mags(const uint8_t *kt, uint32_t tcol, int r, int q) {
-  constexpr int B = kBandsPerThread, W = B / 2;
+__device__ __forceinline__ void mags_regs(const uint8_t *kt, int r, int q,
+                                          uint32_t (&hi)[kBandsPerThread / 2],
+                                          uint32_t (&lo)[kBandsPerThread / 2]) {
+  constexpr int B = kBandsPerThread;
   const int sw = r & 7;
-  uint32_t hi[W], lo[W];
   if (PAIR == TRIA_PAIR_NEOX) {
     // band f: re at dim f, im at dim 64 + f; a word holds bands (2k, 2k + 1)
 #pragma unroll
@@ -557,6 +559,13 @@ __device__ __forceinline__ void mags(const uint8_t *kt, uint32_t tcol, int r, in
       mag_split(band_sq_word(x.z), band_sq_word(x.w), hi[2 * j + 1], lo[2 * j + 1]);
     }
   }
+}
+
+template <int PAIR>
+__device__ __forceinline__ void mags(const uint8_t *kt, uint32_t tcol, int r, int q) {
+  constexpr int W = kBandsPerThread / 2;
+  uint32_t hi[W], lo[W];
+  mags_regs<PAIR>(kt, r, q, hi, lo);
   tmem_st<W>(tcol + (uint32_t)(W * q), hi);
   tmem_st<W>(tcol + (uint32_t)(32 + W * q), lo);
 }
@@ -736,7 +745,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) score_tc_kernel(const __grid_co
   if (warp < kComputeWarps) {
     compute<G, PAIR>(p, sm, tmem, tid);
   } else if (warp == kProducerWarp) {
-    producer<G, LAYOUT>(p, sm, n_items, lane);
+    producer<Cfg::STAGES, LAYOUT>(p, sm, n_items, lane);
   } else if (warp == kMmaWarp) {
     if (lane == 0) mma_issuer<G>(p, sm, tmem);
     __syncwarp();
@@ -748,6 +757,299 @@ __global__ void __launch_bounds__(kTcThreads, 1) score_tc_kernel(const __grid_co
     tmem_dealloc(tmem, kTmemCols);
   }
 }
+
+// ---------------------------------------------------------------------------
+// Max-over-offsets mode (tria_params.offset_reduce = TRIA_OFFSET_MAX).
+//
+// S_g(k) = max_j S_trig,g(k, Delta + delta_j) + S_norm,g(k): per tile two
+// contractions, [k] (128 x 128) . Btrig (128 x 2 |D| G) into the trig
+// accumulator (column pair (hi, lo) per (head, offset); one or two MMAs per
+// K-step, N <= 256 each) and [m_hi | m_lo] . Bnorm (128 x 2G) into the norm
+// accumulator, then a max over the offset pairs in the epilogue.  Tensor
+// memory holds one buffer of each (trig 0..271, norm 288.., magnitudes
+// 320..383), so a tile's epilogue runs before the next tile's MMAs; the
+// compute warps hide it behind the next tile's magnitude math (computed into
+// registers first, stored to tensor memory after the epilogue).
+// ---------------------------------------------------------------------------
+constexpr uint32_t kMaxNormCol = 288, kMaxMagCol = 320;
+
+template <int G>
+struct MaxCfg {
+  static constexpr int NN = (2 * G < 16) ? 16 : 2 * G;                  // norm columns
+  static constexpr int NT_MAX = ((2 * 17 * G + 15) / 16) * 16;          // trig columns at |D| = 17
+  static constexpr int STAGES = (G >= 8) ? 2 : 4;
+  static constexpr int BMAX = (NT_MAX + NN) * 256;                       // coefficient image bytes
+  static constexpr int GQ = (G >= kBandGroups) ? G / kBandGroups : 1;
+};
+
+template <int G>
+struct MaxSmem {
+  alignas(1024) uint8_t k[MaxCfg<G>::STAGES][2][kHalfBlock];
+  alignas(1024) uint8_t b[2][MaxCfg<G>::BMAX];
+  alignas(8) uint64_t full[MaxCfg<G>::STAGES];
+  alignas(8) uint64_t kempty[MaxCfg<G>::STAGES];
+  alignas(8) uint64_t aready;
+  alignas(8) uint64_t accfull;
+  alignas(8) uint64_t bempty[2];
+  SubRec rec[MaxCfg<G>::STAGES];
+  alignas(16) int seq_items[kMaxSeqTable];
+  int seq_len[kMaxSeqTable];
+  uint32_t tmem_base;
+  volatile int abort_flag;
+  __device__ __forceinline__ uint8_t *bbuf(int i) { return &b[i][0]; }
+};
+
+__host__ __device__ constexpr uint32_t idesc_bf16_m128_n(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(kRows >> 4) << 24);
+}
+
+template <int G>
+__device__ void mma_issuer_max(const ScoreParams &p, MaxSmem<G> &sm, uint32_t tmem) {
+  using Cfg = MaxCfg<G>;
+  constexpr int ST = Cfg::STAGES, NN = Cfg::NN;
+  const int NT = p.geo.ncol_t;
+  const int N1 = NT < 256 ? NT : 256, N2 = NT - N1;
+  const uint32_t id1 = idesc_bf16_m128_n(N1), id2 = idesc_bf16_m128_n(N2 > 0 ? N2 : 16);
+  constexpr uint32_t idn = idesc_bf16_m128_n(NN);
+  const uint64_t da0 = sw128_desc(smem_u32(&sm.k[0][0][0]));
+  const uint64_t db0 = sw128_desc(smem_u32(&sm.b[0][0]));
+  constexpr uint32_t kStageBytes = 2 * kHalfBlock;
+  const uint32_t nbase = 2u * NT * 128u;  // norm image after the trig image
+  int i = 0;
+  for (;; ++i) {
+    if (!mbar_wait(&sm.aready, i & 1, &sm.abort_flag, p.status)) break;
+    tc_fence_after();
+    const int stage = i % ST;
+    const SubRec &rec = sm.rec[stage];
+    const int flags = rec.flags, bpar = rec.bpar;
+    if (flags & kFlagEnd) break;
+    const uint64_t da = da0 + (uint64_t)((stage * kStageBytes) >> 4);
+    const uint64_t db = db0 + (uint64_t)(((uint32_t)bpar * (uint32_t)Cfg::BMAX) >> 4);
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const uint32_t ao = (s >> 2) * kHalfBlock + (s & 3) * 32;
+      const uint32_t bo = (uint32_t)(s >> 2) * (uint32_t)NT * 128u + (s & 3) * 32;
+      mma_bf16(tmem, da + (ao >> 4), db + (bo >> 4), id1, s > 0 ? 1u : 0u);
+      if (N2 > 0)
+        mma_bf16(tmem + (uint32_t)N1, da + (ao >> 4), db + ((bo + (uint32_t)N1 * 128u) >> 4), id2,
+                 s > 0 ? 1u : 0u);
+    }
+    mma_commit(&sm.kempty[stage]);  // the K tile is consumed
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const uint32_t bo = nbase + (uint32_t)(s >> 2) * NN * 128u + (s & 3) * 32;
+      mma_bf16_ta(tmem + kMaxNormCol, tmem + kMaxMagCol + (uint32_t)(s * 8), db + (bo >> 4), idn,
+                  s > 0 ? 1u : 0u);
+    }
+    if (flags & kFlagLast) mma_commit(&sm.bempty[bpar]);
+    mma_commit(&sm.accfull);
+  }
+  if (i > 0) mbar_wait(&sm.accfull, (i - 1) & 1, &sm.abort_flag, p.status);
+}
+
+// Raw scores, fp64 moment sums and the item's moment partials of one tile
+// (shared by the max-mode epilogue).
+template <int G>
+__device__ __forceinline__ void emit_scores(const ScoreParams &p, const EpRec &pr,
+                                            const float (&sc)[TcCfg<G>::GQ], bool active, int q,
+                                            int rg, int lane, double (&msum)[TcCfg<G>::GQ],
+                                            double (&msq)[TcCfg<G>::GQ]) {
+  constexpr int GQ = TcCfg<G>::GQ;
+  const Geom &geo = p.geo;
+  if (pr.flags & kFlagFirst) {
+#pragma unroll
+    for (int g = 0; g < GQ; ++g) msum[g] = msq[g] = 0.0;
+  }
+  if (active) {
+    const int slot = pr.slot0 + rg * 32 + lane;
+    if (slot >= geo.sinks && slot < pr.N - geo.window) {
+#pragma unroll
+      for (int g = 0; g < GQ; ++g) {
+        msum[g] += (double)sc[g];
+        msq[g] = fma((double)sc[g], (double)sc[g], msq[g]);
+      }
+      float *dst = pr.raw + (slot - geo.sinks) * G + q * GQ;
+#pragma unroll
+      for (int g = 0; g < GQ; ++g) dst[g] = sc[g];
+    }
+  }
+  if ((pr.flags & kFlagLast) && active) {
+#pragma unroll
+    for (int g = 0; g < GQ; ++g) {
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) {
+        msum[g] += __shfl_xor_sync(kFull, msum[g], o);
+        msq[g] += __shfl_xor_sync(kFull, msq[g], o);
+      }
+    }
+    if (lane == 0) {
+      double *m = pr.mom + (rg * G + q * GQ) * 2;
+#pragma unroll
+      for (int g = 0; g < GQ; ++g) {
+        m[2 * g] = msum[g];
+        m[2 * g + 1] = msq[g];
+      }
+    }
+  }
+}
+
+// Epilogue of the previous tile in max mode: per head of this thread's band
+// group, S = max_j (hi_j + lo_j) + (norm hi + norm lo).
+template <int G>
+__device__ __forceinline__ void epilogue_max(const ScoreParams &p, uint32_t tmem, const EpRec &pr,
+                                             int q, int rg, int lane, double (&msum)[TcCfg<G>::GQ],
+                                             double (&msq)[TcCfg<G>::GQ]) {
+  constexpr int GQ = TcCfg<G>::GQ;
+  const bool active = (G >= kBandGroups) || q < G;
+  const int nd = p.geo.n_off;
+  float sc[GQ];
+  if (active) {
+    const uint32_t lb = tmem + ((uint32_t)(32 * rg) << 16);
+#pragma unroll
+    for (int gi = 0; gi < GQ; ++gi) {
+      const int g = q * GQ + gi;
+      uint32_t t[17][2], nv[2];
+#pragma unroll
+      for (int j = 0; j < 17; ++j)
+        if (j < nd) tmem_ld_nowait<2>(lb + (uint32_t)((g * nd + j) * 2), t[j]);
+      tmem_ld_nowait<2>(lb + kMaxNormCol + (uint32_t)(2 * g), nv);
+      tmem_wait_ld();
+      float m = __uint_as_float(t[0][0]) + __uint_as_float(t[0][1]);
+#pragma unroll
+      for (int j = 1; j < 17; ++j) {
+        if (j < nd) {
+          const float v = __uint_as_float(t[j][0]) + __uint_as_float(t[j][1]);
+          m = (m != m) ? m : ((v != v || v > m) ? v : m);  // NaN propagates
+        }
+      }
+      sc[gi] = m + (__uint_as_float(nv[0]) + __uint_as_float(nv[1]));
+    }
+  } else {
+#pragma unroll
+    for (int gi = 0; gi < GQ; ++gi) sc[gi] = 0.0f;
+  }
+  tc_fence_before();
+  emit_scores<G>(p, pr, sc, active, q, rg, lane, msum, msq);
+}
+
+template <int G, int PAIR>
+__device__ void compute_max(const ScoreParams &p, MaxSmem<G> &sm, uint32_t tmem, int tid) {
+  constexpr int ST = MaxCfg<G>::STAGES, GQ = TcCfg<G>::GQ, W = kBandsPerThread / 2;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int q = warp >> 2, rg = warp & 3, r = rg * 32 + lane;
+  const uint32_t mag = tmem + ((uint32_t)(32 * rg) << 16) + kMaxMagCol;
+  double msum[GQ], msq[GQ];
+#pragma unroll
+  for (int g = 0; g < GQ; ++g) msum[g] = msq[g] = 0.0;
+  EpRec prev{};
+  for (int i = 0;; ++i) {
+    const int stage = i % ST;
+    if (!warp_wait(&sm.full[stage], (i / ST) & 1, &sm.abort_flag, p.status, lane)) return;
+    const SubRec &rc = sm.rec[stage];
+    const int flags = rc.flags;
+    const bool end = (flags & kFlagEnd) != 0;
+    EpRec cur{};
+    uint32_t hi[W], lo[W];
+    if (!end) {
+      cur.raw = rc.raw;
+      cur.mom = rc.mom;
+      cur.slot0 = rc.slot0;
+      cur.N = rc.N;
+      cur.flags = flags;
+      mags_regs<PAIR>(&sm.k[stage][0][0], r, q, hi, lo);
+    }
+    if (i >= 1) {
+      // the previous tile's MMAs are done: its scores, and its magnitude
+      // buffer may be overwritten
+      if (!warp_wait(&sm.accfull, (i - 1) & 1, &sm.abort_flag, p.status, lane)) return;
+      tc_fence_after();
+      epilogue_max<G>(p, tmem, prev, q, rg, lane, msum, msq);
+    }
+    if (!end) {
+      tmem_st<W>(mag + (uint32_t)(W * q), hi);
+      tmem_st<W>(mag + (uint32_t)(32 + W * q), lo);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.aready);
+    if (end) return;
+    prev = cur;
+  }
+}
+
+template <int G, int PAIR, int LAYOUT>
+__global__ void __launch_bounds__(kTcThreads, 1) score_max_kernel(const __grid_constant__ ScoreParams p) {
+  using Cfg = MaxCfg<G>;
+  extern __shared__ uint8_t smem_dyn[];
+  MaxSmem<G> &sm = *reinterpret_cast<MaxSmem<G> *>(
+      (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
+  const Geom &geo = p.geo;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  for (int i = tid; i <= geo.n_seq; i += kTcThreads) sm.seq_items[i] = p.seq_items[i];
+  for (int i = tid; i < geo.n_seq; i += kTcThreads) sm.seq_len[i] = p.cache.seq_lens[i];
+  if (tid == 0) {
+    for (int i = 0; i < Cfg::STAGES; ++i) {
+      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.kempty[i], 1);
+    }
+    mbar_init(&sm.aready, kComputeWarps);
+    mbar_init(&sm.accfull, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&sm.bempty[i], 1);
+    sm.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == kMmaWarp) tmem_alloc(&sm.tmem_base, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const int n_items = sm.seq_items[geo.n_seq];
+
+  if (warp < kComputeWarps) {
+    compute_max<G, PAIR>(p, sm, tmem, tid);
+  } else if (warp == kProducerWarp) {
+    producer<Cfg::STAGES, LAYOUT>(p, sm, n_items, lane);
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) mma_issuer_max<G>(p, sm, tmem);
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int G, int PAIR, int LAYOUT>
+cudaError_t launch_max_t(const ScoreParams &p, cudaStream_t st) {
+  auto kern = score_max_kernel<G, PAIR, LAYOUT>;
+  const int smem = (int)sizeof(MaxSmem<G>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  kern<<<sms, kTcThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int G>
+cudaError_t launch_max_g(const ScoreParams &p, cudaStream_t st) {
+  const bool paged = p.cache.layout == TRIA_LAYOUT_PAGED;
+  if (p.geo.pairing == TRIA_PAIR_NEOX)
+    return paged ? launch_max_t<G, TRIA_PAIR_NEOX, TRIA_LAYOUT_PAGED>(p, st)
+                 : launch_max_t<G, TRIA_PAIR_NEOX, TRIA_LAYOUT_CONTIGUOUS>(p, st);
+  return paged ? launch_max_t<G, TRIA_PAIR_INTERLEAVED, TRIA_LAYOUT_PAGED>(p, st)
+               : launch_max_t<G, TRIA_PAIR_INTERLEAVED, TRIA_LAYOUT_CONTIGUOUS>(p, st);
+}
+
+static_assert(sizeof(MaxSmem<8>) + 1024 <= 232448, "shared memory of the G=8 max-mode kernel");
+static_assert(sizeof(MaxSmem<4>) + 1024 <= 232448, "shared memory of the G=4 max-mode kernel");
+static_assert(MaxCfg<8>::NT_MAX <= 288 - 16, "max-mode trig columns");
 
 template <int G, int PAIR, int LAYOUT>
 cudaError_t launch_t(const ScoreParams &p, cudaStream_t st) {
@@ -778,6 +1080,15 @@ static_assert(sizeof(TcSmem<16>) + 1024 <= 232448, "shared memory of the G=16 ke
 }  // namespace
 
 cudaError_t launch_score(const ScoreParams &p, cudaStream_t st) {
+  if (p.geo.mode == TRIA_OFFSET_MAX) {
+    switch (p.geo.g) {
+      case 1: return launch_max_g<1>(p, st);
+      case 2: return launch_max_g<2>(p, st);
+      case 4: return launch_max_g<4>(p, st);
+      case 8: return launch_max_g<8>(p, st);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (p.geo.g) {
     case 1: return launch_g<1>(p, st);
     case 2: return launch_g<2>(p, st);

@@ -40,7 +40,8 @@ def unit_oracle(w, s: int, layer: int, h: int, k_bits=None, positions=None, form
                           cfg.sinks, cfg.offset_log2_max, form=form)
     N = len(k)
     if res["scores"] is not None:
-        l1 = O.score_l1_scale(k, positions, qc, qa, omega, cfg.pairing, cfg.offset_log2_max)
+        l1 = O.score_l1_scale(k, positions, qc, qa, omega, cfg.pairing, cfg.offset_log2_max,
+                              form="max" if form == "max" else "folded")
         res["l1"] = l1[:, cfg.sinks:N - cfg.window]
     res["N"] = N
     return res

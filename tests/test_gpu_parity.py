@@ -34,11 +34,11 @@ def load_stats(w):
     return T.tria_load_stats(desc, *w.stats)
 
 
-def score_layers(w, st, layer0, layer1, want_scores=True):
+def score_layers(w, st, layer0, layer1, want_scores=True, offset_reduce=0):
     """tria_score + tria_select over [layer0, layer1); host copies."""
     cfg = w.cfg
     cache = T.Cache.from_workload(w)
-    prm = T.params(cfg.budget, cfg.window, cfg.sinks)
+    prm = T.params(cfg.budget, cfg.window, cfg.sinks, offset_reduce)
     ws = T.alloc_workspace(T.tria_workspace_size(st, cache, prm, layer0, layer1))
     T.tria_read_device_status(ws)
     nl = layer1 - layer0
@@ -55,10 +55,10 @@ def score_layers(w, st, layer0, layer1, want_scores=True):
     return (agg.cpu().numpy(), None if sc is None else sc.cpu().numpy(), kept.cpu().numpy())
 
 
-def compress(w, st):
+def compress(w, st, offset_reduce=0):
     cfg = w.cfg
     cache = T.Cache.from_workload(w)
-    prm = T.params(cfg.budget, cfg.window, cfg.sinks)
+    prm = T.params(cfg.budget, cfg.window, cfg.sinks, offset_reduce)
     ws = T.alloc_workspace(T.tria_workspace_size(st, cache, prm))
     T.tria_read_device_status(ws)
     kept = torch.full((cfg.n_seq, cfg.n_layers, cfg.n_kv_heads, cfg.budget), -7, dtype=torch.int32,
@@ -78,7 +78,7 @@ def all_units(cfg):
             for h in range(cfg.n_kv_heads)]
 
 
-def full_check(cfg, units=None, score_layers_sel=None, direct_form=False):
+def full_check(cfg, units=None, score_layers_sel=None, direct_form=False, offset_reduce=0):
     """Score/select parity on `units` (default: all), then the fused pass:
     same kept set, compacted bytes, lengths, positions, freed blocks."""
     w = synth.Workload(cfg)
@@ -92,12 +92,13 @@ def full_check(cfg, units=None, score_layers_sel=None, direct_form=False):
         layers = sorted({l for (_, l, _) in units}) if score_layers_sel is None else score_layers_sel
         sel_kept = {}
         for l in layers:
-            agg, sc, kept = score_layers(w, st, l, l + 1)
+            agg, sc, kept = score_layers(w, st, l, l + 1, offset_reduce=offset_reduce)
             for (s, ll, h) in units:
                 if ll != l:
                     continue
                 kb, _, pos = saved[(s, l, h)]
-                ora = PH.unit_oracle(w, s, l, h, k_bits=kb, positions=pos)
+                ora = PH.unit_oracle(w, s, l, h, k_bits=kb, positions=pos,
+                                     form="max" if offset_reduce else "folded")
                 N = ora["N"]
                 where = f"{cfg.name} s{s} l{l} h{h} N{N}"
                 if ora["scores"] is not None:
@@ -113,7 +114,7 @@ def full_check(cfg, units=None, score_layers_sel=None, direct_form=False):
                 PH.check_kept_vs_oracle(kept[s, 0, h], ora, cfg, where)
                 sel_kept[(s, l, h)] = kept[s, 0, h].copy()
         lens_before = w.lens.copy()
-        kept_all, freed, n_freed = compress(w, st)
+        kept_all, freed, n_freed = compress(w, st, offset_reduce)
         # the fused pass keeps exactly what score + select keep
         for key, k in sel_kept.items():
             s, l, h = key
@@ -384,3 +385,47 @@ def test_full_size_llama3_batched_paged():
     if free < need:
         pytest.skip(f"needs ~{need / 1e9:.0f} GB free, {free / 1e9:.0f} GB available")
     full_check(cfg, units=_sample_units(cfg, 4, 3))
+
+
+# ---------------------------------------------------------------------------
+# max-over-offsets mode (tria_params.offset_reduce = TRIA_OFFSET_MAX)
+# ---------------------------------------------------------------------------
+def test_offset_max_pr1_tiny():
+    full_check(synth.CONFIGS[0], offset_reduce=T.OFFSET_MAX)
+
+
+def test_offset_max_qwen3_32b_shape_small():
+    cfg = synth.CONFIGS[2].scaled(n_layers=2, seq_len=4096)
+    units = [(0, l, h) for l in range(2) for h in (0, 3, 7)]
+    full_check(cfg, units=units, offset_reduce=T.OFFSET_MAX)
+
+
+def test_offset_max_paged_interleaved_sinks():
+    cfg = synth.CONFIGS[3].scaled(n_layers=1, n_seq=3, len_range=(3000, 9000))
+    units = [(s, 0, h) for s in range(3) for h in (0, 5)]
+    full_check(cfg, units=units, offset_reduce=T.OFFSET_MAX)
+
+
+def test_offset_max_eight_offsets():
+    cfg = synth.CONFIGS[2].scaled(n_layers=1, seq_len=3000, offset_log2_max=7)
+    units = [(0, 0, h) for h in (1, 6)]
+    full_check(cfg, units=units, offset_reduce=T.OFFSET_MAX)
+
+
+def test_offset_max_unsupported_shapes():
+    cfg = synth.CONFIGS[0].scaled(n_q_heads=32, n_kv_heads=2)  # G = 16
+    w = synth.Workload(cfg, with_values=False, with_positions=False)
+    st = load_stats(w)
+    try:
+        cache = T.Cache.from_workload(w)
+        prm = T.params(cfg.budget, cfg.window, cfg.sinks, T.OFFSET_MAX)
+        with pytest.raises(T.TriaError) as ei:
+            T.tria_workspace_size(st, cache, prm)
+        assert ei.value.status == 2
+        # the mean mode of the same shape is fine
+        T.tria_workspace_size(st, cache, T.params(cfg.budget, cfg.window, cfg.sinks))
+        with pytest.raises(T.TriaError) as ei:
+            T.tria_workspace_size(st, cache, T.params(cfg.budget, cfg.window, cfg.sinks, 7))
+        assert ei.value.status == 1
+    finally:
+        st.free()
