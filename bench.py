@@ -384,6 +384,7 @@ def main():
     if not args.no_extras:
         line["run16"] = run16(T, w, st, cache, prm, ws, kept, restore)
         line["calibration"] = calibration(T, torch, hbm)
+        line["offset_max"] = offset_max(T, torch, st, cache, cfg, kept, restore, hbm)
         line["e2e"] = e2e(T, torch, w, st, cache, prm, ws, kept, restore, args.e2e_steps, keys, world)
         if rank == 0 and world == 1:
             v, n_units, spent = oracle_unit_keys_per_s(cfg, args.cpu_seconds)
@@ -427,6 +428,42 @@ def calibration(T, torch, hbm, reps=5):
     return {"workload": "one layer, 32768 tokens x 64 query heads x 128 (bf16, 512 MB)",
             "ms": ms, "tokens_per_s": n / (ms * 1e-3), "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
             "frac": nbytes / (ms * 1e-3) / 1e9 / hbm, "reps": reps}
+
+
+def offset_max(T, torch, st, cache, cfg, kept, restore, hbm, passes=5):
+    """The same pass with the maximum over the offsets instead of the folded
+    mean (tria_params.offset_reduce = OFFSET_MAX): per-kernel CUDA-event
+    times over `passes` passes, rows restored between them."""
+    prm = T.params(cfg.budget, cfg.window, cfg.sinks, T.OFFSET_MAX)
+    ws = T.alloc_workspace(T.tria_workspace_size(st, cache, prm))
+    T.tria_read_device_status(ws)
+    evs_all = []
+    for i in range(passes + 2):
+        restore()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        T.tria_set_pass_events(evs)
+        T.tria_compress_pass(st, cache, prm, kept, ws)
+        T.tria_set_pass_events(None)
+        if i >= 2:
+            evs_all.append(evs)
+    torch.cuda.synchronize()
+    if T.tria_read_device_status(ws) != 0:
+        raise RuntimeError("device status flags set (max-over-offsets pass)")
+    seg = [[e[k].elapsed_time(e[k + 1]) for e in evs_all] for k in range(4)]
+    ms = statistics.mean(e[0].elapsed_time(e[4]) for e in evs_all)
+    units = cfg.n_seq * cfg.n_layers * cfg.n_kv_heads
+    C = cfg.seq_len - cfg.window - cfg.sinks
+    score_ms = statistics.mean(seg[1])
+    del ws
+    return {"us_per_pass": 1e3 * ms, "keys_per_s": units * cfg.seq_len / (ms * 1e-3),
+            "kernels_us": {"coef": 1e3 * statistics.mean(seg[0]), "score": 1e3 * score_ms,
+                           "normalize_select": 1e3 * statistics.mean(seg[2]),
+                           "compact": 1e3 * statistics.mean(seg[3])},
+            "score_roofline": {"bound": "hbm", "achieved": units * C * 256 / (score_ms * 1e-3) / 1e9,
+                               "peak": hbm, "unit": "GB/s",
+                               "frac": units * C * 256 / (score_ms * 1e-3) / 1e9 / hbm},
+            "score_tflops": units * C * 2.0 * 128 * (2 * 17 * cfg.group) / (score_ms * 1e-3) / 1e12,
+            "passes": passes}
 
 
 def run16(T, w, st, cache, prm, ws, kept, restore):
