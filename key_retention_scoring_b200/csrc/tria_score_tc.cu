@@ -298,14 +298,24 @@ __device__ __forceinline__ void tmem_ld_nowait(uint32_t taddr, uint32_t (&r)[N])
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
                    "=r"(r[6]), "=r"(r[7])
                  : "r"(taddr));
-  } else {
-    static_assert(N == 16, "tmem_ld_nowait width");
+  } else if constexpr (N == 16) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
         "%14,%15}, [%16];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
           "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
           "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+  } else {
+    static_assert(N == 32, "tmem_ld_nowait width");
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
   }
 }
@@ -894,6 +904,13 @@ __device__ __forceinline__ void emit_scores(const ScoreParams &p, const EpRec &p
   }
 }
 
+// Maximum that returns NaN when either operand is NaN.
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
 // Epilogue of the previous tile in max mode: per head of this thread's band
 // group, S = max_j (hi_j + lo_j) + (norm hi + norm lo).
 template <int G>
@@ -909,20 +926,29 @@ __device__ __forceinline__ void epilogue_max(const ScoreParams &p, uint32_t tmem
 #pragma unroll
     for (int gi = 0; gi < GQ; ++gi) {
       const int g = q * GQ + gi;
-      uint32_t t[17][2], nv[2];
-#pragma unroll
-      for (int j = 0; j < 17; ++j)
-        if (j < nd) tmem_ld_nowait<2>(lb + (uint32_t)((g * nd + j) * 2), t[j]);
+      // the head's 2 nd columns: one 32-column load (offsets 0..15; beyond
+      // 2 nd it reads the next head's columns, unused) and one 2-column load
+      // for offset 16
+      uint32_t t[32], t16[2], nv[2];
+      const uint32_t c0 = lb + (uint32_t)(g * nd * 2);
+      tmem_ld_nowait<32>(c0, t);
+      if (nd == 17) tmem_ld_nowait<2>(c0 + 32, t16);
       tmem_ld_nowait<2>(lb + kMaxNormCol + (uint32_t)(2 * g), nv);
       tmem_wait_ld();
-      float m = __uint_as_float(t[0][0]) + __uint_as_float(t[0][1]);
+      // offsets past |D| read as -inf; a pairwise tree of NaN-propagating
+      // maxes, built in place over the loaded words
 #pragma unroll
-      for (int j = 1; j < 17; ++j) {
-        if (j < nd) {
-          const float v = __uint_as_float(t[j][0]) + __uint_as_float(t[j][1]);
-          m = (m != m) ? m : ((v != v || v > m) ? v : m);  // NaN propagates
-        }
+      for (int j = 0; j < 16; ++j)
+        t[j] = __float_as_uint((j < nd) ? __uint_as_float(t[2 * j]) + __uint_as_float(t[2 * j + 1])
+                                        : -INFINITY);
+      const float v16 = (nd == 17) ? __uint_as_float(t16[0]) + __uint_as_float(t16[1]) : -INFINITY;
+#pragma unroll
+      for (int w = 1; w < 16; w *= 2) {
+#pragma unroll
+        for (int j = 0; j + w < 16; j += 2 * w)
+          t[j] = __float_as_uint(max_nan(__uint_as_float(t[j]), __uint_as_float(t[j + w])));
       }
+      const float m = max_nan(__uint_as_float(t[0]), v16);
       sc[gi] = m + (__uint_as_float(nv[0]) + __uint_as_float(nv[1]));
     }
   } else {
