@@ -478,7 +478,7 @@ __device__ void agg_range(const float *__restrict__ raw, float *agg, int c0, int
 // larger than the list falls back to passes over all keys.  The emission is
 // one more pass.
 // ---------------------------------------------------------------------------
-struct UnitScalars {
+struct alignas(16) UnitScalars {  // 16-byte size: the key area after it is read as uint4
   int warp_tmp[32];
   uint32_t prefix;
   int remaining;
@@ -579,11 +579,25 @@ __device__ void unit_keys(const float *raw, int C, const float *s_mean, const fl
   }
 }
 
+static_assert(sizeof(UnitScalars) % 16 == 0, "shared-memory areas after UnitScalars stay 16-byte aligned");
+
+// Warp-wide inclusive scan of v (lane order).
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, v, o);
+    if (lane >= o) v += y;
+  }
+  return v;
+}
+
+// keys: shared memory, readable (as uint4) up to a multiple of 4 NT entries
+// past C; entries >= C are ignored.  Warp w owns the candidates
+// [w R, (w + 1) R), R = steps * 128; a lane takes 4 consecutive keys per step.
 template <int NT>
 __device__ void select_keys(const uint32_t *keys, int C, int K, int N, int B, int W, int S,
                             int32_t *kept, uint32_t *hist, uint2 *list, UnitScalars &sc, int tid) {
   const int lane = tid & 31, warp = tid >> 5;
-  const uint32_t lt = (1u << lane) - 1u;
   for (int j = tid; j < S; j += NT) kept[j] = j;
   for (int j = tid; j < W; j += NT) kept[B - W + j] = N - W + j;
   if (K <= 0) return;
@@ -594,32 +608,46 @@ __device__ void select_keys(const uint32_t *keys, int C, int K, int N, int B, in
   }
   __syncthreads();
   pick_bin<0, NT>(hist, kHistBins, sc, 20, tid);
-  // warp w owns candidates [w R, (w + 1) R), R = 32 steps
-  const int steps = (C + NT - 1) / NT;
-  const int cb = warp * steps * 32;
+  const int steps = (C + NT * 4 - 1) / (NT * 4);
+  const int R = steps * 128;
+  const int cb = warp * R;
   clear_words<NT>(hist, kHistBins, tid);
   __syncthreads();
   const uint32_t d1 = sc.prefix >> 20;
   {
+    // keys above the chosen first-digit bin, per warp; the bin's keys go to
+    // the second-digit histogram and the list
     int above = 0;
     for (int e = 0; e < steps; ++e) {
-      const int c = cb + e * 32 + lane;
-      const bool valid = c < C;
-      const uint32_t k = valid ? keys[c] : 0u;
-      above += __popc(__ballot_sync(kFull, valid && (k >> 20) > d1));
-      const bool in = valid && (k >> 20) == d1;
-      const uint32_t bal = __ballot_sync(kFull, in);
-      if (bal) {
+      const int c0 = cb + e * 128 + lane * 4;
+      const uint4 k4 = *reinterpret_cast<const uint4 *>(keys + c0);
+      const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+      uint32_t inmask = 0u;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const bool valid = c0 + i < C;
+        above += (valid && (kk[i] >> 20) > d1) ? 1 : 0;
+        inmask |= (valid && (kk[i] >> 20) == d1) ? (1u << i) : 0u;
+      }
+      if (__ballot_sync(kFull, inmask != 0u)) {
+        const int cnt = __popc(inmask);
+        const int incl = warp_incl_scan(cnt, lane);
         int base = 0;
-        if (lane == 0) base = atomicAdd(&sc.list_n, __popc(bal));
-        base = __shfl_sync(kFull, base, 0);
-        if (in) {
-          atomicAdd(hist + ((k >> 8) & 0xfffu), 1u);
-          const int idx = base + __popc(bal & lt);
-          if (idx < kListCap) list[idx] = make_uint2(k, (uint32_t)c);
+        if (lane == 31) base = atomicAdd(&sc.list_n, incl);
+        base = __shfl_sync(kFull, base, 31);
+        int idx = base + incl - cnt;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if ((inmask >> i) & 1u) {
+            atomicAdd(hist + ((kk[i] >> 8) & 0xfffu), 1u);
+            if (idx < kListCap) list[idx] = make_uint2(kk[i], (uint32_t)(c0 + i));
+            ++idx;
+          }
         }
       }
     }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) above += __shfl_xor_sync(kFull, above, o);
     if (lane == 0) {
       sc.warp_gt[warp] = above;
       sc.warp_eq[warp] = 0;
@@ -653,17 +681,27 @@ __device__ void select_keys(const uint32_t *keys, int C, int K, int N, int B, in
   if (use_list) {
     for (int i = tid; i < ln; i += NT) {
       const uint2 e = list[i];
-      const int w = (int)e.y / (steps * 32);
+      const int w = (int)e.y / R;
       if (e.x > T) atomicAdd(&sc.warp_gt[w], 1);
       else if (e.x == T) atomicAdd(&sc.warp_eq[w], 1);
     }
   } else {
     int gt = 0, eq = 0;
     for (int e = 0; e < steps; ++e) {
-      const int c = cb + e * 32 + lane;
-      const uint32_t k = (c < C) ? keys[c] : 0u;
-      gt += __popc(__ballot_sync(kFull, c < C && (k >> 20) == d1 && k > T));
-      eq += __popc(__ballot_sync(kFull, c < C && k == T));
+      const int c0 = cb + e * 128 + lane * 4;
+      const uint4 k4 = *reinterpret_cast<const uint4 *>(keys + c0);
+      const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const bool valid = c0 + i < C;
+        gt += (valid && (kk[i] >> 20) == d1 && kk[i] > T) ? 1 : 0;
+        eq += (valid && kk[i] == T) ? 1 : 0;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      gt += __shfl_xor_sync(kFull, gt, o);
+      eq += __shfl_xor_sync(kFull, eq, o);
     }
     if (lane == 0) {
       atomicAdd(&sc.warp_gt[warp], gt);
@@ -680,19 +718,42 @@ __device__ void select_keys(const uint32_t *keys, int C, int K, int N, int B, in
   int run_keep = gt_before + min(eq_before, need);
   int run_eq = eq_before;
   for (int e = 0; e < steps; ++e) {
-    const int c = cb + e * 32 + lane;
-    const bool valid = c < C;
-    const uint32_t k = valid ? keys[c] : 0u;
-    const bool is_eq = valid && k == T;
-    const uint32_t beq = __ballot_sync(kFull, is_eq);
-    const bool keep = valid && (k > T || (is_eq && run_eq + __popc(beq & lt) < need));
-    const uint32_t bk = __ballot_sync(kFull, keep);
-    if (keep) {
-      const int pos = run_keep + __popc(bk & lt);
-      if (pos < K) kept[S + pos] = S + c;
+    const int c0 = cb + e * 128 + lane * 4;
+    const uint4 k4 = *reinterpret_cast<const uint4 *>(keys + c0);
+    const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+    uint32_t gtm = 0u, eqm = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool valid = c0 + i < C;
+      gtm |= (valid && kk[i] > T) ? (1u << i) : 0u;
+      eqm |= (valid && kk[i] == T) ? (1u << i) : 0u;
     }
-    run_eq += __popc(beq);
-    run_keep += __popc(bk);
+    uint32_t keepm = gtm;
+    if (__ballot_sync(kFull, eqm != 0u)) {
+      // ties in slot order: lanes in order, then a lane's keys in order
+      const int ne = __popc(eqm);
+      const int incl = warp_incl_scan(ne, lane);
+      int rank = run_eq + incl - ne;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if ((eqm >> i) & 1u) {
+          if (rank < need) keepm |= 1u << i;
+          ++rank;
+        }
+      }
+      run_eq += __shfl_sync(kFull, incl, 31);
+    }
+    const int nk = __popc(keepm);
+    const int incl = warp_incl_scan(nk, lane);
+    int pos = run_keep + incl - nk;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if ((keepm >> i) & 1u) {
+        if (pos < K) kept[S + pos] = S + c0 + i;
+        ++pos;
+      }
+    }
+    run_keep += __shfl_sync(kFull, incl, 31);
   }
 }
 

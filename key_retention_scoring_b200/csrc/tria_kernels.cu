@@ -273,9 +273,11 @@ __global__ void __launch_bounds__(kThreads) tail_kernel(const __grid_constant__ 
 // ---------------------------------------------------------------------------
 constexpr int kUnitThreads = 1024;
 
+// the key area is read 4 NT keys at a time by the selection: padded to that
 size_t unit_tail_smem_bytes(int c_max) {
+  const size_t pad = (size_t)kUnitThreads * 4;
   return sizeof(UnitScalars) + (size_t)kHistBins * 4 + (size_t)kListCap * 8 +
-         (size_t)((c_max + 3) & ~3) * 4;
+         (((size_t)c_max + pad - 1) / pad) * pad * 4;
 }
 
 template <int G>
