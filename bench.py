@@ -385,6 +385,7 @@ def main():
         line["run16"] = run16(T, w, st, cache, prm, ws, kept, restore)
         line["calibration"] = calibration(T, torch, hbm)
         line["offset_max"] = offset_max(T, torch, st, cache, cfg, kept, restore, hbm)
+        line["layer_budgets"] = layer_budgets(T, torch, w, st, cfg, restore, hbm)
         line["e2e"] = e2e(T, torch, w, st, cache, prm, ws, kept, restore, args.e2e_steps, keys, world)
         if rank == 0 and world == 1:
             v, n_units, spent = oracle_unit_keys_per_s(cfg, args.cpu_seconds)
@@ -464,6 +465,61 @@ def offset_max(T, torch, st, cache, cfg, kept, restore, hbm, passes=5):
                                "frac": units * C * 256 / (score_ms * 1e-3) / 1e9 / hbm},
             "score_tflops": units * C * 2.0 * 128 * (2 * 17 * cfg.group) / (score_ms * 1e-3) / 1e12,
             "passes": passes}
+
+
+def layer_budgets(T, torch, w, st, cfg, restore, hbm, passes=5):
+    """The same pass with per-layer budgets (tria_params.layer_budget_scales,
+    linear from 0.5 to 1.5 over the layers, mean 1) and lengths per (sequence,
+    layer) (tria_cache_view.layer_seq_lens): per-kernel CUDA-event times over
+    `passes` passes, rows and lengths restored between them."""
+    L = cfg.n_layers
+    scales = [0.5 + l / max(1, L - 1) for l in range(L)]
+    ll = torch.full((cfg.n_seq, L), cfg.seq_len, dtype=torch.int32, device="cuda")
+    cache = T.Cache.from_workload(w, layer_seq_lens=ll)
+    prm = T.params(cfg.budget, cfg.window, cfg.sinks, layer_budget_scales=scales)
+    budgets, bmax = T.tria_layer_budgets(st, cache, prm)
+    B = cfg.budget
+    # rows past the default budget that this variant's compaction overwrites
+    kx = [t[:, :, B:bmax].clone() for t in w.k]
+    vx = [t[:, :, B:bmax].clone() for t in w.v]
+    kept = torch.empty((cfg.n_seq, L, cfg.n_kv_heads, bmax), dtype=torch.int32, device="cuda")
+    ws = T.alloc_workspace(T.tria_workspace_size(st, cache, prm))
+    T.tria_read_device_status(ws)
+    evs_all = []
+    for i in range(passes + 2):
+        restore()
+        for l in range(L):
+            w.k[l][:, :, B:bmax].copy_(kx[l])
+            w.v[l][:, :, B:bmax].copy_(vx[l])
+        ll.fill_(cfg.seq_len)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        T.tria_set_pass_events(evs)
+        T.tria_compress_pass(st, cache, prm, kept, ws)
+        T.tria_set_pass_events(None)
+        if i >= 2:
+            evs_all.append(evs)
+    torch.cuda.synchronize()
+    if T.tria_read_device_status(ws) != 0:
+        raise RuntimeError("device status flags set (per-layer budgets pass)")
+    if sorted(set(ll[0].cpu().tolist())) != sorted(set(budgets)):
+        raise RuntimeError("per-layer lengths after the pass differ from the budgets")
+    seg = [[e[k].elapsed_time(e[k + 1]) for e in evs_all] for k in range(4)]
+    ms = statistics.mean(e[0].elapsed_time(e[4]) for e in evs_all)
+    units = cfg.n_seq * L * cfg.n_kv_heads
+    C = cfg.seq_len - cfg.window - cfg.sinks
+    score_ms = statistics.mean(seg[1])
+    kept_rows = cfg.n_seq * cfg.n_kv_heads * sum(budgets)  # every unit is compressed
+    del ws, kx, vx
+    return {"workload": f"scales 0.5 .. 1.5 linear over {L} layers (budgets {min(budgets)} .. "
+                        f"{max(budgets)}), lengths per (sequence, layer)",
+            "us_per_pass": 1e3 * ms, "keys_per_s": units * cfg.seq_len / (ms * 1e-3),
+            "kernels_us": {"coef": 1e3 * statistics.mean(seg[0]), "score": 1e3 * score_ms,
+                           "normalize_select": 1e3 * statistics.mean(seg[2]),
+                           "compact_and_lengths": 1e3 * statistics.mean(seg[3])},
+            "score_roofline": {"bound": "hbm", "achieved": units * C * 256 / (score_ms * 1e-3) / 1e9,
+                               "peak": hbm, "unit": "GB/s",
+                               "frac": units * C * 256 / (score_ms * 1e-3) / 1e9 / hbm},
+            "kept_rows": kept_rows, "passes": passes}
 
 
 def run16(T, w, st, cache, prm, ws, kept, restore):

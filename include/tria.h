@@ -40,7 +40,8 @@
  *     scoring kernel reads K through TMA tensor maps that the library encodes
  *     (and caches) per layer base pointer; a stride pattern the tensor-map
  *     encoder rejects returns TRIA_ERR_UNSUPPORTED.
- *   - A unit whose length N is at most the budget is left unchanged.
+ *   - A unit whose length N is at most its layer's budget B_l (plus the
+ *     compression interval, see tria_params) is left unchanged.
  *   - Floating point decides the kept set only through the fp32 aggregated
  *     score agg (below); exactly equal agg go to the lower slot; -0.0 equals
  *     +0.0; NaN ranks below every number.
@@ -121,8 +122,8 @@ typedef struct {
   int64_t num_blocks;        /* paged: blocks in each layer's K (and V) pool; block
                                 ids outside [0, num_blocks) read as zero rows        */
   int32_t *seq_lens;         /* device [n_seq] cached tokens N per sequence; set to
-                                min(N, budget) by tria_compact when it covers the last
-                                layer                                                */
+                                the budget for every compressed sequence by
+                                tria_compact when it covers the last layer           */
   const int64_t *query_pos;  /* device [n_seq] position p_q of the current query: the
                                 position of the newest cached token (offsets
                                 delta in D are added to it)                          */
@@ -130,6 +131,13 @@ typedef struct {
                                 token position of every slot; compacted with the
                                 rows when non-null.  Scoring never reads it: the
                                 post-RoPE key already carries its position.          */
+  int32_t *layer_seq_lens;   /* optional device [n_seq][n_layers]: cached tokens N of
+                                each (sequence, layer).  When non-null it replaces
+                                seq_lens (which is then neither read nor written and
+                                may be NULL) and tria_compact updates the entries of
+                                the layers it covers.  Required when the per-layer
+                                budgets differ (tria_params.layer_budget_scales),
+                                since the layers then keep different lengths.        */
 } tria_cache_view;
 
 /* How the trigonometric term combines the future offsets delta in D. */
@@ -142,12 +150,30 @@ typedef enum {
                            G * |D| <= 136 (G <= 8 at |D| = 17), else UNSUPPORTED    */
 } tria_offset_reduce;
 
-/* Retention parameters (one set for all units of a call). */
+/* Retention parameters (one set for all units of a call).
+ *
+ * Budget of layer l (rows kept per unit, window and sinks included):
+ *   base = budget_pct > 0 ? floor(budget_pct * max_seq_len / 100) : budget
+ *   B_l  = floor(base * scale_l + 1/2), scale_l = layer_budget_scales[l] (1 if NULL)
+ * (the runtime of GitHub issue #10 of the llama.cpp TurboQuant HIP fork takes a
+ * percentage budget, "budget=50%", and per-layer budget scales that default to
+ * 1.0; the percentage is read as a share of the cache capacity max_seq_len).
+ * Every B_l must be >= window + sinks, else INVALID_ARG.  A unit with N cached
+ * rows is compressed only when N - B_l >= max(interval, 1): pruning runs once
+ * per window of interval generated tokens (academ.us article 2607.13051, sec. 8,
+ * beta = 128; the same issue's runtime log, "interval=128"); every other unit is
+ * left as it is.  kept_idx rows have B_max = max_l B_l entries (over all layers
+ * of the model; tria_layer_budgets returns it). */
 typedef struct {
   int budget;  /* B: rows kept per unit, window and sinks included; >= window + sinks */
   int window;  /* W: the newest W slots are always kept                               */
   int sinks;   /* S: the oldest S slots are always kept                               */
   int offset_reduce;  /* tria_offset_reduce; 0 (mean) when zero-initialised           */
+  float budget_pct;   /* > 0: percentage budget, replaces budget (see above); 0: off  */
+  const float *layer_budget_scales;  /* optional host [n_layers], finite and > 0;
+                                        NULL = 1.0 for every layer                   */
+  int interval;       /* compression interval beta >= 0 (0 and 1: compress whenever
+                         N > B_l)                                                   */
 } tria_params;
 
 /* Human-readable name of a status code (static string). */
@@ -186,6 +212,16 @@ tria_status tria_free_stats(tria_stats *stats);
 tria_status tria_stats_desc(const tria_stats *stats, tria_model_desc *desc_out);
 
 /*
+ * tria_layer_budgets - the budget B_l of every layer of the model under these
+ * parameters (formula at tria_params) and the kept_idx row length B_max.
+ *   budgets : optional host int [n_layers] (NULL: not written)
+ *   row_len : optional host int, B_max = max_l B_l
+ * Errors: INVALID_ARG (the same parameter checks as the pass entry points).
+ */
+tria_status tria_layer_budgets(const tria_stats *stats, const tria_cache_view *cache,
+                               const tria_params *params, int *budgets, int *row_len);
+
+/*
  * tria_workspace_size - device workspace bytes that tria_score, tria_select
  * and tria_compress_pass need for this cache view, these parameters and the
  * layer range [layer0, layer1).  The workspace is scratch: no state is kept
@@ -207,7 +243,8 @@ tria_status tria_workspace_size(const tria_stats *stats, const tria_cache_view *
  *              population std of head g over the unit's C candidates;
  *   scores_out optional [n_seq][layer1 - layer0][n_kv_heads][C_max][G]:
  *              S~_g of candidate c for the G query heads of the KV head.
- * Entries c >= C, and units with N <= budget, are not written.
+ * Entries c >= C, and units that are not compressed (N - B_l < max(interval,
+ * 1)), are not written.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  */
 tria_status tria_score(const tria_stats *stats, const tria_cache_view *cache,
@@ -218,10 +255,11 @@ tria_status tria_score(const tria_stats *stats, const tria_cache_view *cache,
 /*
  * tria_select - kept slots of every unit of layers [layer0, layer1) from
  * agg (layout of tria_score's agg_out).
- *   kept_idx (device int32 [n_seq][layer1 - layer0][n_kv_heads][budget]):
- *   ascending slots: 0 .. sinks-1, then the top K = budget - window - sinks
- *   candidates by agg (ties: lower slot), then N-window .. N-1.  A unit with
- *   N <= budget gets 0 .. N-1 followed by -1.
+ *   kept_idx (device int32 [n_seq][layer1 - layer0][n_kv_heads][B_max]):
+ *   ascending slots: 0 .. sinks-1, then the top K = B_l - window - sinks
+ *   candidates by agg (ties: lower slot), then N-window .. N-1, then -1 up to
+ *   B_max.  A unit that is not compressed gets j at entry j < min(N, B_max)
+ *   and -1 after it (nothing moves).
  * Errors: INVALID_ARG, WORKSPACE, CUDA.
  */
 tria_status tria_select(const tria_stats *stats, const tria_cache_view *cache,
@@ -235,11 +273,16 @@ tria_status tria_select(const tria_stats *stats, const tria_cache_view *cache,
  * the old row kept_idx[j] (kept_idx as tria_select writes it; -1 entries and
  * entries equal to j move nothing).  kept_idx must be strictly ascending
  * with kept_idx[j] >= j (tria_select guarantees it); rows are byte-copied.
- * When layer1 == n_layers, seq_lens[s] becomes min(N_s, budget) and, for the
- * paged layout, the blocks of each sequence past ceil(budget / block_size)
- * that held rows are listed in freed_blocks (device int32 [n_seq][max_blocks_per_seq],
- * nullable) with their count in n_freed (device int32 [n_seq], nullable); the
- * block table itself is not modified.
+ * Without layer_seq_lens: when layer1 == n_layers, seq_lens[s] becomes B
+ * for every compressed sequence and, for the paged layout, the blocks of each
+ * sequence past ceil(B / block_size) that held rows are listed in freed_blocks
+ * (device int32 [n_seq][max_blocks_per_seq], nullable) with their count in
+ * n_freed (device int32 [n_seq], nullable); the block table itself is not
+ * modified.  With layer_seq_lens: the length of every compressed (sequence,
+ * layer) of [layer0, layer1) becomes B_l; blocks are shared by the layers, so
+ * a call over every layer lists the blocks past ceil(max_l new N / block_size)
+ * up to ceil(max_l old N / block_size), and a call over part of the layers
+ * frees none (n_freed[s] = 0).
  * Errors: INVALID_ARG, CUDA.
  */
 tria_status tria_compact(const tria_stats *stats, const tria_cache_view *cache,
@@ -250,7 +293,7 @@ tria_status tria_compact(const tria_stats *stats, const tria_cache_view *cache,
 /*
  * tria_compress_pass - the whole pass over every layer: score, select and
  * compact, with scores and agg kept in the workspace.  kept_idx: optional
- * device [n_seq][n_layers][n_kv_heads][budget] copy of the kept slots (NULL:
+ * device [n_seq][n_layers][n_kv_heads][B_max] copy of the kept slots (NULL:
  * kept in the workspace only).  freed_blocks / n_freed as in tria_compact.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
  */

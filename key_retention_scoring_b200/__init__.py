@@ -30,7 +30,8 @@ MAX_LAYERS = 128
 EXPORTS = ["tria_status_string", "tria_version", "tria_load_stats", "tria_free_stats",
            "tria_stats_desc", "tria_workspace_size", "tria_score", "tria_select", "tria_compact",
            "tria_compress_pass", "tria_read_device_status", "tria_set_pass_events",
-           "tria_compress_pass_static", "tria_calib_accumulate", "tria_calib_finalize"]
+           "tria_compress_pass_static", "tria_calib_accumulate", "tria_calib_finalize",
+           "tria_layer_budgets"]
 STATIC_SCRATCH_BYTES = 32 * 1024 * 1024   # TRIA_STATIC_SCRATCH_BYTES
 
 
@@ -56,12 +57,15 @@ class CacheView(ctypes.Structure):
                 ("block_table", ctypes.c_void_p), ("max_blocks_per_seq", ctypes.c_int),
                 ("block_size", ctypes.c_int), ("num_blocks", ctypes.c_int64),
                 ("seq_lens", ctypes.c_void_p),
-                ("query_pos", ctypes.c_void_p), ("positions", ctypes.c_void_p)]
+                ("query_pos", ctypes.c_void_p), ("positions", ctypes.c_void_p),
+                ("layer_seq_lens", ctypes.c_void_p)]
 
 
 class Params(ctypes.Structure):
     _fields_ = [("budget", ctypes.c_int), ("window", ctypes.c_int), ("sinks", ctypes.c_int),
-                ("offset_reduce", ctypes.c_int)]
+                ("offset_reduce", ctypes.c_int), ("budget_pct", ctypes.c_float),
+                ("layer_budget_scales", ctypes.POINTER(ctypes.c_float)),
+                ("interval", ctypes.c_int)]
 
 
 _lib = None
@@ -103,6 +107,8 @@ def lib() -> ctypes.CDLL:
                                         ctypes.c_int64, ctypes.c_int64, _VP, _VP]
     L.tria_calib_finalize.argtypes = [ctypes.POINTER(ModelDesc), _VP, ctypes.c_int64, _VP, _VP,
                                       _VP, _VP]
+    L.tria_layer_budgets.argtypes = [_VP, ctypes.POINTER(CacheView), ctypes.POINTER(Params),
+                                     ctypes.POINTER(_I), ctypes.POINTER(_I)]
     for name in EXPORTS:
         if name not in ("tria_status_string", "tria_version"):
             getattr(L, name).restype = _I
@@ -188,33 +194,60 @@ class Cache:
     def __init__(self, layout, k_layers, v_layers, seq_lens, query_pos, max_seq_len, *,
                  stride_seq=0, stride_head=0, stride_token=128, stride_block=0,
                  block_table=None, max_blocks_per_seq=0, block_size=0, num_blocks=0,
-                 positions=None):
-        self._keep = (k_layers, v_layers, seq_lens, query_pos, block_table, positions)
+                 positions=None, layer_seq_lens=None, n_seq=None):
+        """layer_seq_lens: optional int32 [n_seq][n_layers] lengths per (sequence,
+        layer); seq_lens may then be None (n_seq is taken from layer_seq_lens)."""
+        self._keep = (k_layers, v_layers, seq_lens, query_pos, block_table, positions,
+                      layer_seq_lens)
         n = len(k_layers)
         self._k = (_VP * n)(*[_ptr(t) for t in k_layers])
         self._v = (_VP * n)(*[_ptr(t) for t in v_layers]) if v_layers is not None else None
+        if n_seq is None:
+            n_seq = int(seq_lens.numel()) if seq_lens is not None else int(layer_seq_lens.shape[0])
         self.view = CacheView(
-            layout, int(seq_lens.numel()), int(max_seq_len),
+            layout, int(n_seq), int(max_seq_len),
             ctypes.cast(self._k, ctypes.POINTER(_VP)),
             ctypes.cast(self._v, ctypes.POINTER(_VP)) if self._v is not None else None,
             stride_seq, stride_head, stride_token, stride_block, _ptr(block_table),
             max_blocks_per_seq, block_size, num_blocks, _ptr(seq_lens), _ptr(query_pos),
-            _ptr(positions))
+            _ptr(positions), _ptr(layer_seq_lens))
 
     @classmethod
-    def from_workload(cls, w) -> "Cache":
-        """View of a ``synth.Workload``."""
+    def from_workload(cls, w, layer_seq_lens=None) -> "Cache":
+        """View of a ``synth.Workload`` (optionally with lengths per (sequence,
+        layer) instead of its per-sequence lengths)."""
         st = w.strides
-        return cls(w.cfg.layout, w.k, w.v, w.seq_lens, w.query_pos, w.max_seq_len,
+        return cls(w.cfg.layout, w.k, w.v, None if layer_seq_lens is not None else w.seq_lens,
+                   w.query_pos, w.max_seq_len,
                    stride_seq=st["seq"], stride_head=st["head"], stride_token=st["token"],
                    stride_block=st["block"], block_table=w.block_table,
                    max_blocks_per_seq=w.max_blocks, block_size=w.cfg.block_size,
-                   num_blocks=getattr(w, "n_blocks", 0), positions=w.positions)
+                   num_blocks=getattr(w, "n_blocks", 0), positions=w.positions,
+                   layer_seq_lens=layer_seq_lens, n_seq=int(w.seq_lens.numel()))
 
 
-def params(budget, window, sinks, offset_reduce=0) -> Params:
-    """offset_reduce: OFFSET_MEAN (the published average over D) or OFFSET_MAX."""
-    return Params(budget, window, sinks, offset_reduce)
+def params(budget, window, sinks, offset_reduce=0, budget_pct=0.0, layer_budget_scales=None,
+           interval=0) -> Params:
+    """offset_reduce: OFFSET_MEAN (the published average over D) or OFFSET_MAX.
+    budget_pct > 0: the budget is that percentage of the cache capacity;
+    layer_budget_scales: per-layer multipliers of the budget (None: 1.0);
+    interval: a unit is compressed only once it is that many rows past its budget."""
+    prm = Params(budget, window, sinks, offset_reduce, float(budget_pct), None, int(interval))
+    if layer_budget_scales is not None:
+        arr = (ctypes.c_float * len(layer_budget_scales))(*[float(x) for x in layer_budget_scales])
+        prm._scales = arr  # kept alive with the parameters
+        prm.layer_budget_scales = ctypes.cast(arr, ctypes.POINTER(ctypes.c_float))
+    return prm
+
+
+def tria_layer_budgets(stats, cache, prm):
+    """(per-layer budgets B_l as a list, kept_idx row length B_max)."""
+    n = stats.desc.n_layers
+    out = (_I * n)()
+    row = _I()
+    _check(lib().tria_layer_budgets(stats.handle, ctypes.byref(cache.view), ctypes.byref(prm),
+                                    out, ctypes.byref(row)), "tria_layer_budgets")
+    return list(out), row.value
 
 
 def tria_workspace_size(stats: Stats, cache: Cache, prm: Params, layer0=0, layer1=None) -> int:

@@ -47,12 +47,14 @@ tria_status make_geom(const tria_stats *stats, const tria_cache_view *cache,
   if (layer0 < 0 || layer1 <= layer0 || layer1 > d.n_layers) return TRIA_ERR_INVALID_ARG;
   if (cache->n_seq < 1 || cache->n_seq > TRIA_MAX_SEQS) return TRIA_ERR_INVALID_ARG;
   if (cache->max_seq_len < 1) return TRIA_ERR_INVALID_ARG;
-  if (params->window < 0 || params->sinks < 0 || params->budget < 1 ||
-      params->budget < params->window + params->sinks)
-    return TRIA_ERR_INVALID_ARG;
+  if (params->window < 0 || params->sinks < 0 || params->interval < 0) return TRIA_ERR_INVALID_ARG;
+  const double pct = params->budget_pct;  // the fp32 value, exactly
+  if (!std::isfinite(pct) || pct < 0.0 || pct > 100.0) return TRIA_ERR_INVALID_ARG;
   if (cache->layout != TRIA_LAYOUT_CONTIGUOUS && cache->layout != TRIA_LAYOUT_PAGED)
     return TRIA_ERR_INVALID_ARG;
-  if (cache->k_layers == nullptr || cache->seq_lens == nullptr || cache->query_pos == nullptr)
+  const bool layer_lens = cache->layer_seq_lens != nullptr;
+  if (cache->k_layers == nullptr || cache->query_pos == nullptr ||
+      (!layer_lens && cache->seq_lens == nullptr))
     return TRIA_ERR_INVALID_ARG;
   for (int l = layer0; l < layer1; ++l)
     if (cache->k_layers[l] == nullptr || !aligned16(cache->k_layers[l])) return TRIA_ERR_INVALID_ARG;
@@ -80,7 +82,41 @@ tria_status make_geom(const tria_stats *stats, const tria_cache_view *cache,
   g.hkv = d.n_kv_heads;
   g.hq = d.n_q_heads;
   g.g = d.n_q_heads / d.n_kv_heads;
-  g.budget = params->budget;
+  // budget of every layer: base = the absolute budget, or pct % of the
+  // capacity; B_l = round-half-up(base * scale_l); B_max sizes the kept rows
+  const double base = pct > 0.0 ? std::floor(pct * (double)cache->max_seq_len / 100.0)
+                                 : (double)params->budget;
+  int bmax = 0, b_first = 0;
+  bool uniform = true;
+  for (int l = 0; l < d.n_layers; ++l) {
+    double sc = 1.0;
+    if (params->layer_budget_scales != nullptr) {
+      sc = params->layer_budget_scales[l];
+      if (!std::isfinite(sc) || !(sc > 0.0)) return TRIA_ERR_INVALID_ARG;
+    }
+    const double b = std::floor(base * sc + 0.5);
+    if (!(b >= 1.0) || b > (double)(INT32_MAX / 4)) return TRIA_ERR_INVALID_ARG;
+    const int bl = (int)b;
+    if (bl < params->window + params->sinks) return TRIA_ERR_INVALID_ARG;
+    if (l == 0) b_first = bl;
+    uniform = uniform && bl == b_first;
+    bmax = bl > bmax ? bl : bmax;
+    if (l >= layer0 && l < layer1) g.lbudget[l - layer0] = bl;
+  }
+  // one length per sequence cannot describe layers kept at different budgets
+  if (!uniform && !layer_lens) return TRIA_ERR_INVALID_ARG;
+  g.budget = bmax;
+  g.trigger = params->interval > 1 ? params->interval : 1;
+  g.per_layer = layer_lens ? 1 : 0;
+  if (layer_lens) {
+    g.lens = cache->layer_seq_lens + layer0;
+    g.lens_s = d.n_layers;
+    g.lens_l = 1;
+  } else {
+    g.lens = cache->seq_lens;
+    g.lens_s = 1;
+    g.lens_l = 0;
+  }
   g.window = params->window;
   g.sinks = params->sinks;
   g.max_seq_len = cache->max_seq_len;
@@ -229,12 +265,12 @@ CoefParams make_coef(const tria_stats *st, const Geom &g, const tria_cache_view 
   cp.w_norm = st->dev.w_norm;
   cp.omega = st->dev.omega;
   cp.query_pos = c->query_pos;
-  cp.seq_lens = c->seq_lens;
   cp.btile = at<uint16_t>(ws, wl.btile);
   cp.item_counter = at<uint32_t>(ws, wl.hdr);
   cp.status = at<int32_t>(ws, wl.hdr + 4);
   cp.unit_done = at<uint32_t>(ws, wl.unit_done);
   cp.seq_items = at<int32_t>(ws, wl.seq_items);
+  cp.row_items = at<int32_t>(ws, wl.row_items);
   cp.kept = kept;
   cp.hist = with_hist ? at<uint32_t>(ws, wl.hist) : nullptr;
   return cp;
@@ -253,6 +289,7 @@ tria_status make_score(const Geom &g, const tria_cache_view *c, int layer0, int 
   sp.item_counter = at<uint32_t>(ws, wl.hdr);
   sp.status = at<int32_t>(ws, wl.hdr + 4);
   sp.seq_items = at<int32_t>(ws, wl.seq_items);
+  sp.row_items = at<int32_t>(ws, wl.row_items);
   sp.moments = at<double>(ws, wl.moments);
   sp.raw = at<float>(ws, wl.raw);
   sp.raw_stride = wl.raw_stride;
@@ -262,7 +299,6 @@ tria_status make_score(const Geom &g, const tria_cache_view *c, int layer0, int 
 TailParams make_tail(const Geom &g, const tria_cache_view *c, void *ws, const WsLayout &wl) {
   TailParams tp{};
   tp.geo = g;
-  tp.seq_lens = c->seq_lens;
   tp.status = at<int32_t>(ws, wl.hdr + 4);
   tp.moments = at<double>(ws, wl.moments);
   tp.raw = at<float>(ws, wl.raw);
@@ -280,6 +316,21 @@ TailParams make_tail(const Geom &g, const tria_cache_view *c, void *ws, const Ws
   return tp;
 }
 
+LensParams make_lens(const Geom &g, const tria_cache_view *c, int layer0, int layer1,
+                     int32_t *freed_blocks, int32_t *n_freed) {
+  LensParams lp{};
+  lp.geo = g;
+  lp.layer_lens = c->layer_seq_lens;
+  lp.paged = c->layout == TRIA_LAYOUT_PAGED ? 1 : 0;
+  lp.block_table = c->block_table;
+  lp.max_blocks = c->max_blocks_per_seq;
+  lp.block_size = c->block_size;
+  lp.all_layers = (layer0 == 0 && layer1 == g.n_layers) ? 1 : 0;
+  lp.freed_blocks = freed_blocks;
+  lp.n_freed = n_freed;
+  return lp;
+}
+
 }  // namespace
 
 WsLayout ws_layout(const Geom &g) {
@@ -295,6 +346,7 @@ WsLayout ws_layout(const Geom &g) {
   w.hdr = take(256);
   w.unit_done = take((size_t)g.n_units * 4);
   w.seq_items = take((size_t)(g.n_seq + 1) * 4);
+  w.row_items = take(((size_t)g.n_seq * g.nl + 1) * 4);
   w.btile = take((size_t)g.n_units * g.b_bytes);
   w.moments = take((size_t)g.n_units * g.tiles_max * kRowGroups * g.g * 2 * 8);
   w.hist = take((size_t)g.n_units * kAggHistBins * 4);
@@ -428,6 +480,19 @@ tria_status tria_stats_desc(const tria_stats *st, tria_model_desc *out) {
   return TRIA_OK;
 }
 
+tria_status tria_layer_budgets(const tria_stats *stats, const tria_cache_view *cache,
+                               const tria_params *params, int *budgets, int *row_len) {
+  if (stats == nullptr) return TRIA_ERR_INVALID_ARG;
+  const int L = stats->dev.desc.n_layers;
+  Geom g;
+  const tria_status st = make_geom(stats, cache, params, 0, L, &g);
+  if (st != TRIA_OK) return st;
+  if (budgets != nullptr)
+    for (int l = 0; l < L; ++l) budgets[l] = g.lbudget[l];
+  if (row_len != nullptr) *row_len = g.budget;
+  return TRIA_OK;
+}
+
 tria_status tria_workspace_size(const tria_stats *stats, const tria_cache_view *cache,
                                 const tria_params *params, int layer0, int layer1,
                                 size_t *bytes) {
@@ -480,7 +545,6 @@ tria_status tria_select(const tria_stats *stats, const tria_cache_view *cache,
   if ((st = check_workspace(g, ws, ws_bytes, &wl)) != TRIA_OK) return st;
   SelectParams p{};
   p.geo = g;
-  p.seq_lens = cache->seq_lens;
   p.status = at<int32_t>(ws, wl.hdr + 4);
   p.agg = agg;
   p.agg_stride = g.c_max;
@@ -502,10 +566,13 @@ tria_status tria_compact(const tria_stats *stats, const tria_cache_view *cache,
   p.geo = g;
   p.cache = make_cache_dev(cache, layer0, layer1);
   p.kept = kept_idx;
-  p.update_lens = (layer1 == g.n_layers) ? 1 : 0;
+  p.update_lens = (!g.per_layer && layer1 == g.n_layers) ? 1 : 0;
   p.freed_blocks = freed_blocks;
   p.n_freed = n_freed;
-  return cuda_status(launch_compact(p, reinterpret_cast<cudaStream_t>(stream)));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (launch_compact(p, s) != cudaSuccess) return TRIA_ERR_CUDA;
+  if (!g.per_layer) return TRIA_OK;
+  return cuda_status(launch_layer_lens(make_lens(g, cache, layer0, layer1, freed_blocks, n_freed), s));
 }
 
 static thread_local cudaEvent_t g_pass_events[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
@@ -555,10 +622,13 @@ tria_status tria_compress_pass(const tria_stats *stats, const tria_cache_view *c
   cp.geo = g;
   cp.cache = make_cache_dev(cache, 0, L);
   cp.kept = kept;
-  cp.update_lens = 1;
+  cp.update_lens = g.per_layer ? 0 : 1;
   cp.freed_blocks = freed_blocks;
   cp.n_freed = n_freed;
   if (launch_compact(cp, s) != cudaSuccess) return TRIA_ERR_CUDA;
+  if (g.per_layer &&
+      launch_layer_lens(make_lens(g, cache, 0, L, freed_blocks, n_freed), s) != cudaSuccess)
+    return TRIA_ERR_CUDA;
   return cuda_status(mark(4, s));
 }
 

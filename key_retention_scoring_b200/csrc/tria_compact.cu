@@ -85,7 +85,8 @@ __device__ __forceinline__ void cp_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Length and freed blocks of sequence s, from the kept list of its unit 0.
+// Length and freed blocks of sequence s (one length for all its layers), from
+// the kept list of its unit 0.
 __device__ void update_len(const CompactParams &p, const ItemGeo &g) {
   const Geom &geo = p.geo;
   const int s = g.s;
@@ -95,7 +96,7 @@ __device__ void update_len(const CompactParams &p, const ItemGeo &g) {
     newlen = 0;
     while (newlen < geo.budget && g.kept[newlen] >= 0) ++newlen;
   }
-  if (N > geo.budget && N <= geo.max_seq_len) {
+  if (compresses(geo, N, 0)) {
     if (p.cache.layout == TRIA_LAYOUT_PAGED && p.n_freed != nullptr) {
       const int bs = p.cache.block_size;
       const int keep_blocks = (newlen + bs - 1) / bs;
@@ -197,7 +198,63 @@ __global__ void __launch_bounds__(kCpThreads, 1) compact_kernel(const __grid_con
   cp_wait<0>();
 }
 
+// Per-(sequence, layer) lengths: every compressed (sequence, layer) of the
+// call now holds B_l rows (C > K whenever N - B_l >= 1, so the selection
+// always fills the budget).  The paged blocks are shared by the layers: a call
+// over every layer frees the blocks past the longest new length that held
+// rows of the longest old one.  One block of kLensThreads per sequence.
+constexpr int kLensThreads = 128;
+
+__global__ void __launch_bounds__(kLensThreads) layer_lens_kernel(const __grid_constant__ LensParams p) {
+  const Geom &g = p.geo;
+  const int s = blockIdx.x, t = threadIdx.x;
+  int old_max = 0, new_max = 0, bad = 0;
+  for (int lr = t; lr < g.nl; lr += kLensThreads) {
+    const int n = unit_len(g, s, lr);
+    if (!len_valid(g, n)) {
+      bad = 1;
+      continue;
+    }
+    const int nn = compresses(g, n, lr) ? g.lbudget[lr] : n;
+    old_max = max(old_max, n);
+    new_max = max(new_max, nn);
+    if (nn != n) p.layer_lens[(int64_t)s * g.n_layers + g.layer0 + lr] = nn;
+  }
+  old_max = __reduce_max_sync(kFull, old_max);
+  new_max = __reduce_max_sync(kFull, new_max);
+  bad = __reduce_or_sync(kFull, bad);
+  __shared__ int red[3][kLensThreads / 32];
+  const int w = t >> 5;
+  if ((t & 31) == 0) {
+    red[0][w] = old_max;
+    red[1][w] = new_max;
+    red[2][w] = bad;
+  }
+  __syncthreads();
+  if (t != 0 || !p.paged || p.n_freed == nullptr) return;
+  for (int i = 1; i < kLensThreads / 32; ++i) {
+    old_max = max(old_max, red[0][i]);
+    new_max = max(new_max, red[1][i]);
+    bad |= red[2][i];
+  }
+  int nf = 0;
+  if (p.all_layers && !bad) {
+    const int bs = p.block_size;
+    for (int b = (new_max + bs - 1) / bs; b < (old_max + bs - 1) / bs; ++b) {
+      if (p.freed_blocks != nullptr)
+        p.freed_blocks[(int64_t)s * p.max_blocks + nf] = p.block_table[(int64_t)s * p.max_blocks + b];
+      ++nf;
+    }
+  }
+  p.n_freed[s] = nf;
+}
+
 }  // namespace
+
+cudaError_t launch_layer_lens(const LensParams &p, cudaStream_t st) {
+  layer_lens_kernel<<<(unsigned)p.geo.n_seq, kLensThreads, 0, st>>>(p);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_compact(const CompactParams &p, cudaStream_t st) {
   const int smem = (int)sizeof(CpSmem);

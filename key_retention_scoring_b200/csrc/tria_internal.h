@@ -35,7 +35,15 @@ struct Geom {
   int layer0;
   int n_layers;  // of the model
   int hkv, hq, g;
-  int budget, window, sinks;
+  int budget;    // B_max: kept_idx row length (max over the model's layers)
+  int window, sinks;
+  int trigger;   // max(interval, 1): a unit is compressed when N - B_l >= trigger
+  int per_layer; // lengths per (sequence, layer) (layer_seq_lens)
+  // N of unit (s, lrel) = lens[s * lens_s + lrel * lens_l]
+  const int32_t *lens;
+  int64_t lens_s;
+  int lens_l;
+  int lbudget[TRIA_MAX_LAYERS];  // B_l of call layer lrel (layer0 + lrel)
   int max_seq_len;
   int c_max;     // max_seq_len - window - sinks (>= 1)
   int tiles_max; // upper bound of the scheduling tiles of one unit
@@ -68,6 +76,7 @@ struct WsLayout {
   size_t hdr;         // 256 B: u32 item counter, i32 status flags
   size_t unit_done;   // n_units x u32: finished normalization chunks per unit
   size_t seq_items;   // (n_seq + 1) x i32 prefix of scheduling items per sequence
+  size_t row_items;   // (n_seq x nl + 1) x i32 prefix per (sequence, layer) (per-layer lengths)
   size_t btile;       // n_units x ncol x kCoefK bf16 coefficient tiles
   size_t moments;     // n_units x tiles_max x kRowGroups x g x 2 fp64
   size_t hist;        // n_units x kAggHistBins u32: histogram of the top 12 bits of agg keys
@@ -98,6 +107,7 @@ struct ScoreParams {
   uint32_t *item_counter;
   int32_t *status;
   const int32_t *seq_items;
+  const int32_t *row_items;  // per-layer lengths: prefix per (sequence, layer)
   double *moments;
   float *raw;           // [unit][raw_stride], per candidate G floats
   int64_t raw_stride;
@@ -106,7 +116,6 @@ struct ScoreParams {
 // Normalize-then-max (and selection) kernel parameters.
 struct TailParams {
   Geom geo;
-  const int32_t *seq_lens;
   int32_t *status;
   const double *moments;
   float *raw;
@@ -127,19 +136,18 @@ struct CoefParams {
   const double *w_norm;
   const double *omega;
   const int64_t *query_pos;
-  const int32_t *seq_lens;
   uint16_t *btile;
   uint32_t *item_counter;
   uint32_t *unit_done;
   int32_t *seq_items;
+  int32_t *row_items;
   int32_t *status;
-  int32_t *kept;      // identity rows for units with N <= budget (may be null)
+  int32_t *kept;      // identity rows for units that are not compressed (may be null)
   uint32_t *hist;     // zeroed per unit (may be null)
 };
 
 struct SelectParams {
   Geom geo;
-  const int32_t *seq_lens;
   int32_t *status;
   const float *agg;
   int64_t agg_stride;
@@ -150,7 +158,18 @@ struct CompactParams {
   Geom geo;
   CacheDev cache;
   const int32_t *kept;
-  int update_lens;      // layer1 == n_layers
+  int update_lens;      // layer1 == n_layers (one length per sequence)
+  int32_t *freed_blocks;
+  int32_t *n_freed;
+};
+
+// Per-(sequence, layer) lengths after compaction, and the freed blocks.
+struct LensParams {
+  Geom geo;
+  int32_t *layer_lens;  // [n_seq][n_layers]
+  const int32_t *block_table;
+  int max_blocks, block_size, paged;
+  int all_layers;       // the call covers every layer: blocks may be freed
   int32_t *freed_blocks;
   int32_t *n_freed;
 };
@@ -165,5 +184,17 @@ cudaError_t launch_select(const SelectParams &p, cudaStream_t st);
 bool unit_tail_fits(const Geom &g);
 cudaError_t launch_unit_tail(const TailParams &p, cudaStream_t st);
 cudaError_t launch_compact(const CompactParams &p, cudaStream_t st);
+cudaError_t launch_layer_lens(const LensParams &p, cudaStream_t st);
+
+// Length N of unit (s, lrel) and whether the pass compresses it.
+__host__ __device__ __forceinline__ int unit_len(const Geom &g, int s, int lrel) {
+  return g.lens[(int64_t)s * g.lens_s + (int64_t)lrel * g.lens_l];
+}
+__host__ __device__ __forceinline__ bool len_valid(const Geom &g, int n) {
+  return n >= 0 && n <= g.max_seq_len;
+}
+__host__ __device__ __forceinline__ bool compresses(const Geom &g, int n, int lrel) {
+  return len_valid(g, n) && n - g.lbudget[lrel] >= g.trigger;
+}
 
 }  // namespace tria

@@ -51,49 +51,79 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
   const int lrel = (int)((u / g.hkv) % g.nl);
   const int s = (int)(u / ((int64_t)g.hkv * g.nl));
   const int l = g.layer0 + lrel;
-  const int N = p.seq_lens[s];
-  const bool bad = (N < 0 || N > g.max_seq_len);
+  const int N = unit_len(g, s, lrel);
+  const bool bad = !len_valid(g, N);
+  const bool comp = compresses(g, N, lrel);
   __shared__ double2 rot[kBands];
   __shared__ float cf[TRIA_MAX_GROUP][3 * kBands];
   __shared__ int s_part[kThreads];
 
   if (u == 0) {
     if (t == 0) *p.item_counter = 0u;
-    // items per sequence, prefix over sequences (n_seq <= 1024: <= 4 per thread)
-    const int per = (g.n_seq + kThreads - 1) / kThreads;
-    int local = 0;
-    for (int i = 0; i < per; ++i) {
-      const int sq = t * per + i;
-      if (sq < g.n_seq) {
-        const int n = p.seq_lens[sq];
-        if (n >= 0 && n <= g.max_seq_len && n > g.budget)
-          local += unit_tiles(n, g.window, g.sinks) * g.nl * g.hkv;
+    if (!g.per_layer) {
+      // one length per sequence: items per sequence, prefix over sequences
+      // (n_seq <= 1024: <= 4 per thread)
+      const int per = (g.n_seq + kThreads - 1) / kThreads;
+      int local = 0;
+      for (int i = 0; i < per; ++i) {
+        const int sq = t * per + i;
+        if (sq < g.n_seq) {
+          const int n = unit_len(g, sq, 0);
+          if (compresses(g, n, 0)) local += unit_tiles(n, g.window, g.sinks) * g.nl * g.hkv;
+        }
+      }
+      int total;
+      int run = block_excl_scan<0, kThreads>(local, t, s_part, &total);
+      for (int i = 0; i < per; ++i) {
+        const int sq = t * per + i;
+        if (sq < g.n_seq) {
+          p.seq_items[sq] = run;
+          const int n = unit_len(g, sq, 0);
+          if (compresses(g, n, 0)) run += unit_tiles(n, g.window, g.sinks) * g.nl * g.hkv;
+        }
+      }
+      if (t == 0) p.seq_items[g.n_seq] = total;
+    } else {
+      // a length per (sequence, layer): items per row (s, lrel) = hkv x tiles
+      // of the row's units; prefix over the rows, and over the sequences
+      const int rows = g.n_seq * g.nl;
+      const int per = (rows + kThreads - 1) / kThreads;
+      auto row_n = [&](int r) {
+        const int n = unit_len(g, r / g.nl, r % g.nl);
+        return compresses(g, n, r % g.nl) ? unit_tiles(n, g.window, g.sinks) * g.hkv : 0;
+      };
+      int local = 0;
+      for (int i = 0; i < per; ++i) {
+        const int r = t * per + i;
+        if (r < rows) local += row_n(r);
+      }
+      int total;
+      int run = block_excl_scan<0, kThreads>(local, t, s_part, &total);
+      for (int i = 0; i < per; ++i) {
+        const int r = t * per + i;
+        if (r < rows) {
+          p.row_items[r] = run;
+          if (r % g.nl == 0) p.seq_items[r / g.nl] = run;
+          run += row_n(r);
+        }
+      }
+      if (t == 0) {
+        p.row_items[rows] = total;
+        p.seq_items[g.n_seq] = total;
       }
     }
-    int total;
-    int run = block_excl_scan<0, kThreads>(local, t, s_part, &total);
-    for (int i = 0; i < per; ++i) {
-      const int sq = t * per + i;
-      if (sq < g.n_seq) {
-        p.seq_items[sq] = run;
-        const int n = p.seq_lens[sq];
-        if (n >= 0 && n <= g.max_seq_len && n > g.budget)
-          run += unit_tiles(n, g.window, g.sinks) * g.nl * g.hkv;
-      }
-    }
-    if (t == 0) p.seq_items[g.n_seq] = total;
   }
   if (t == 0) {
     p.unit_done[u] = 0u;
-    if (bad && lrel == 0 && h == 0) atomicOr(p.status, 1);
+    if (bad && h == 0 && (lrel == 0 || g.per_layer)) atomicOr(p.status, 1);
   }
   if (p.hist != nullptr)
     for (int j = t; j < kAggHistBins; j += kThreads) p.hist[u * kAggHistBins + j] = 0u;
-  if (p.kept != nullptr && (bad || N <= g.budget)) {
+  if (p.kept != nullptr && !comp) {
     int32_t *kr = p.kept + u * g.budget;
     for (int j = t; j < g.budget; j += kThreads) kr[j] = (!bad && j < N) ? j : -1;
   }
-  if (bad || N <= g.budget) return;
+  if (!comp) return;
 
   if (g.mode == TRIA_OFFSET_MAX) {
     // max over the offsets: one coefficient vector per (head, offset delta_j)
@@ -223,8 +253,9 @@ __global__ void __launch_bounds__(kThreads) tail_kernel(const __grid_constant__ 
   const int64_t u = blockIdx.x / nch_max;
   const int chunk = (int)(blockIdx.x % nch_max);
   const int s = (int)(u / ((int64_t)geo.nl * geo.hkv));
-  const int N = p.seq_lens[s];
-  if (N < 0 || N > geo.max_seq_len || N <= geo.budget) return;
+  const int lrel = (int)((u / geo.hkv) % geo.nl);
+  const int N = unit_len(geo, s, lrel);
+  if (!compresses(geo, N, lrel)) return;
   const int C = N - geo.window - geo.sinks;
   const int nch = (C + kAggChunk - 1) / kAggChunk;
   if (chunk >= nch) return;
@@ -255,9 +286,11 @@ __global__ void __launch_bounds__(kThreads) tail_kernel(const __grid_constant__ 
   if (!s_last) return;
   for (int i = t; i < kAggHistBins; i += kThreads) ts.hist[i] = __ldcg(gh + i);
   __syncthreads();
-  const int K = geo.budget - geo.window - geo.sinks;
-  select_unit<0, kThreads>(agg, C, K, N, geo.budget, geo.window, geo.sinks,
-                           p.kept + u * geo.budget, ts, sc, true, t);
+  const int B = geo.lbudget[lrel];
+  int32_t *kept = p.kept + u * geo.budget;
+  select_unit<0, kThreads>(agg, C, B - geo.window - geo.sinks, N, B, geo.window, geo.sinks, kept,
+                           ts, sc, true, t);
+  for (int j = B + t; j < geo.budget; j += kThreads) kept[j] = -1;
   __syncthreads();
   if (p.discard_agg) {
     const int64_t lines = ((int64_t)C * 4 + 127) / 128;
@@ -289,13 +322,14 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_tail_kernel(const __grid
   uint32_t *keys = reinterpret_cast<uint32_t *>(list + kListCap);
   const Geom &geo = p.geo;
   const int t = threadIdx.x;
-  const int K = geo.budget - geo.window - geo.sinks;
   for (int64_t u = blockIdx.x; u < geo.n_units; u += gridDim.x) {
     const int s = (int)(u / ((int64_t)geo.nl * geo.hkv));
-    const int N = p.seq_lens[s];
-    // invalid lengths and units within the budget: the coefficient kernel
+    const int lrel = (int)((u / geo.hkv) % geo.nl);
+    const int N = unit_len(geo, s, lrel);
+    // invalid lengths and units left as they are: the coefficient kernel
     // wrote their kept rows and flagged the former
-    if (N < 0 || N > geo.max_seq_len || N <= geo.budget) continue;
+    if (!compresses(geo, N, lrel)) continue;
+    const int B = geo.lbudget[lrel];
     const int C = N - geo.window - geo.sinks;
     unit_norm<G, 0, kUnitThreads>(p.moments + u * geo.tiles_max * kRowGroups * G * 2,
                                   unit_tiles(N, geo.window, geo.sinks), C, t, sc);
@@ -308,8 +342,10 @@ __global__ void __launch_bounds__(kUnitThreads, 1) unit_tail_kernel(const __grid
       const int64_t lines = ((int64_t)C * G * 4 + 127) / 128;
       for (int64_t i = t; i < lines; i += kUnitThreads) discard_line(raw + i * 32);
     }
-    select_keys<kUnitThreads>(keys, C, K, N, geo.budget, geo.window, geo.sinks,
-                              p.kept + u * geo.budget, hist, list, sc, t);
+    int32_t *kept = p.kept + u * geo.budget;
+    select_keys<kUnitThreads>(keys, C, B - geo.window - geo.sinks, N, B, geo.window, geo.sinks,
+                              kept, hist, list, sc, t);
+    for (int j = B + t; j < geo.budget; j += kUnitThreads) kept[j] = -1;
     __syncthreads();
   }
 }
@@ -323,19 +359,21 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const __grid_constant_
   const Geom &geo = p.geo;
   const int64_t u = blockIdx.x;
   const int s = (int)(u / ((int64_t)geo.nl * geo.hkv));
-  const int N = p.seq_lens[s];
+  const int lrel = (int)((u / geo.hkv) % geo.nl);
+  const int N = unit_len(geo, s, lrel);
   int32_t *kept = p.kept + u * geo.budget;
   const int t = threadIdx.x;
-  if (N < 0 || N > geo.max_seq_len || N <= geo.budget) {
-    const bool bad = (N < 0 || N > geo.max_seq_len);
-    if (bad && t == 0 && u == 0) atomicOr(p.status, 1);
+  if (!compresses(geo, N, lrel)) {
+    const bool bad = !len_valid(geo, N);
+    if (bad && t == 0) atomicOr(p.status, 1);
     for (int j = t; j < geo.budget; j += kThreads) kept[j] = (!bad && j < N) ? j : -1;
     return;
   }
   const int C = N - geo.window - geo.sinks;
-  const int K = geo.budget - geo.window - geo.sinks;
-  select_unit<0, kThreads>(p.agg + u * p.agg_stride, C, K, N, geo.budget, geo.window, geo.sinks,
-                           kept, ts, sc, false, t);
+  const int B = geo.lbudget[lrel];
+  select_unit<0, kThreads>(p.agg + u * p.agg_stride, C, B - geo.window - geo.sinks, N, B,
+                           geo.window, geo.sinks, kept, ts, sc, false, t);
+  for (int j = B + t; j < geo.budget; j += kThreads) kept[j] = -1;
 }
 
 }  // namespace

@@ -394,14 +394,32 @@ __device__ void producer(const ScoreParams &p, Smem &sm, int n_items, int lane) 
         if (sm.seq_items[mid] <= it) lo = mid; else hi = mid - 1;
       }
       s = lo;
-      ntiles = (sm.seq_items[s + 1] - sm.seq_items[s]) / units_per_seq;
-      const int rem = it - sm.seq_items[s];
-      const int ul = rem / ntiles;
-      tile = rem % ntiles;
-      lrel = ul / geo.hkv;
-      h = ul % geo.hkv;
-      u = (long long)s * units_per_seq + ul;
-      N = sm.seq_len[s];
+      if (!geo.per_layer) {
+        ntiles = (sm.seq_items[s + 1] - sm.seq_items[s]) / units_per_seq;
+        const int rem = it - sm.seq_items[s];
+        const int ul = rem / ntiles;
+        tile = rem % ntiles;
+        lrel = ul / geo.hkv;
+        h = ul % geo.hkv;
+        N = sm.seq_len[s];
+      } else {
+        // a length per (sequence, layer): the layer is the last row of the
+        // sequence whose first item is at or before this one (rows without
+        // items share their successor's start)
+        const int32_t *ri = p.row_items + (int64_t)s * geo.nl;
+        int cnt = 0;
+        for (int l0 = 0; l0 < geo.nl; l0 += 32) {
+          const int l = l0 + lane;
+          cnt += __popc(__ballot_sync(kFull, l < geo.nl && __ldcg(ri + l) <= it));
+        }
+        lrel = cnt - 1;
+        N = unit_len(geo, s, lrel);
+        ntiles = unit_tiles(N, W, S);
+        const int rem = it - __ldcg(ri + lrel);
+        h = rem / ntiles;
+        tile = rem % ntiles;
+      }
+      u = (long long)s * units_per_seq + lrel * geo.hkv + h;
       tbase = (S / kTileKeys + tile) * kTileKeys;
       const int c_lo = max(S, tbase), c_hi = min(N - W, tbase + kTileKeys);
       sub_first = (c_lo - tbase) / kRows;
@@ -731,7 +749,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) score_tc_kernel(const __grid_co
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   for (int i = tid; i <= geo.n_seq; i += kTcThreads) sm.seq_items[i] = p.seq_items[i];
-  for (int i = tid; i < geo.n_seq; i += kTcThreads) sm.seq_len[i] = p.cache.seq_lens[i];
+  for (int i = tid; i < geo.n_seq; i += kTcThreads) sm.seq_len[i] = unit_len(geo, i, 0);
   if (tid == 0) {
     for (int i = 0; i < Cfg::STAGES; ++i) {
       mbar_init(&sm.full[i], 1);
@@ -1015,7 +1033,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) score_max_kernel(const __grid_c
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   for (int i = tid; i <= geo.n_seq; i += kTcThreads) sm.seq_items[i] = p.seq_items[i];
-  for (int i = tid; i < geo.n_seq; i += kTcThreads) sm.seq_len[i] = p.cache.seq_lens[i];
+  for (int i = tid; i < geo.n_seq; i += kTcThreads) sm.seq_len[i] = unit_len(geo, i, 0);
   if (tid == 0) {
     for (int i = 0; i < Cfg::STAGES; ++i) {
       mbar_init(&sm.full[i], 1);

@@ -35,6 +35,11 @@ design notes of the repository):
   heads sharing a KV head ([P5] sec. 4 "normalize-then-max").
 * Budget B counts every kept row, window W and sinks S included; candidates
   are slots [S, N - W) ([P4] log line n_old = n_kv - window).
+* Budget variants ([P4] runtime: a percentage budget and per-layer budget
+  scales that default to 1.0; [P5] sec. 8: pruning once per window of beta
+  generated tokens): a percentage is of the cache capacity (the rows a
+  sequence can hold); layer l keeps B_l = floor(base * scale_l + 1/2) rows;
+  a unit is compressed only when N - B_l >= max(beta, 1).
 * Exact ties on the aggregated score go to the lower slot; the kept list is in
   ascending slot order; NaN ranks below every number and -0.0 equals +0.0.
 * The optional high-frequency band mask multiplies |mu'_f| only ([P5] sec. 7,
@@ -296,13 +301,62 @@ def compact_rows(rows: np.ndarray, kept: np.ndarray) -> np.ndarray:
     return np.asarray(rows)[np.asarray(kept)]
 
 
+def layer_budgets(n_layers: int, budget: int, capacity: int, budget_pct: float = 0.0,
+                  scales=None) -> np.ndarray:
+    """Budget of every layer.  [P4]'s runtime takes the budget as a
+    percentage ("budget=50%") and per-layer budget scales that default to 1.0
+    (uniform); [P1] gives absolute budgets (2048, 12000).  Readings: the
+    percentage is of the cache capacity `capacity` (the rows one sequence can
+    hold), base = floor(pct * capacity / 100); layer l keeps
+    B_l = floor(base * scale_l + 1/2).  pct and the scales enter as the fp32
+    values a caller passes."""
+    pct = float(np.float32(budget_pct))
+    base = np.floor(pct * float(capacity) / 100.0) if pct > 0.0 else float(budget)
+    out = np.empty(int(n_layers), dtype=np.int64)
+    for l in range(int(n_layers)):
+        sc = 1.0 if scales is None else float(np.float32(scales[l]))
+        out[l] = int(np.floor(base * sc + 0.5))
+    return out
+
+
+def is_compressed(n_tokens: int, budget: int, interval: int = 0) -> bool:
+    """Pruning runs once per window of beta generated tokens ([P5] sec. 8,
+    beta = 128; [P4] runtime log, interval 128): a unit is compressed once it
+    holds at least max(beta, 1) rows more than its budget, else left as is."""
+    return int(n_tokens) - int(budget) >= max(int(interval), 1)
+
+
+def pass_lengths(lens: np.ndarray, budgets: np.ndarray, interval: int = 0) -> np.ndarray:
+    """Lengths [n_seq][n_layers] after one pass: a compressed (sequence,
+    layer) keeps its budget's rows, every other one its length."""
+    lens = np.asarray(lens, dtype=np.int64)
+    out = lens.copy()
+    for s in range(lens.shape[0]):
+        for l in range(lens.shape[1]):
+            if is_compressed(lens[s, l], budgets[l], interval):
+                out[s, l] = budgets[l]
+    return out
+
+
+def freed_block_range(old_lens: np.ndarray, new_lens: np.ndarray, block_size: int):
+    """Paged cache whose blocks hold the rows of every layer: after a pass
+    over all layers of a sequence, the blocks [first, end) are no longer used
+    by any layer: first = ceil(max_l new / bs), end = ceil(max_l old / bs)."""
+    bs = int(block_size)
+    first = -(-int(np.max(new_lens)) // bs)
+    end = -(-int(np.max(old_lens)) // bs)
+    return first, max(first, end)
+
+
 def compress_unit(k_post, positions, p_q, q_center, q_abs_mean, omega, pairing,
-                  budget, window, sinks, log2_max=16, band_mask=None, form="folded"):
+                  budget, window, sinks, log2_max=16, band_mask=None, form="folded",
+                  interval=0):
     """One (sequence, layer, KV head) through the whole pass: scores of the
     candidate slots, normalize-then-max, selection.  Returns a dict with
-    'scores' [G, C], 'agg' [C], 'mean', 'std', 'kept' [min(N, B)]."""
+    'scores' [G, C], 'agg' [C], 'mean', 'std', 'kept' [B] (all N rows when the
+    unit is not compressed)."""
     N = k_post.shape[0]
-    if N <= budget:
+    if not is_compressed(N, budget, interval):
         return {"scores": None, "agg": None, "mean": None, "std": None,
                 "kept": np.arange(N, dtype=np.int64)}
     S_all = unit_scores(k_post, positions, p_q, q_center, q_abs_mean, omega, pairing,

@@ -454,4 +454,55 @@ def pin_whole_unit_pipeline():
     assert list(res2["kept"]) == list(range(15))
 
 
+def pin_budget_variants_golden():
+    """Percentage budget, per-layer scales, the compression interval and the
+    freed blocks, against tests/golden/budget_variants.txt (worked by hand from
+    the runtime log of GitHub issue #10 and article 2607.13051 sec. 8)."""
+    g = _golden_kv("budget_variants.txt")
+    cap, n_kv, w = int(g["capacity"]), int(g["n_kv"]), int(g["window"])
+    b50 = O.layer_budgets(1, 0, cap, budget_pct=50.0)
+    assert list(b50) == [int(g["pct50_budget"])]
+    assert list(O.layer_budgets(3, 0, cap, budget_pct=25.0)) == [int(g["pct25_budget"])] * 3
+    # the logged pass evicts nothing: every one of the n_kv rows stays
+    assert not O.is_compressed(n_kv, int(b50[0]), 128)
+    agg = np.zeros(n_kv - w)
+    assert len(O.select_kept(agg, n_kv, int(b50[0]), w, 0)) == n_kv
+    sc = [float(x) for x in g["scales"].split()]
+    want = [int(x) for x in g["budgets"].split()]
+    assert list(O.layer_budgets(len(sc), int(g["base"]), cap, scales=sc)) == want
+    assert list(O.layer_budgets(4, int(g["base"]), cap)) == [int(g["base"])] * 4
+    assert list(O.layer_budgets(4, int(g["base"]), cap, scales=[1.0] * 4)) == [int(g["base"])] * 4
+    assert list(O.layer_budgets(1, 7, cap, scales=[0.5])) == [int(g["half7"])]
+    assert list(O.layer_budgets(1, 9, cap, scales=[0.5])) == [int(g["half9"])]
+    B = int(g["base"])
+    assert not O.is_compressed(B + 127, B, 128) and O.is_compressed(B + 128, B, 128)
+    assert O.is_compressed(B + 1, B, 0) and not O.is_compressed(B, B, 0)
+    assert O.is_compressed(B + 1, B, 1) and not O.is_compressed(B, B, 1)
+    grow_in = [int(x) for x in g["growth_in"].split()]
+    grow_out = [int(x) for x in g["growth_out"].split()]
+    for n_in, n_out in zip(grow_in, grow_out):
+        assert int(O.pass_lengths(np.array([[n_in]]), np.array([B]), 128)[0, 0]) == n_out
+    old = np.array([2176, 2176])
+    new_a = O.pass_lengths(old[None], np.array([2048, 1024]), 128)[0]
+    assert list(new_a) == [2048, 1024]
+    assert O.freed_block_range(old, new_a, 16) == tuple(int(x) for x in g["freed_a"].split())
+    new_b = O.pass_lengths(old[None], np.array([1024, 1024]), 128)[0]
+    assert O.freed_block_range(old, new_b, 16) == tuple(int(x) for x in g["freed_b"].split())
+
+
+def pin_interval_unit_pipeline():
+    """compress_unit with an interval: a unit short of B + beta rows keeps all
+    of them; at B + beta it is cut to exactly B with window and sinks kept."""
+    rng = np.random.default_rng(31)
+    d, G, theta = 16, 2, 1e4
+    qc, qa, _, k_post, pos, p_q = _random_unit(rng, d, G, 40, O.PAIR_NEOX, theta)
+    omega = O.band_frequencies(d, theta)
+    kw = dict(budget=24, window=6, sinks=1, interval=16)
+    short = O.compress_unit(k_post[:39], pos[:39], p_q, qc, qa, omega, O.PAIR_NEOX, **kw)
+    assert list(short["kept"]) == list(range(39)) and short["agg"] is None
+    full = O.compress_unit(k_post, pos, p_q, qc, qa, omega, O.PAIR_NEOX, **kw)
+    kept = full["kept"]
+    assert len(kept) == 24 and kept[0] == 0 and list(kept[-6:]) == list(range(34, 40))
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -21,11 +21,15 @@ from oracle import tria_oracle as O
 SCORE_RTOL = 1e-4
 
 
-def unit_oracle(w, s: int, layer: int, h: int, k_bits=None, positions=None, form="folded"):
-    """Oracle of one unit of a synth.Workload (reads K rows back unless given)."""
+def unit_oracle(w, s: int, layer: int, h: int, k_bits=None, positions=None, form="folded",
+                budget=None, interval=0, n=None):
+    """Oracle of one unit of a synth.Workload (reads K rows back unless given).
+    budget: the unit's budget (default: the configuration's); n: its length
+    (default: the sequence's)."""
     cfg = w.cfg
+    B = cfg.budget if budget is None else int(budget)
     if k_bits is None:
-        k_bits = w.unit_rows("k", s, layer, h)
+        k_bits = w.unit_rows("k", s, layer, h, n)
     if positions is None:
         positions = w.unit_positions(s, layer, h, len(k_bits))
     k = O.bf16_bits_to_f64(k_bits)
@@ -36,9 +40,11 @@ def unit_oracle(w, s: int, layer: int, h: int, k_bits=None, positions=None, form
     qa = am[layer, h * G:(h + 1) * G].astype(np.float64)
     omega = O.band_frequencies(cfg.head_dim, cfg.theta)
     p_q = int(w.query_pos[s].item())
-    res = O.compress_unit(k, positions, p_q, qc, qa, omega, cfg.pairing, cfg.budget, cfg.window,
-                          cfg.sinks, cfg.offset_log2_max, form=form)
+    res = O.compress_unit(k, positions, p_q, qc, qa, omega, cfg.pairing, B, cfg.window,
+                          cfg.sinks, cfg.offset_log2_max, form=form, interval=interval)
     N = len(k)
+    res["B"] = B
+    res["compressed"] = O.is_compressed(N, B, interval)
     if res["scores"] is not None:
         l1 = O.score_l1_scale(k, positions, qc, qa, omega, cfg.pairing, cfg.offset_log2_max,
                               form="max" if form == "max" else "folded")
@@ -74,26 +80,29 @@ def check_agg(gpu_agg: np.ndarray, ora: dict, where=""):
     return tau
 
 
-def check_kept_same_precision(gpu_kept: np.ndarray, gpu_agg: np.ndarray, N: int, cfg, where=""):
+def check_kept_same_precision(gpu_kept: np.ndarray, gpu_agg: np.ndarray, N: int, cfg, where="",
+                              budget=None):
     """The GPU's kept set equals the oracle's selection applied to the GPU's
     own fp32 agg (the floating point that decides is the same)."""
-    ref = O.select_kept(np.asarray(gpu_agg, dtype=np.float32).astype(np.float64), N, cfg.budget,
+    B = cfg.budget if budget is None else int(budget)
+    ref = O.select_kept(np.asarray(gpu_agg, dtype=np.float32).astype(np.float64), N, B,
                         cfg.window, cfg.sinks)
     got = np.asarray(gpu_kept[: len(ref)])
     assert np.array_equal(got, ref), f"{where}: kept set differs from select(gpu agg)"
-    if len(ref) < cfg.budget:
-        assert np.all(np.asarray(gpu_kept[len(ref):]) == -1)
+    assert np.all(np.asarray(gpu_kept[len(ref):]) == -1)
 
 
 def check_kept_vs_oracle(gpu_kept: np.ndarray, ora: dict, cfg, where=""):
     """Outside the tie band the kept sets agree; inside it any choice with
     |kept| = budget is valid."""
-    N, B, W, S = ora["N"], cfg.budget, cfg.window, cfg.sinks
+    N, B, W, S = ora["N"], ora.get("B", cfg.budget), cfg.window, cfg.sinks
     kept = np.asarray(gpu_kept)
-    if N <= B:
-        assert np.array_equal(kept[:N], np.arange(N)), where
+    if not ora.get("compressed", N > B):
+        n = min(N, len(kept))
+        assert np.array_equal(kept[:n], np.arange(n)) and np.all(kept[n:] == -1), where
         return 0
-    assert len(kept) == B
+    assert np.all(kept[B:] == -1), f"{where}: entries past the unit's budget"
+    kept = kept[:B]
     assert np.all(np.diff(kept) > 0), f"{where}: kept not strictly ascending"
     assert set(range(S)) <= set(kept.tolist()) and set(range(N - W, N)) <= set(kept.tolist())
     K = B - W - S

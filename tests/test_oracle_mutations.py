@@ -160,6 +160,36 @@ def _max_is_min(q_center, k_pre, omega, delta, offsets):
     return np.min(np.sum(mag[..., None, :] * np.cos(ang), axis=-1), axis=-1)
 
 
+def _budget_pct_of_fraction(n_layers, budget, capacity, budget_pct=0.0, scales=None):
+    pct = float(budget_pct)
+    if pct > 0:
+        return _orig["layer_budgets"](n_layers, budget, capacity, 0.0, scales) * 0 + int(pct * capacity)
+    return _orig["layer_budgets"](n_layers, budget, capacity, budget_pct, scales)
+
+
+def _budget_floor_not_round(n_layers, budget, capacity, budget_pct=0.0, scales=None):
+    base = np.floor(float(budget_pct) * capacity / 100.0) if budget_pct > 0 else float(budget)
+    sc = np.ones(n_layers) if scales is None else np.asarray(scales, dtype=np.float32)
+    return np.floor(base * sc).astype(np.int64)
+
+
+def _budget_scales_ignored(n_layers, budget, capacity, budget_pct=0.0, scales=None):
+    return _orig["layer_budgets"](n_layers, budget, capacity, budget_pct, None)
+
+
+def _interval_strict(n_tokens, budget, interval=0):
+    return int(n_tokens) - int(budget) > max(int(interval), 1)
+
+
+def _interval_ignored(n_tokens, budget, interval=0):
+    return int(n_tokens) > int(budget)
+
+
+def _freed_from_shortest_layer(old_lens, new_lens, block_size):
+    bs = int(block_size)
+    return -(-int(np.min(new_lens)) // bs), -(-int(np.max(old_lens)) // bs)
+
+
 _orig = {name: getattr(O, name) for name in dir(O) if callable(getattr(O, name))}
 
 MUTATIONS = {
@@ -191,6 +221,12 @@ MUTATIONS = {
     "calibration Re and Im swapped": ("calibration_stats", _calib_re_im_swapped),
     "offset max taken as the mean": ("s_trig_direct_max", _max_is_mean),
     "offset max taken as the min": ("s_trig_direct_max", _max_is_min),
+    "percentage taken as a fraction": ("layer_budgets", _budget_pct_of_fraction),
+    "layer budget rounded down": ("layer_budgets", _budget_floor_not_round),
+    "layer budget scales ignored": ("layer_budgets", _budget_scales_ignored),
+    "interval needs one row more": ("is_compressed", _interval_strict),
+    "interval ignored": ("is_compressed", _interval_ignored),
+    "freed blocks from the shortest layer": ("freed_block_range", _freed_from_shortest_layer),
 }
 
 
