@@ -15,6 +15,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import sys
@@ -382,6 +383,8 @@ def main():
     }
 
     if not args.no_extras:
+        line["decode_attention"] = decode_attention(T, torch, w, st, cache, prm, ws, kept, restore,
+                                                    cfg, hbm)
         line["run16"] = run16(T, w, st, cache, prm, ws, kept, restore)
         line["calibration"] = calibration(T, torch, hbm)
         line["offset_max"] = offset_max(T, torch, st, cache, cfg, kept, restore, hbm)
@@ -520,6 +523,97 @@ def layer_budgets(T, torch, w, st, cfg, restore, hbm, passes=5):
                                "peak": hbm, "unit": "GB/s",
                                "frac": units * C * 256 / (score_ms * 1e-3) / 1e9 / hbm},
             "kept_rows": kept_rows, "passes": passes}
+
+
+def decode_attention(T, torch, w, st, cache, prm, ws, kept, restore, cfg, hbm, reps=3):
+    """Decode-step attention (tria_decode_attention) of every layer with
+    seeded decode queries at the next position: over the full cache, and over
+    the cache one compression pass pruned to the budget.  Per-layer time is
+    the mean over all layers run back to back from one CUDA graph (the
+    layers' K and V together exceed L2).  Also the share of each head's full-cache attention mass that
+    the kept rows hold, on sampled layers, next to a random kept set of the
+    same size (window included)."""
+    import synth
+
+    L, S, Hq, Hkv, G = cfg.n_layers, cfg.n_seq, cfg.n_q_heads, cfg.n_kv_heads, cfg.group
+    N, B, W = cfg.seq_len, cfg.budget, cfg.window
+    pos = w.query_pos.cpu().numpy() + 1
+    qs = [torch.from_numpy(synth.decode_queries(cfg, l, pos).view(np.int16)).cuda()
+          .view(torch.bfloat16) for l in range(L)]
+    scale = 1.0 / math.sqrt(128.0)
+    out = torch.empty((S, Hq, 128), device="cuda")
+    dws = T.alloc_workspace(T.tria_decode_workspace_size(st, cache))
+    T.tria_read_device_status(dws)
+
+    def per_layer_us():
+        # the layers' launches captured once in a CUDA graph (a decode step
+        # replays it), then replayed `reps` times
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for l in range(L):
+                T.tria_decode_attention(st, cache, l, qs[l], scale, out, dws)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for l in range(L):
+                T.tria_decode_attention(st, cache, l, qs[l], scale, out, dws)
+        graph.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            graph.replay()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(1e3 * a.elapsed_time(b) / L)
+        del graph
+        return statistics.mean(ts)
+
+    restore()
+    torch.cuda.synchronize()
+    sample = sorted({0, L // 3, 2 * L // 3, L - 1})
+    zbuf = torch.empty((S, Hq, w.max_seq_len), device="cuda")
+    full_z = {}
+    for l in sample:
+        T.tria_decode_attention(st, cache, l, qs[l], scale, out, dws, logits=zbuf)
+        full_z[l] = zbuf[:, :, :N].cpu().numpy().astype(np.float64)
+    full_us = per_layer_us()
+    T.tria_compress_pass(st, cache, prm, kept, ws)
+    torch.cuda.synchronize()
+    pruned_us = per_layer_us()
+    if T.tria_read_device_status(dws) != 0:
+        raise RuntimeError("device status flags set (decode attention)")
+    kh = kept.cpu().numpy()
+    rng = np.random.default_rng(0)
+    rec, rnd = [], []
+    for l in sample:
+        for s in range(S):
+            for h in range(Hkv):
+                z = full_z[l][s, h * G:(h + 1) * G]
+                p = np.exp(z - z.max(axis=1, keepdims=True))
+                p /= p.sum(axis=1, keepdims=True)
+                rec.append(float(p[:, kh[s, l, h]].sum(axis=1).mean()))
+                r = np.concatenate([rng.choice(N - W, B - W, replace=False), np.arange(N - W, N)])
+                rnd.append(float(p[:, r].sum(axis=1).mean()))
+    restore()
+    torch.cuda.synchronize()
+    full_bytes = S * Hkv * N * 512
+    pruned_bytes = S * Hkv * B * 512
+    del dws, zbuf
+    return {"workload": f"one decode query per sequence and query head, every layer, over {N} rows "
+                        f"(full) and {B} rows (pruned) per KV head",
+            "full_us_per_layer": full_us, "pruned_us_per_layer": pruned_us,
+            "full_roofline": {"bound": "hbm", "kernel": "decode_kernel + decode_combine_kernel",
+                              "achieved": full_bytes / (full_us * 1e-6) / 1e9, "peak": hbm,
+                              "unit": "GB/s", "frac": full_bytes / (full_us * 1e-6) / 1e9 / hbm,
+                              "algorithmic_bytes": full_bytes},
+            "pruned_gbs": pruned_bytes / (pruned_us * 1e-6) / 1e9,
+            "attention_mass_kept": statistics.mean(rec),
+            "attention_mass_random_same_size": statistics.mean(rnd),
+            "sampled_layers": sample, "reps": reps}
 
 
 def run16(T, w, st, cache, prm, ws, kept, restore):

@@ -402,6 +402,42 @@ tria_status tria_read_device_status(void *workspace, tria_stream_t stream,
  */
 tria_status tria_set_pass_events(void *const *events);
 
+/*
+ * tria_decode_attention - the attention of one decode step over the cached
+ * rows of one layer: the kernel that runs for every generated token, on the
+ * cache that the pass pruned (academ.us article 2607.13051, sec. 8).  For
+ * sequence s, query head qh and its KV head h = qh / G, over the rows
+ * j < N(s, layer) of unit (s, layer, h):
+ *   z_j  = scale * (q . k_j)
+ *   out  = sum_j softmax(z)_j v_j,      lse = log sum_j exp(z_j)
+ * The cached keys carry their rotation already (RoPE at the key's position),
+ * so a row keeps its logit when compaction moves it: the retained rows
+ * reproduce the full-cache logits of the keys they hold (Eq. 3: the phase
+ * depends only on the rotations already applied to q and k).
+ *   q       device bf16 [n_seq][n_q_heads][128], the post-RoPE decode query
+ *           (16-byte aligned, contiguous)
+ *   scale   softmax scale (1/sqrt(128) for standard attention); finite
+ *   out     device fp32 [n_seq][n_q_heads][128]
+ *   lse     optional device fp32 [n_seq][n_q_heads] (natural log; -inf when
+ *           N = 0, with out = 0)
+ *   logits  optional device fp32 [n_seq][n_q_heads][max_seq_len]: z_j at
+ *           j < N (entries j >= N are not written)
+ * N comes from layer_seq_lens when the view has it, else seq_lens; a length
+ * outside [0, max_seq_len] sets status bit 0 and is read as 0.  Paged block
+ * ids outside [0, num_blocks) read as zero rows.  The cache is only read.
+ * Workspace: tria_decode_workspace_size bytes (256-byte aligned), all zero
+ * before its first use (it holds per-unit arrival counts that every call
+ * leaves at zero); its first 256 bytes hold the status flags read by
+ * tria_read_device_status.  Calls that may overlap need separate workspaces.
+ * Errors: INVALID_ARG, UNSUPPORTED (head_dim != 128), WORKSPACE, CUDA.
+ */
+tria_status tria_decode_workspace_size(const tria_stats *stats, const tria_cache_view *cache,
+                                       size_t *bytes);
+tria_status tria_decode_attention(const tria_stats *stats, const tria_cache_view *cache,
+                                  int layer, const void *q, float scale, float *out,
+                                  float *lse, float *logits, void *workspace,
+                                  size_t workspace_bytes, tria_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -31,7 +31,7 @@ EXPORTS = ["tria_status_string", "tria_version", "tria_load_stats", "tria_free_s
            "tria_stats_desc", "tria_workspace_size", "tria_score", "tria_select", "tria_compact",
            "tria_compress_pass", "tria_read_device_status", "tria_set_pass_events",
            "tria_compress_pass_static", "tria_calib_accumulate", "tria_calib_finalize",
-           "tria_layer_budgets"]
+           "tria_layer_budgets", "tria_decode_workspace_size", "tria_decode_attention"]
 STATIC_SCRATCH_BYTES = 32 * 1024 * 1024   # TRIA_STATIC_SCRATCH_BYTES
 
 
@@ -109,6 +109,10 @@ def lib() -> ctypes.CDLL:
                                       _VP, _VP]
     L.tria_layer_budgets.argtypes = [_VP, ctypes.POINTER(CacheView), ctypes.POINTER(Params),
                                      ctypes.POINTER(_I), ctypes.POINTER(_I)]
+    L.tria_decode_workspace_size.argtypes = [_VP, ctypes.POINTER(CacheView),
+                                             ctypes.POINTER(ctypes.c_size_t)]
+    L.tria_decode_attention.argtypes = [_VP, ctypes.POINTER(CacheView), _I, _VP, ctypes.c_float,
+                                        _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP]
     for name in EXPORTS:
         if name not in ("tria_status_string", "tria_version"):
             getattr(L, name).restype = _I
@@ -327,6 +331,26 @@ def tria_calib_finalize(desc, acc, n_tokens, q_mean_re, q_mean_im, q_abs_mean, s
            "tria_calib_finalize")
 
 
+def tria_decode_workspace_size(stats, cache) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().tria_decode_workspace_size(stats.handle, ctypes.byref(cache.view),
+                                            ctypes.byref(out)), "tria_decode_workspace_size")
+    return out.value
+
+
+def tria_decode_attention(stats, cache, layer, q, scale, out, workspace, lse=None, logits=None,
+                          stream=None):
+    """Decode-step attention of layer `layer` over the cached rows:
+    q bf16 [n_seq][n_q_heads][128] (post-RoPE), out fp32 [n_seq][n_q_heads][128];
+    lse fp32 [n_seq][n_q_heads] and logits fp32 [n_seq][n_q_heads][max_seq_len]
+    optional."""
+    _check(lib().tria_decode_attention(stats.handle, ctypes.byref(cache.view), int(layer), _ptr(q),
+                                       float(scale), _ptr(out), _ptr(lse), _ptr(logits),
+                                       _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(),
+                                       _stream(stream)), "tria_decode_attention")
+
+
 def tria_read_device_status(workspace, stream=None) -> int:
     out = ctypes.c_int32()
     _check(lib().tria_read_device_status(_ptr(workspace), _stream(stream), ctypes.byref(out)),
@@ -335,10 +359,10 @@ def tria_read_device_status(workspace, stream=None) -> int:
 
 
 def alloc_workspace(nbytes: int, device="cuda"):
-    """A 256-byte aligned device buffer (torch allocations are)."""
+    """A zeroed, 256-byte aligned device buffer (torch allocations are)."""
     import torch
 
-    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
 def tria_set_pass_events(events):

@@ -369,6 +369,40 @@ def compress_unit(k_post, positions, p_q, q_center, q_abs_mean, omega, pairing,
 
 
 # ----------------------------------------------------------------------------
+# Decode attention over the (pruned) cache
+# ----------------------------------------------------------------------------
+def decode_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
+    """Attention of one decode query per head over a unit's cached rows, the
+    kernel that runs for every generated token on the pruned cache ([P5]
+    sec. 8).  q: [G, d] post-RoPE queries; k, v: [N, d] cached rows (keys
+    carry their RoPE rotation, so no position enters here: [P5] Eq. 3).
+    Returns (out [G, d], lse [G], logits [G, N]) with logits = scale q.k_j,
+    out = sum_j softmax(logits)_j v_j, lse = log sum_j exp(logits_j); N = 0
+    gives out = 0 and lse = -inf."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    z = float(scale) * (q @ k.T)                       # [G, N]
+    if z.shape[1] == 0:
+        return np.zeros((q.shape[0], v.shape[1])), np.full(q.shape[0], -np.inf), z
+    m = z.max(axis=1, keepdims=True)
+    e = np.exp(z - m)
+    tot = e.sum(axis=1, keepdims=True)
+    out = (e / tot) @ v
+    lse = (m + np.log(tot))[:, 0]
+    return out, lse, z
+
+
+def attention_recall(logits: np.ndarray, kept) -> np.ndarray:
+    """Share of each head's full-cache attention mass that falls on the kept
+    rows: sum_{j in kept} softmax(logits)_j, per head ([G, N] logits)."""
+    z = np.asarray(logits, dtype=np.float64)
+    e = np.exp(z - z.max(axis=1, keepdims=True))
+    p = e / e.sum(axis=1, keepdims=True)
+    return p[:, np.asarray(kept, dtype=np.int64)].sum(axis=1)
+
+
+# ----------------------------------------------------------------------------
 # Helpers used by the parity tests
 # ----------------------------------------------------------------------------
 def score_l1_scale(k_post, positions, q_center, q_abs_mean, omega, pairing,

@@ -162,6 +162,31 @@ def host_key_rows(cfg: Config, centers: np.ndarray, s: int, layer: int, h: int,
     return P.f32_to_bf16_bits(post.astype(np.float32))
 
 
+def decode_queries(cfg: Config, layer: int, positions, noise: float = 0.5,
+                   stream_seed: int = 0) -> np.ndarray:
+    """Post-RoPE decode queries of one layer, bf16 bits [n_seq][Hq][128]: the
+    pre-RoPE band f of query head qh is the calibrated center E[q_f] of
+    make_stats plus complex normal noise (per part N(0, noise^2)), rotated to
+    the sequence's query position with the config's pairing and theta."""
+    re, im, _ = make_stats(cfg)
+    pos = np.asarray(positions, dtype=np.int64)
+    S, H = len(pos), cfg.n_q_heads
+    s_i, h_i, f_i = np.meshgrid(np.arange(S), np.arange(H), np.arange(64), indexing="ij")
+    n = P.normals4(f_i, h_i, layer + 256 * s_i, P.STREAM_DECODE_Q, cfg.seed + 977 * stream_seed)
+    zr = re[layer][None].astype(np.float64) + noise * n[0]
+    zi = im[layer][None].astype(np.float64) + noise * n[1]
+    om = cfg.theta ** (-2.0 * np.arange(64) / 128.0)
+    ang = om[None, None, :] * pos[:, None, None].astype(np.float64)
+    cs, sn = np.cos(ang), np.sin(ang)
+    pr, pi = zr * cs - zi * sn, zr * sn + zi * cs
+    out = np.empty((S, H, 128))
+    if cfg.pairing == PAIR_NEOX:
+        out[..., :64], out[..., 64:] = pr, pi
+    else:
+        out[..., 0::2], out[..., 1::2] = pr, pi
+    return P.f32_to_bf16_bits(out.astype(np.float32))
+
+
 # ---------------------------------------------------------------------------
 # device generator
 # ---------------------------------------------------------------------------

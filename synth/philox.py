@@ -27,6 +27,7 @@ STREAM_LENGTHS = 7
 STREAM_BLOCKS = 8
 STREAM_QCAL_CENTER = 9
 STREAM_QCAL_NOISE = 10
+STREAM_DECODE_Q = 11
 
 
 def philox4x32_10(c0, c1, c2, c3, k0, k1=KEY_TAG):

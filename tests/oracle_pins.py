@@ -505,4 +505,52 @@ def pin_interval_unit_pipeline():
     assert len(kept) == 24 and kept[0] == 0 and list(kept[-6:]) == list(range(34, 40))
 
 
+def pin_decode_attention_closed_forms():
+    """Softmax attention by closed forms: one row returns its value and its
+    logit; equal logits average the values; two keys whose logits differ by
+    ln 3 weigh 3/4 and 1/4; a constant added to every logit moves lse by that
+    constant and leaves the output; the row order does not matter; no rows
+    give zero and -inf."""
+    rng = np.random.default_rng(37)
+    d = 8
+    q = rng.normal(size=(2, d))
+    k1, v1 = rng.normal(size=(1, d)), rng.normal(size=(1, d))
+    out, lse, z = O.decode_attention(q, k1, v1, 0.5)
+    assert np.allclose(out, np.repeat(v1, 2, axis=0)) and np.allclose(lse, 0.5 * (q @ k1[0]))
+    kk = np.repeat(k1, 4, axis=0)
+    vv = rng.normal(size=(4, d))
+    out, lse, _ = O.decode_attention(q, kk, vv, 1.0)
+    assert np.allclose(out, np.repeat(vv.mean(axis=0)[None], 2, axis=0))
+    assert np.allclose(lse, q @ k1[0] + np.log(4.0))
+    # logits 0 and ln 3 with scale 1/2: keys 0 and e * 2 ln 3 / (q . e), one head
+    e0 = np.zeros(d)
+    e0[0] = 1.0
+    qh = np.array([[2.0] + [0.0] * (d - 1)])
+    k2 = np.stack([np.zeros(d), e0 * np.log(3.0)])     # q.k = 0, 2 ln 3; scaled 0, ln 3
+    v2 = np.stack([np.full(d, 1.0), np.full(d, -1.0)])
+    out, lse, z = O.decode_attention(qh, k2, v2, 0.5)
+    assert np.allclose(z, [[0.0, np.log(3.0)]])
+    assert np.allclose(out, 0.25 * v2[0] + 0.75 * v2[1]) and np.allclose(lse, np.log(4.0))
+    # a key along q moves every logit of that head by the same amount
+    k3 = rng.normal(size=(6, d))
+    v3 = rng.normal(size=(6, d))
+    o_a, l_a, _ = O.decode_attention(qh, k3, v3, 0.3)
+    o_b, l_b, _ = O.decode_attention(qh, k3 + 1.5 * e0, v3, 0.3)
+    assert np.allclose(o_a, o_b) and np.allclose(l_b - l_a, 0.3 * 2.0 * 1.5)
+    perm = rng.permutation(6)
+    o_c, l_c, _ = O.decode_attention(qh, k3[perm], v3[perm], 0.3)
+    assert np.allclose(o_a, o_c) and np.allclose(l_a, l_c)
+    out, lse, _ = O.decode_attention(q, np.zeros((0, d)), np.zeros((0, d)), 1.0)
+    assert np.all(out == 0) and np.all(np.isneginf(lse))
+
+
+def pin_attention_recall():
+    """All rows kept: 1; none: 0; two rows with logits 0 and ln 3: keeping the
+    second keeps 3/4 of the mass."""
+    z = np.array([[0.0, np.log(3.0)], [1.0, 1.0]])
+    assert np.allclose(O.attention_recall(z, [0, 1]), [1.0, 1.0])
+    assert np.allclose(O.attention_recall(z, []), [0.0, 0.0])
+    assert np.allclose(O.attention_recall(z, [1]), [0.75, 0.5])
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -190,6 +190,38 @@ def _freed_from_shortest_layer(old_lens, new_lens, block_size):
     return -(-int(np.min(new_lens)) // bs), -(-int(np.max(old_lens)) // bs)
 
 
+def _attn_no_scale(q, k, v, scale):
+    return _orig["decode_attention"](q, k, v, 1.0)
+
+
+def _attn_keys_as_values(q, k, v, scale):
+    return _orig["decode_attention"](q, k, k, scale)
+
+
+def _attn_softmax_over_heads(q, k, v, scale):
+    q = np.asarray(q, dtype=np.float64)
+    z = float(scale) * (q @ np.asarray(k, dtype=np.float64).T)
+    if z.shape[1] == 0:
+        return _orig["decode_attention"](q, k, v, scale)
+    e = np.exp(z - z.max(axis=0, keepdims=True))
+    p = e / e.sum(axis=0, keepdims=True)
+    m = z.max(axis=1, keepdims=True)
+    return p @ np.asarray(v, dtype=np.float64), (m + np.log(np.exp(z - m).sum(axis=1, keepdims=True)))[:, 0], z
+
+
+def _attn_lse_without_max(q, k, v, scale):
+    out, lse, z = _orig["decode_attention"](q, k, v, scale)
+    if z.shape[1] == 0:
+        return out, lse, z
+    return out, np.log(np.exp(z - z.max(axis=1, keepdims=True)).sum(axis=1)), z
+
+
+def _recall_of_dropped(logits, kept):
+    z = np.asarray(logits, dtype=np.float64)
+    drop = np.setdiff1d(np.arange(z.shape[1]), np.asarray(kept, dtype=np.int64))
+    return _orig["attention_recall"](logits, drop)
+
+
 _orig = {name: getattr(O, name) for name in dir(O) if callable(getattr(O, name))}
 
 MUTATIONS = {
@@ -227,6 +259,11 @@ MUTATIONS = {
     "interval needs one row more": ("is_compressed", _interval_strict),
     "interval ignored": ("is_compressed", _interval_ignored),
     "freed blocks from the shortest layer": ("freed_block_range", _freed_from_shortest_layer),
+    "attention without the scale": ("decode_attention", _attn_no_scale),
+    "attention returns keys": ("decode_attention", _attn_keys_as_values),
+    "softmax over the heads": ("decode_attention", _attn_softmax_over_heads),
+    "lse without the max": ("decode_attention", _attn_lse_without_max),
+    "recall of the dropped rows": ("attention_recall", _recall_of_dropped),
 }
 
 
