@@ -45,6 +45,10 @@ constexpr int kPart = 132;                     // per (head, partial): o[128], m
 constexpr int kMaxSplits = 160;                // blocks per (sequence, KV head), at most
 constexpr size_t kDecHeader = 256;
 constexpr float kLn2 = 0.6931471805599453f;
+// a head's running maximum (base 2) moves only when a tile exceeds it by more
+// than this, so most tiles skip rescaling the accumulators; the weights then
+// stay below 2^kRescale, well inside fp32 and bf16
+constexpr float kRescale = 8.f;
 
 struct DecodeParams {
   const uint16_t *k, *v;
@@ -138,7 +142,7 @@ __device__ __forceinline__ uint32_t tile_off(int r, int c) {
 // (each lane holds two rows of heads gid and gid + 8), then O += P V with P
 // as bf16 hi + lo (V through ldmatrix.trans).  The block's warps then merge
 // their (o, m, l) in shared memory into the block's partial.
-template <int G>
+template <int G, int LAYOUT>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t sm_dec[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -183,19 +187,29 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     }
     // tile rows [r0, r0 + 16) of K and V into stage stg; rows past the range
     // and rows of invalid blocks are zero
+    // contiguous layout: this lane's first row of a tile, then a fixed stride
+    const int64_t unit_off = (int64_t)s * p.s_seq + (int64_t)h * p.s_head + (lane & 15) * 8;
     auto load_tile = [&](int r0, int stg) {
       const uint32_t kt = ring + (uint32_t)(stg * 2 * kTileBytes), vt = kt + kTileBytes;
+      const bool full = r0 + kWTile <= r_end;
 #pragma unroll
       for (int i = 0; i < kWTile / 2; ++i) {
         const int row = i * 2 + (lane >> 4), c = lane & 15;
         const int r = r0 + row;
-        bool ok = false;
-        int64_t off = 0;
-        if (r < r_end) off = dec_row(p, s, h, r, ok);
         const uint32_t so = tile_off(row, c);
+        bool ok;
+        int64_t off;
+        if (LAYOUT == TRIA_LAYOUT_CONTIGUOUS) {
+          ok = full || r < r_end;
+          off = unit_off + (int64_t)r * p.s_tok;
+        } else {
+          ok = false;
+          off = 0;
+          if (full || r < r_end) off = dec_row(p, s, h, r, ok) + c * 8;
+        }
         if (ok) {
-          cp_async16(kt + so, p.k + off + c * 8);
-          cp_async16(vt + so, p.v + off + c * 8);
+          cp_async16(kt + so, p.k + off);
+          cp_async16(vt + so, p.v + off);
         } else {
           asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(kt + so), "r"(0u) : "memory");
           asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vt + so), "r"(0u) : "memory");
@@ -232,48 +246,62 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
           mma16816(sc[nt], qa[2 * kp + 1], b2, b3);
         }
       }
-      // rows past the range drop out; logits to the caller; base-2 scale
+      // logits to the caller; base-2 scale; rows past the range drop out
+      if (p.logits != nullptr) {
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int row = r0 + nt * 8 + 2 * tig + (e & 1);
-          const int head = (e < 2) ? gid : gid + 8;
-          const bool valid = row < r_end;
-          if (p.logits != nullptr && valid && head < G)
-            p.logits[((int64_t)s * p.hq + qh0 + head) * p.max_seq_len + row] = sc[nt][e] * p.scale;
-          sc[nt][e] = valid ? sc[nt][e] * p.qscale : -INFINITY;
-        }
+          for (int e = 0; e < 4; ++e) {
+            const int row = r0 + nt * 8 + 2 * tig + (e & 1);
+            const int head = (e < 2) ? gid : gid + 8;
+            if (row < r_end && head < G)
+              p.logits[((int64_t)s * p.hq + qh0 + head) * p.max_seq_len + row] = sc[nt][e] * p.scale;
+          }
       }
-      // online softmax: the tile maximum of each head over the 4 lanes of its group
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[nt][e] *= p.qscale;
+      if (r0 + kWTile > r_end) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (r0 + nt * 8 + 2 * tig + (e & 1) >= r_end) sc[nt][e] = -INFINITY;
+      }
+      // online softmax: the tile maximum of each head over the 4 lanes of its
+      // group; the running maximum moves (and the accumulators are rescaled)
+      // only when the tile exceeds it by more than kRescale
       float t0 = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
       float t1 = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
       t0 = fmaxf(t0, __shfl_xor_sync(kFull, t0, 1));
       t0 = fmaxf(t0, __shfl_xor_sync(kFull, t0, 2));
       t1 = fmaxf(t1, __shfl_xor_sync(kFull, t1, 1));
       t1 = fmaxf(t1, __shfl_xor_sync(kFull, t1, 2));
-      const float mn0 = fmaxf(m0, t0), mn1 = fmaxf(m1, t1);
-      const float a0 = exp2f(m0 - mn0), a1 = exp2f(m1 - mn1);  // 0 at the first tile
-      m0 = mn0;
-      m1 = mn1;
-      float sum0 = 0.f, sum1 = 0.f;
+      const bool up0 = t0 > m0 + kRescale, up1 = t1 > m1 + kRescale;  // always at the first tile
+      if (__any_sync(kFull, up0 || up1)) {
+        const float mn0 = up0 ? t0 : m0, mn1 = up1 ? t1 : m1;
+        const float a0 = exp2f(m0 - mn0), a1 = exp2f(m1 - mn1);  // 0 at the first tile
+        m0 = mn0;
+        m1 = mn1;
+        l0 *= a0;
+        l1 *= a1;
+#pragma unroll
+        for (int dt = 0; dt < 16; ++dt) {
+          o[dt][0] *= a0;
+          o[dt][1] *= a0;
+          o[dt][2] *= a1;
+          o[dt][3] *= a1;
+        }
+      }
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
-        sc[nt][0] = exp2f(sc[nt][0] - mn0);
-        sc[nt][1] = exp2f(sc[nt][1] - mn0);
-        sc[nt][2] = exp2f(sc[nt][2] - mn1);
-        sc[nt][3] = exp2f(sc[nt][3] - mn1);
-        sum0 += sc[nt][0] + sc[nt][1];
-        sum1 += sc[nt][2] + sc[nt][3];
-      }
-      l0 = fmaf(l0, a0, sum0);
-      l1 = fmaf(l1, a1, sum1);
-#pragma unroll
-      for (int dt = 0; dt < 16; ++dt) {
-        o[dt][0] *= a0;
-        o[dt][1] *= a0;
-        o[dt][2] *= a1;
-        o[dt][3] *= a1;
+        sc[nt][0] = exp2f(sc[nt][0] - m0);
+        sc[nt][1] = exp2f(sc[nt][1] - m0);
+        sc[nt][2] = exp2f(sc[nt][2] - m1);
+        sc[nt][3] = exp2f(sc[nt][3] - m1);
+        l0 += sc[nt][0] + sc[nt][1];
+        l1 += sc[nt][2] + sc[nt][3];
       }
       // O += P V: one k-step of 16 rows, 16 column tiles of 8 dims
       uint32_t ah[4], al[4];
@@ -416,12 +444,19 @@ cudaError_t launch_decode_g(const DecodeParams &p, cudaStream_t st) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (attr_dev != dev) {
-    e = cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
+    e = cudaFuncSetAttribute(decode_kernel<G, TRIA_LAYOUT_CONTIGUOUS>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(decode_kernel<G, TRIA_LAYOUT_PAGED>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
   const int64_t blocks = (int64_t)p.n_seq * p.hkv * p.splits;
-  decode_kernel<G><<<(unsigned)blocks, kDecThreads, kDecSmem, st>>>(p);
+  if (p.layout == TRIA_LAYOUT_CONTIGUOUS)
+    decode_kernel<G, TRIA_LAYOUT_CONTIGUOUS><<<(unsigned)blocks, kDecThreads, kDecSmem, st>>>(p);
+  else
+    decode_kernel<G, TRIA_LAYOUT_PAGED><<<(unsigned)blocks, kDecThreads, kDecSmem, st>>>(p);
   return cudaGetLastError();
 }
 
