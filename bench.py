@@ -606,7 +606,7 @@ def decode_attention(T, torch, w, st, cache, prm, ws, kept, restore, cfg, hbm, r
     return {"workload": f"one decode query per sequence and query head, every layer, over {N} rows "
                         f"(full) and {B} rows (pruned) per KV head",
             "full_us_per_layer": full_us, "pruned_us_per_layer": pruned_us,
-            "full_roofline": {"bound": "hbm", "kernel": "decode_kernel + decode_combine_kernel",
+            "full_roofline": {"bound": "hbm", "kernel": "decode_kernel",
                               "achieved": full_bytes / (full_us * 1e-6) / 1e9, "peak": hbm,
                               "unit": "GB/s", "frac": full_bytes / (full_us * 1e-6) / 1e9 / hbm,
                               "algorithmic_bytes": full_bytes},

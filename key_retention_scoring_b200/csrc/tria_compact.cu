@@ -11,7 +11,8 @@
 //   * chunk c + A is read before chunk c is written: its sources are at or
 //     above its first destination, above every destination of chunk c.
 // One block per SM walks the chunks of its items (unit, K or V) as one
-// stream, reading A = 2 chunks ahead of the chunk it writes.  A thread always
+// stream, reading A = 2 chunks ahead of the chunk it writes; an item has
+// ceil(B_l / kCpRows) chunks for the budget B_l of its layer.  A thread always
 // handles the same rows and 16-byte pieces of a chunk: it loads their kept
 // entries one chunk before it starts their copies, keeps their sources in
 // shared memory for the write-back, and writes back exactly the pieces it
@@ -123,36 +124,54 @@ __global__ void __launch_bounds__(kCpThreads, 1) compact_kernel(const __grid_con
   const int t = threadIdx.x;
   const int piece = t % kPieces, rr = t / kPieces;
   const int cap = geo.max_seq_len;
-  const int nch = (geo.budget + kCpRows - 1) / kCpRows;
   const int64_t n_items = geo.n_units * 2;
   const int64_t my_items =
       (blockIdx.x < n_items) ? (n_items - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  const int64_t total = my_items * nch;  // chunks of this block, item-major
+  // The block's items form one stream of chunks, item-major; an item has
+  // ceil(B_l / kCpRows) chunks for the budget B_l of its layer.  A cursor is
+  // a position in that stream.
+  struct Cur {
+    int64_t i;  // item ordinal within the block (>= my_items: past the end)
+    int c, nch;
+  };
+  auto item_of = [&](int64_t i) { return (int64_t)blockIdx.x + i * gridDim.x; };
+  auto chunks_of = [&](int64_t i) {
+    const int64_t u = item_of(i) >> 1;
+    const int lrel = (int)((u / geo.hkv) % geo.nl);
+    return (geo.lbudget[lrel] + kCpRows - 1) / kCpRows;
+  };
+  auto start = [&]() {
+    Cur q{0, 0, 0};
+    if (my_items > 0) q.nch = chunks_of(0);
+    return q;
+  };
+  auto advance = [&](Cur &q) {
+    if (++q.c >= q.nch) {
+      ++q.i;
+      q.c = 0;
+      q.nch = q.i < my_items ? chunks_of(q.i) : 0;
+    }
+  };
 
-  // kept entries (raw) of this thread's rows of stream chunk k
-  auto fetch = [&](int64_t k, int (&kv)[kRowsPerThread]) {
-    if (k < total) {
-      const int64_t it = blockIdx.x + (k / nch) * gridDim.x;
-      const int c = (int)(k % nch);
-      const int32_t *kept = p.kept + (it >> 1) * geo.budget;
+  // kept entries (raw) of this thread's rows of chunk q
+  auto fetch = [&](const Cur &q, int (&kv)[kRowsPerThread]) {
+    if (q.i < my_items) {
+      const int32_t *kept = p.kept + (item_of(q.i) >> 1) * geo.budget;
 #pragma unroll
       for (int e = 0; e < kRowsPerThread; ++e) {
-        const int j = c * kCpRows + rr + e * kRowStep;
+        const int j = q.c * kCpRows + rr + e * kRowStep;
         kv[e] = (j < geo.budget) ? __ldg(kept + j) : -1;
       }
     }
   };
-  // copies of this thread's pieces of stream chunk k into buffer k % depth
-  // (one commit group per chunk, empty past the end)
-  auto issue = [&](int64_t k, const int (&kv)[kRowsPerThread]) {
-    if (k < total) {
-      const int64_t it = blockIdx.x + (k / nch) * gridDim.x;
-      const int c = (int)(k % nch);
-      const ItemGeo g = item_geo(p, it);
-      const int b = (int)(k % kCpDepth);
+  // copies of this thread's pieces of chunk q into buffer b (one commit
+  // group per chunk, empty past the end)
+  auto issue = [&](const Cur &q, int b, const int (&kv)[kRowsPerThread]) {
+    if (q.i < my_items) {
+      const ItemGeo g = item_geo(p, item_of(q.i));
 #pragma unroll
       for (int e = 0; e < kRowsPerThread; ++e) {
-        const int r = rr + e * kRowStep, j = c * kCpRows + r;
+        const int r = rr + e * kRowStep, j = q.c * kCpRows + r;
         const int v = kv[e];
         const int src = (j >= geo.budget || v == j || v < 0 || v >= cap || j >= cap) ? -1 : v;
         if (piece == 0) sm.src[b][r] = src;
@@ -166,23 +185,28 @@ __global__ void __launch_bounds__(kCpThreads, 1) compact_kernel(const __grid_con
   };
 
   int kv[kRowsPerThread];
+  Cur fc = start();  // next chunk to fetch
   for (int k = 0; k < kCpAhead; ++k) {
-    fetch(k, kv);
-    issue(k, kv);
+    fetch(fc, kv);
+    issue(fc, k % kCpDepth, kv);
+    advance(fc);
   }
-  fetch(kCpAhead, kv);
-  for (int64_t k = 0; k < total; ++k) {
-    issue(k + kCpAhead, kv);
-    fetch(k + kCpAhead + 1, kv);  // used at the next iteration
+  Cur pend = fc;  // fetched, to be issued at the next iteration
+  fetch(pend, kv);
+  advance(fc);
+  Cur wc = start();  // chunk to write back
+  for (int64_t k = 0; wc.i < my_items; ++k) {
+    issue(pend, (int)((k + kCpAhead) % kCpDepth), kv);
+    pend = fc;
+    fetch(pend, kv);  // used at the next iteration
+    advance(fc);
     cp_wait<kCpAhead>();  // this thread's copies of chunk k have landed
     __syncthreads();      // ... and every other thread's
-    const int64_t it = blockIdx.x + (k / nch) * gridDim.x;
-    const int c = (int)(k % nch);
-    const ItemGeo g = item_geo(p, it);
+    const ItemGeo g = item_geo(p, item_of(wc.i));
     const int b = (int)(k % kCpDepth);
 #pragma unroll
     for (int e = 0; e < kRowsPerThread; ++e) {
-      const int r = rr + e * kRowStep, j = c * kCpRows + r;
+      const int r = rr + e * kRowStep, j = wc.c * kCpRows + r;
       // the row's source, recorded (and now read) by the row's piece-0 thread
       const int mine = (piece == 0) ? sm.src[b][r] : 0;
       const int src = __shfl_sync(kFull, mine, (threadIdx.x & 31) & ~(kPieces - 1));
@@ -193,7 +217,8 @@ __global__ void __launch_bounds__(kCpThreads, 1) compact_kernel(const __grid_con
       }
     }
     // sequence length / freed blocks: once per sequence, after the last layer
-    if (c == nch - 1 && p.update_lens && g.part == 0 && g.ul == 0 && t == 0) update_len(p, g);
+    if (wc.c == wc.nch - 1 && p.update_lens && g.part == 0 && g.ul == 0 && t == 0) update_len(p, g);
+    advance(wc);
   }
   cp_wait<0>();
 }
