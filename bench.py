@@ -149,7 +149,7 @@ def oracle_unit_keys_per_s(cfg, seconds: float, max_units: int = 64):
     N = int(synth.seq_lengths(cfg)[0])
     spent, keys, units = 0.0, 0, 0
     rng = np.random.default_rng(0)
-    while spent < seconds and units < max_units:
+    while units == 0 or (spent < seconds and units < max_units):  # at least one unit
         l, h = int(rng.integers(cfg.n_layers)), int(rng.integers(cfg.n_kv_heads))
         bits = synth.host_key_rows(cfg, centers, 0, l, h, np.arange(N))
         k = O.bf16_bits_to_f64(bits)

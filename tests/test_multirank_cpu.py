@@ -73,3 +73,20 @@ def test_reference_arm_rank_gating(capsys, monkeypatch):
     # a non-zero rank prints nothing and exits 0 without work
     assert bench.run_reference(A(), 1, 2) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_on_rank0(capsys):
+    """Rank 0 times the oracle on one unit per step and prints the contract's
+    JSON line (the tiny configuration keeps this to a second)."""
+    import json
+
+    import bench
+
+    class A:
+        steps, warmup, config = 2, 1, 0
+
+    assert bench.run_reference(A(), 0, 1) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["steps"] == 2
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
