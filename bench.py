@@ -236,6 +236,10 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, run16 and CPU baseline")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the workload's layer count (small profiling cases)")
+    ap.add_argument("--only-extra", default="",
+                    choices=["", "decode_attention", "offset_max", "layer_budgets", "calibration"],
+                    help="after the warm-up passes run just this extra and print its result "
+                         "(profiling of one kernel on a small case)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -307,6 +311,18 @@ def main():
     torch.cuda.synchronize()
     if T.tria_read_device_status(ws) != 0:
         raise RuntimeError("device status flags set")
+    if args.only_extra:
+        hbm, _ = peaks()
+        run = {"decode_attention": lambda: decode_attention(T, torch, w, st, cache, prm, ws, kept,
+                                                            restore, cfg, hbm),
+               "offset_max": lambda: offset_max(T, torch, st, cache, cfg, kept, restore, hbm),
+               "layer_budgets": lambda: layer_budgets(T, torch, w, st, cfg, restore, hbm),
+               "calibration": lambda: calibration(T, torch, hbm)}[args.only_extra]
+        res = run()
+        st.free()
+        if rank == 0:
+            print(json.dumps({"extra": args.only_extra, "config": config_desc(cfg), **res}), flush=True)
+        return 0
     # moved rows of one pass (for the compaction bytes)
     kh = kept.cpu().numpy()
     moved = int(np.sum(kh != np.arange(B)[None, None, None, :]))
