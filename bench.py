@@ -136,8 +136,9 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # oracle (CPU baseline and reference arm)
 # ---------------------------------------------------------------------------
-def oracle_unit_keys_per_s(cfg, seconds: float, max_units: int = 64):
-    """Time the fp64 oracle (folded form, normalize-then-max, selection) on
+def oracle_unit_keys_per_s(cfg, seconds: float, max_units: int = 64, form: str = "folded"):
+    """Time the fp64 oracle (normalize-then-max and selection after the
+    scores in `form`: the folded Eq. 7 or the direct 17-offset Eq. 4) on
     units of the workload generated on the host with the same recipe."""
     import synth
     from oracle import tria_oracle as O
@@ -157,7 +158,7 @@ def oracle_unit_keys_per_s(cfg, seconds: float, max_units: int = 64):
         qa = am[l, h * G:(h + 1) * G].astype(np.float64)
         t0 = time.perf_counter()
         O.compress_unit(k, np.arange(N), N - 1, qc, qa, omega, cfg.pairing, cfg.budget,
-                        cfg.window, cfg.sinks, cfg.offset_log2_max)
+                        cfg.window, cfg.sinks, cfg.offset_log2_max, form=form)
         spent += time.perf_counter() - t0
         keys += N
         units += 1
@@ -408,7 +409,13 @@ def main():
         line["e2e"] = e2e(T, torch, w, st, cache, prm, ws, kept, restore, args.e2e_steps, keys, world)
         if rank == 0 and world == 1:
             v, n_units, spent = oracle_unit_keys_per_s(cfg, args.cpu_seconds)
+            # the direct 17-offset form (Eq. 4), the reference-style scorer,
+            # on a bounded sample of the same workload
+            vd, nd_units, spent_d = oracle_unit_keys_per_s(cfg, 0.0, max_units=1, form="direct")
             line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                    "direct_form": {"value": vd, "unit": UNIT, "cores": 1,
+                                                    "sample": f"{nd_units} unit of {N} keys, "
+                                                              f"{spent_d:.1f} s, 17 offsets per band"},
                                     "sample": f"{n_units} units of {N} keys (G={cfg.group}), "
                                               f"{spent:.1f} s, fp64 numpy (single thread), "
                                               "folded form + z-norm + selection"}
