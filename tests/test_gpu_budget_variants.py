@@ -37,7 +37,8 @@ def _stats(w):
     return T.tria_load_stats(desc, *w.stats)
 
 
-def run_variant(cfg, layer_lens=None, scales=None, pct=0.0, interval=0, split_layers=None):
+def run_variant(cfg, layer_lens=None, scales=None, pct=0.0, interval=0, split_layers=None,
+                offset_reduce=0):
     """One fused pass with the given budget variant; every unit checked
     against the oracle with its own budget and length: kept set, compacted
     K/V bytes and positions, the new lengths and the freed paged blocks.
@@ -54,7 +55,7 @@ def run_variant(cfg, layer_lens=None, scales=None, pct=0.0, interval=0, split_la
         else:
             lens = np.repeat(w.lens.astype(np.int64)[:, None], L, axis=1)
         cache = T.Cache.from_workload(w, layer_seq_lens=d_ll)
-        prm = T.params(cfg.budget, cfg.window, cfg.sinks, budget_pct=pct,
+        prm = T.params(cfg.budget, cfg.window, cfg.sinks, offset_reduce, budget_pct=pct,
                        layer_budget_scales=scales, interval=interval)
         budgets, bmax = T.tria_layer_budgets(st, cache, prm)
         want_b = O.layer_budgets(L, cfg.budget, w.max_seq_len, pct, scales)
@@ -68,7 +69,8 @@ def run_variant(cfg, layer_lens=None, scales=None, pct=0.0, interval=0, split_la
                     pos = w.unit_positions(s, l, h, n)
                     saved[(s, l, h)] = (kb, w.unit_rows("v", s, l, h, n), pos)
                     oras[(s, l, h)] = PH.unit_oracle(w, s, l, h, k_bits=kb, positions=pos,
-                                                     budget=budgets[l], interval=interval, n=n)
+                                                     budget=budgets[l], interval=interval, n=n,
+                                                     form="max" if offset_reduce else "folded")
         ws = T.alloc_workspace(T.tria_workspace_size(st, cache, prm))
         T.tria_read_device_status(ws)
         sep = {}
@@ -221,3 +223,11 @@ def test_budget_variant_validation():
         assert status(nothing) == 1
     finally:
         st.free()
+
+
+def test_layer_scales_max_over_offsets():
+    # the max-over-offsets scorer with per-layer budgets and lengths
+    cfg = synth.CONFIGS[2].scaled(n_layers=2, seq_len=4096)
+    lens = np.array([[4096, 3000]])
+    run_variant(cfg, layer_lens=lens, scales=[1.0, 0.5], split_layers=(0, 2),
+                offset_reduce=T.OFFSET_MAX)
