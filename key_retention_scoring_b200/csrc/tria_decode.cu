@@ -118,6 +118,14 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// transpose of an 8x8 b16 matrix held one row pair per lane (lane: row
+// lane / 4, columns 2 (lane % 4), + 1)
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
 // two weights as bf16 pairs hi + lo (hi = bf16(x), lo = bf16(x - hi)): the
 // product with a bf16 value then keeps ~16 bits of the weight
 __device__ __forceinline__ void split2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
@@ -135,13 +143,16 @@ __device__ __forceinline__ uint32_t tile_off(int r, int c) {
 }
 
 // Warp-level flash decoding on the tensor cores (mma.sync m16n8k16, bf16 in,
-// fp32 accumulate).  The G query heads are the M side (zero rows past G);
-// each warp owns a contiguous range of the unit's rows, streamed through its
-// own ring of 16-row K and V tiles (cp.async, 3 in flight).  Per tile:
-// S^T = Q K^T (2 column tiles x 8 k-steps), the online softmax in registers
-// (each lane holds two rows of heads gid and gid + 8), then O += P V with P
-// as bf16 hi + lo (V through ldmatrix.trans).  The block's warps then merge
-// their (o, m, l) in shared memory into the block's partial.
+// fp32 accumulate).  Each warp owns a contiguous range of the unit's rows,
+// streamed through its own ring of 16-row K and V tiles (cp.async, 3 in
+// flight).  Per tile and 8-head column tile: S = K Q^T with the 16 rows as
+// M and the heads as N (K fragments straight from ldmatrix, Q^T fragments in
+// registers); the online softmax in registers (a lane holds rows gid and
+// gid + 8 of heads 2 tig and 2 tig + 1); then O^T += V^T P^T with the dims
+// as M (V^T through ldmatrix.trans) and P^T as B, each 8x8 block of P
+// transposed in registers by movmatrix and split into bf16 hi + lo.  The
+// block's warps then merge their (o, m, l) in shared memory into the
+// block's partial.
 template <int G, int LAYOUT>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t sm_dec[];
@@ -166,29 +177,43 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
   const int per_block = per * kDecWarps;
   if (sp * per_block >= n) return;  // the whole block is past the rows (uniform)
   const uint32_t ring = (uint32_t)__cvta_generic_to_shared(sm_dec + warp * kWarpSmem);
+  constexpr int NT = (G + 7) / 8;  // 8-head column tiles
 
-  float o[16][4];
+  // O^T accumulators: o[nt][mt] holds (dim 16 mt + gid, heads 8 nt + 2 tig,
+  // + 1) and (dim 16 mt + gid + 8, the same heads)
+  float o[NT][8][4];
 #pragma unroll
-  for (int dt = 0; dt < 16; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+  // running maximum (base 2) and lane-partial sum of heads 8 nt + 2 tig + e
+  float m[NT][2], l[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    m[nt][0] = m[nt][1] = -INFINITY;
+    l[nt][0] = l[nt][1] = 0.f;
+  }
 
   if (r_begin < r_end) {
-    // A fragments of the query per k-step: heads gid, gid + 8 (zero past G)
-    uint32_t qa[8][4];
+    // B fragments of the query per k-step: head 8 nt + gid (zero past G),
+    // dims 16 ks + 2 tig, + 1 and 16 ks + 8 + 2 tig, + 1
+    uint32_t qb[NT][8][2];
     {
       const uint32_t *q32 = reinterpret_cast<const uint32_t *>(p.q + ((int64_t)s * p.hq + qh0) * 128);
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        qa[ks][0] = gid < G ? q32[gid * 64 + ks * 8 + tig] : 0u;
-        qa[ks][1] = gid + 8 < G ? q32[(gid + 8) * 64 + ks * 8 + tig] : 0u;
-        qa[ks][2] = gid < G ? q32[gid * 64 + ks * 8 + 4 + tig] : 0u;
-        qa[ks][3] = gid + 8 < G ? q32[(gid + 8) * 64 + ks * 8 + 4 + tig] : 0u;
+      for (int nt = 0; nt < NT; ++nt) {
+        const int hd = nt * 8 + gid;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          qb[nt][ks][0] = hd < G ? q32[hd * 64 + ks * 8 + tig] : 0u;
+          qb[nt][ks][1] = hd < G ? q32[hd * 64 + ks * 8 + 4 + tig] : 0u;
+        }
       }
     }
-    // tile rows [r0, r0 + 16) of K and V into stage stg; rows past the range
-    // and rows of invalid blocks are zero
     // contiguous layout: this lane's first row of a tile, then a fixed stride
     const int64_t unit_off = (int64_t)s * p.s_seq + (int64_t)h * p.s_head + (lane & 15) * 8;
+    // tile rows [r0, r0 + 16) of K and V into stage stg; rows past the range
+    // and rows of invalid blocks are zero
     auto load_tile = [&](int r0, int stg) {
       const uint32_t kt = ring + (uint32_t)(stg * 2 * kTileBytes), vt = kt + kTileBytes;
       const bool full = r0 + kWTile <= r_end;
@@ -223,6 +248,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
       if (i < ntiles) load_tile(r_begin + i * kWTile, i);
       asm volatile("cp.async.commit_group;" ::: "memory");
     }
+    const int mi = lane >> 3;  // the 8x8 matrix this lane addresses in an ldmatrix.x4
     for (int it = 0; it < ntiles; ++it) {
       const int r0 = r_begin + it * kWTile;
       if (it + kWStages - 1 < ntiles)
@@ -232,101 +258,111 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
       __syncwarp();
       const uint32_t kt = ring + (uint32_t)((it % kWStages) * 2 * kTileBytes), vt = kt + kTileBytes;
 
-      // S^T = Q K^T over the tile's 2 column tiles of 8 rows
-      float sc[2][4];
+      // S = K Q^T: 16 rows x 8 heads per column tile, 8 k-steps; the K
+      // fragments (rows gid, gid + 8) come straight from ldmatrix
+      float sc[NT][4];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+      for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
 #pragma unroll
-        for (int kp = 0; kp < 4; ++kp) {
-          const int row = nt * 8 + (lane & 7);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(kt + tile_off(row, kp * 4 + (lane >> 3)), b0, b1, b2, b3);
-          mma16816(sc[nt], qa[2 * kp], b0, b1);
-          mma16816(sc[nt], qa[2 * kp + 1], b2, b3);
-        }
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t a[4];
+        ldsm_x4(kt + tile_off((lane & 7) + ((mi & 1) << 3), 2 * ks + (mi >> 1)), a[0], a[1], a[2], a[3]);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma16816(sc[nt], a, qb[nt][ks][0], qb[nt][ks][1]);
       }
-      // logits to the caller; base-2 scale; rows past the range drop out
+      // sc[nt][e]: row gid + 8 (e >> 1), head 8 nt + 2 tig + (e & 1)
       if (p.logits != nullptr) {
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int row = r0 + nt * 8 + 2 * tig + (e & 1);
-            const int head = (e < 2) ? gid : gid + 8;
+            const int row = r0 + gid + 8 * (e >> 1);
+            const int head = nt * 8 + 2 * tig + (e & 1);
             if (row < r_end && head < G)
               p.logits[((int64_t)s * p.hq + qh0 + head) * p.max_seq_len + row] = sc[nt][e] * p.scale;
           }
       }
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) sc[nt][e] *= p.qscale;
       if (r0 + kWTile > r_end) {
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            if (r0 + nt * 8 + 2 * tig + (e & 1) >= r_end) sc[nt][e] = -INFINITY;
+            if (r0 + gid + 8 * (e >> 1) >= r_end) sc[nt][e] = -INFINITY;
       }
-      // online softmax: the tile maximum of each head over the 4 lanes of its
-      // group; the running maximum moves (and the accumulators are rescaled)
-      // only when the tile exceeds it by more than kRescale
-      float t0 = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-      float t1 = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
-      t0 = fmaxf(t0, __shfl_xor_sync(kFull, t0, 1));
-      t0 = fmaxf(t0, __shfl_xor_sync(kFull, t0, 2));
-      t1 = fmaxf(t1, __shfl_xor_sync(kFull, t1, 1));
-      t1 = fmaxf(t1, __shfl_xor_sync(kFull, t1, 2));
-      const bool up0 = t0 > m0 + kRescale, up1 = t1 > m1 + kRescale;  // always at the first tile
-      if (__any_sync(kFull, up0 || up1)) {
-        const float mn0 = up0 ? t0 : m0, mn1 = up1 ? t1 : m1;
-        const float a0 = exp2f(m0 - mn0), a1 = exp2f(m1 - mn1);  // 0 at the first tile
-        m0 = mn0;
-        m1 = mn1;
-        l0 *= a0;
-        l1 *= a1;
+      // online softmax: the tile maximum of each head over its 16 rows (the
+      // 8 lanes that share tig); the running maximum moves, and the
+      // accumulators are rescaled, only when the tile exceeds it by more
+      // than kRescale
+      float t[NT][2];
+      bool up = false;
 #pragma unroll
-        for (int dt = 0; dt < 16; ++dt) {
-          o[dt][0] *= a0;
-          o[dt][1] *= a0;
-          o[dt][2] *= a1;
-          o[dt][3] *= a1;
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float x = fmaxf(sc[nt][e], sc[nt][e + 2]);
+          x = fmaxf(x, __shfl_xor_sync(kFull, x, 4));
+          x = fmaxf(x, __shfl_xor_sync(kFull, x, 8));
+          x = fmaxf(x, __shfl_xor_sync(kFull, x, 16));
+          t[nt][e] = x;
+          up = up || x > m[nt][e] + kRescale;  // always at the first tile
+        }
+      if (__any_sync(kFull, up)) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float a[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float mn = t[nt][e] > m[nt][e] + kRescale ? t[nt][e] : m[nt][e];
+            a[e] = exp2f(m[nt][e] - mn);  // 0 at the first tile
+            m[nt][e] = mn;
+            l[nt][e] *= a[e];
+          }
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            o[nt][mt][0] *= a[0];
+            o[nt][mt][1] *= a[1];
+            o[nt][mt][2] *= a[0];
+            o[nt][mt][3] *= a[1];
+          }
         }
       }
+      // weights; P^T as the B operand of O^T += V^T P^T: each 8x8 block of
+      // P (rows x heads) transposed in registers (movmatrix), bf16 hi + lo
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        sc[nt][0] = exp2f(sc[nt][0] - m0);
-        sc[nt][1] = exp2f(sc[nt][1] - m0);
-        sc[nt][2] = exp2f(sc[nt][2] - m1);
-        sc[nt][3] = exp2f(sc[nt][3] - m1);
-        l0 += sc[nt][0] + sc[nt][1];
-        l1 += sc[nt][2] + sc[nt][3];
-      }
-      // O += P V: one k-step of 16 rows, 16 column tiles of 8 dims
-      uint32_t ah[4], al[4];
-      split2(sc[0][0], sc[0][1], ah[0], al[0]);
-      split2(sc[0][2], sc[0][3], ah[1], al[1]);
-      split2(sc[1][0], sc[1][1], ah[2], al[2]);
-      split2(sc[1][2], sc[1][3], ah[3], al[3]);
+      for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-      for (int dp = 0; dp < 8; ++dp) {
-        const int mi = lane >> 3;
-        const int row = (lane & 7) + ((mi & 1) << 3);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(vt + tile_off(row, 2 * dp + (mi >> 1)), b0, b1, b2, b3);
-        mma16816(o[2 * dp], ah, b0, b1);
-        mma16816(o[2 * dp], al, b0, b1);
-        mma16816(o[2 * dp + 1], ah, b2, b3);
-        mma16816(o[2 * dp + 1], al, b2, b3);
+        for (int e = 0; e < 4; ++e) {
+          sc[nt][e] = exp2f(sc[nt][e] - m[nt][e & 1]);
+          l[nt][e & 1] += sc[nt][e];
+        }
+        uint32_t h0, l0, h1, l1;
+        split2(sc[nt][0], sc[nt][1], h0, l0);  // rows 0..7
+        split2(sc[nt][2], sc[nt][3], h1, l1);  // rows 8..15
+        const uint32_t bh0 = movm_t(h0), bl0 = movm_t(l0), bh1 = movm_t(h1), bl1 = movm_t(l1);
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          uint32_t a[4];
+          // V^T fragments: dims 16 mt + gid (+ 8) x rows 2 tig (+ 8)
+          ldsm_x4_t(vt + tile_off((lane & 7) + ((mi >> 1) << 3), 2 * mt + (mi & 1)), a[0], a[1], a[2], a[3]);
+          mma16816(o[nt][mt], a, bh0, bh1);
+          mma16816(o[nt][mt], a, bl0, bl1);
+        }
       }
       __syncwarp();  // the stage is read: the next loads may overwrite it
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
-    l0 += __shfl_xor_sync(kFull, l0, 1);
-    l0 += __shfl_xor_sync(kFull, l0, 2);
-    l1 += __shfl_xor_sync(kFull, l1, 1);
-    l1 += __shfl_xor_sync(kFull, l1, 2);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        l[nt][e] += __shfl_xor_sync(kFull, l[nt][e], 4);
+        l[nt][e] += __shfl_xor_sync(kFull, l[nt][e], 8);
+        l[nt][e] += __shfl_xor_sync(kFull, l[nt][e], 16);
+      }
   }
 
   // merge the warps: (o, m, l) of every warp and head to shared memory (over
@@ -335,24 +371,24 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
   float *wo = reinterpret_cast<float *>(sm_dec);          // [kDecWarps][G][128]
   float *wm = wo + kDecWarps * G * 128;                    // [kDecWarps][G]
   float *wl = wm + kDecWarps * G;                          // [kDecWarps][G]
-  if (gid < G) {
 #pragma unroll
-    for (int dt = 0; dt < 16; ++dt)
-      *reinterpret_cast<float2 *>(wo + (warp * G + gid) * 128 + dt * 8 + 2 * tig) = make_float2(o[dt][0], o[dt][1]);
-    if (tig == 0) {
-      wm[warp * G + gid] = m0;
-      wl[warp * G + gid] = l0;
-    }
-  }
-  if (gid + 8 < G) {
+  for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int dt = 0; dt < 16; ++dt)
-      *reinterpret_cast<float2 *>(wo + (warp * G + gid + 8) * 128 + dt * 8 + 2 * tig) = make_float2(o[dt][2], o[dt][3]);
-    if (tig == 0) {
-      wm[warp * G + gid + 8] = m1;
-      wl[warp * G + gid + 8] = l1;
+    for (int e = 0; e < 2; ++e) {
+      const int head = nt * 8 + 2 * tig + e;
+      if (head < G) {
+        float *dst = wo + (warp * G + head) * 128;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          dst[16 * mt + gid] = o[nt][mt][e];
+          dst[16 * mt + gid + 8] = o[nt][mt][e + 2];
+        }
+        if (gid == 0) {
+          wm[warp * G + head] = m[nt][e];
+          wl[warp * G + head] = l[nt][e];
+        }
+      }
     }
-  }
   __syncthreads();
   for (int i = threadIdx.x; i < G * 128; i += kDecThreads) {
     const int g = i >> 7, d = i & 127;
