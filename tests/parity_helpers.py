@@ -53,6 +53,33 @@ def unit_oracle(w, s: int, layer: int, h: int, k_bits=None, positions=None, form
     return res
 
 
+def check_direct_sample(gpu_scores: np.ndarray, w, s: int, layer: int, h: int, k_bits, positions,
+                        ora: dict, frac: float = 0.01, seed: int = 0, where=""):
+    """The GPU scores of a seeded sample (frac) of the unit's candidates
+    against the direct 17-offset form (Eq. 4 evaluated offset by offset),
+    within the same 1e-4 * L1 bound as the folded comparison."""
+    cfg = w.cfg
+    C = gpu_scores.shape[0]
+    n = max(1, int(round(frac * C)))
+    cand = np.sort(np.random.default_rng(seed + 7919 * (layer * 64 + h)).choice(C, n, replace=False))
+    slots = cand + cfg.sinks
+    k = O.bf16_bits_to_f64(np.asarray(k_bits)[slots])
+    G = cfg.group
+    re, im, am = w.stats
+    qc = (re[layer, h * G:(h + 1) * G].astype(np.float64)
+          + 1j * im[layer, h * G:(h + 1) * G].astype(np.float64))
+    qa = am[layer, h * G:(h + 1) * G].astype(np.float64)
+    omega = O.band_frequencies(cfg.head_dim, cfg.theta)
+    p_q = int(w.query_pos[s].item())
+    direct = O.unit_scores(k, np.asarray(positions)[slots], p_q, qc, qa, omega, cfg.pairing,
+                           cfg.offset_log2_max, form="direct")
+    err = np.abs(np.asarray(gpu_scores, dtype=np.float64)[cand].T - direct)
+    bound = SCORE_RTOL * ora["l1"][:, cand]
+    assert np.all(err <= bound), (f"{where}: {np.sum(err > bound)} sampled scores off the direct "
+                                  f"form; worst ratio {np.max(err / bound):.3g}")
+    return n
+
+
 def check_scores(gpu_scores: np.ndarray, ora: dict, where=""):
     """gpu_scores: [C, G] fp32."""
     S = np.asarray(gpu_scores, dtype=np.float64).T

@@ -78,7 +78,8 @@ def all_units(cfg):
             for h in range(cfg.n_kv_heads)]
 
 
-def full_check(cfg, units=None, score_layers_sel=None, direct_form=False, offset_reduce=0):
+def full_check(cfg, units=None, score_layers_sel=None, direct_form=False, offset_reduce=0,
+               direct_sample=0.0):
     """Score/select parity on `units` (default: all), then the fused pass:
     same kept set, compacted bytes, lengths, positions, freed blocks."""
     w = synth.Workload(cfg)
@@ -109,6 +110,9 @@ def full_check(cfg, units=None, score_layers_sel=None, direct_form=False, offset
                     if direct_form:
                         ora_d = PH.unit_oracle(w, s, l, h, k_bits=kb, positions=pos, form="direct")
                         PH.check_scores(sc[s, 0, h, :C], ora_d, where + " direct")
+                    elif direct_sample > 0 and not offset_reduce:
+                        PH.check_direct_sample(sc[s, 0, h, :C], w, s, l, h, kb, pos, ora,
+                                               frac=direct_sample, where=where + " direct sample")
                 else:
                     PH.check_kept_same_precision(kept[s, 0, h], np.zeros(0), N, cfg, where)
                 PH.check_kept_vs_oracle(kept[s, 0, h], ora, cfg, where)
@@ -363,19 +367,21 @@ def _sample_units(cfg, n, seed):
     return sorted(out)
 
 
+# sampled units against the folded oracle on every key, and against the direct
+# 17-offset form on a seeded 1 % of their keys
 def test_full_size_qwen3_8b():
     cfg = synth.CONFIGS[1]
-    full_check(cfg, units=_sample_units(cfg, 6, 1))
+    full_check(cfg, units=_sample_units(cfg, 6, 1), direct_sample=0.01)
 
 
 def test_full_size_qwen3_32b_32k():
     cfg = synth.CONFIGS[2]
-    full_check(cfg, units=_sample_units(cfg, 4, 2))
+    full_check(cfg, units=_sample_units(cfg, 4, 2), direct_sample=0.01)
 
 
 def test_full_size_qwen3_32b_131k():
     cfg = synth.CONFIGS[4]
-    full_check(cfg, units=_sample_units(cfg, 3, 4))
+    full_check(cfg, units=_sample_units(cfg, 3, 4), direct_sample=0.01)
 
 
 def test_full_size_llama3_batched_paged():
@@ -384,7 +390,7 @@ def test_full_size_llama3_batched_paged():
     need = 178e9
     if free < need:
         pytest.skip(f"needs ~{need / 1e9:.0f} GB free, {free / 1e9:.0f} GB available")
-    full_check(cfg, units=_sample_units(cfg, 4, 3))
+    full_check(cfg, units=_sample_units(cfg, 4, 3), direct_sample=0.01)
 
 
 # ---------------------------------------------------------------------------
