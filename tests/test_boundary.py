@@ -102,3 +102,17 @@ def test_product_path_does_not_import_the_oracle():
             if f.endswith((".py", ".cu", ".h", ".cuh")):
                 src = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in src.replace("oracle/", ""), f
+
+
+def test_newer_entry_points_reject_missing_objects_on_the_host():
+    # budget variants and decode attention validate before any CUDA call
+    lib = T.lib()
+    b = (ctypes.c_int * 4)()
+    row = ctypes.c_int()
+    assert lib.tria_layer_budgets(None, None, None, b, ctypes.byref(row)) == 1
+    size = ctypes.c_size_t()
+    assert lib.tria_decode_workspace_size(None, None, ctypes.byref(size)) == 1
+    assert lib.tria_decode_attention(None, None, 0, None, 1.0, None, None, None, None, 0, None) == 1
+    prm = T.params(2048, 256, 0, budget_pct=50.0, layer_budget_scales=[1.0, 0.5], interval=128)
+    assert abs(prm.budget_pct - 50.0) < 1e-6 and prm.interval == 128
+    assert abs(prm.layer_budget_scales[1] - 0.5) < 1e-7
