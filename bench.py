@@ -407,6 +407,12 @@ def main():
         line["offset_max"] = offset_max(T, torch, st, cache, cfg, kept, restore, hbm)
         line["layer_budgets"] = layer_budgets(T, torch, w, st, cfg, restore, hbm)
         line["e2e"] = e2e(T, torch, w, st, cache, prm, ws, kept, restore, args.e2e_steps, keys, world)
+        if world > 1:
+            # the job's end-to-end time is the slowest rank's (every rank
+            # takes this collective)
+            ms_e2e = max_over_ranks(line["e2e"]["ms_per_step"], dist, "cuda")
+            line["e2e"]["ms_per_step"] = ms_e2e
+            line["e2e"]["value"] = keys * world / (ms_e2e * 1e-3)
         if rank == 0 and world == 1:
             v, n_units, spent = oracle_unit_keys_per_s(cfg, args.cpu_seconds)
             # the direct 17-offset form (Eq. 4), the reference-style scorer,
