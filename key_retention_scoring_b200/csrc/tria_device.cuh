@@ -225,6 +225,42 @@ template <int NT>
 __device__ void gather_pass(const float *agg, int C, uint32_t pmask, uint32_t prefix,
                             TailScratch &ts, SelScalars &sc, int tid) {
   const int lane = tid & 31;
+  if (aligned16p(agg)) {
+    // 8 candidates per thread per round (2 float4 loads in flight); the
+    // list order does not matter
+    const int C4 = C >> 2;
+    const float4 *a4 = reinterpret_cast<const float4 *>(agg);
+    for (int b = 0; b < C4 + 1; b += NT * 2) {
+      float4 v[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int i = b + e * NT + tid;
+        v[e] = (i < C4) ? __ldcg(a4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int i = b + e * NT + tid;
+        const float x[4] = {v[e].x, v[e].y, v[e].z, v[e].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          // candidates past the float4s (at most 3) ride on index C4
+          const int c = (i < C4) ? 4 * i + q : (i == C4 ? 4 * C4 + q : C);
+          const float xv = (i < C4) ? x[q] : (c < C ? __ldcg(agg + c) : 0.f);
+          const uint32_t k = order_key(xv);
+          const bool m = c < C && (k & pmask) == prefix;
+          const uint32_t bal = __ballot_sync(kFull, m);
+          int base = 0;
+          if (lane == 0 && bal) base = atomicAdd(&sc.list_n, __popc(bal));
+          base = __shfl_sync(kFull, base, 0);
+          if (m) {
+            const int idx = base + __popc(bal & ((1u << lane) - 1u));
+            if (idx < kListCap) ts.list[idx] = make_uint2(k, (uint32_t)c);
+          }
+        }
+      }
+    }
+    return;
+  }
   for (int c0 = 0; c0 < C; c0 += NT * 4) {
     float x[4];
 #pragma unroll
