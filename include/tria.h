@@ -100,7 +100,8 @@ typedef struct {
 /* Opaque, library-owned device copy of the folded statistics. */
 typedef struct tria_stats tria_stats;
 
-/* The caller's KV cache.  Every pointer stays owned by the caller. */
+/* The caller's KV cache.  Every pointer stays owned by the caller.
+ * Zero-initialise the struct: optional fields are off at zero (NULL). */
 typedef struct {
   int layout;                /* tria_layout                                          */
   int n_seq;                 /* 1 .. TRIA_MAX_SEQS                                   */
@@ -150,7 +151,8 @@ typedef enum {
                            G * |D| <= 136 (G <= 8 at |D| = 17), else UNSUPPORTED    */
 } tria_offset_reduce;
 
-/* Retention parameters (one set for all units of a call).
+/* Retention parameters (one set for all units of a call).  Zero-initialise
+ * the struct and set what is needed: every field past `sinks` is off at zero.
  *
  * Budget of layer l (rows kept per unit, window and sinks included):
  *   base = budget_pct > 0 ? floor(budget_pct * max_seq_len / 100) : budget
