@@ -65,7 +65,9 @@ typedef enum {
   TRIA_ERR_UNSUPPORTED = 2, /* valid but not built: head_dim != 128, G > 16 */
   TRIA_ERR_WORKSPACE = 3,   /* workspace null or smaller than required */
   TRIA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
-  TRIA_ERR_OOM = 5          /* device allocation failed (tria_load_stats) */
+  TRIA_ERR_OOM = 5,         /* device allocation failed (tria_load_stats) */
+  TRIA_ERR_IO = 6           /* a stats file could not be opened, read or written,
+                               or is not in this library's format */
 } tria_status;
 
 typedef enum {
@@ -206,6 +208,44 @@ tria_status tria_load_stats(const tria_model_desc *desc, const float *q_mean_re,
                             const float *q_mean_im, const float *q_abs_mean,
                             const float *band_mask, tria_stream_t stream,
                             tria_stats **out);
+
+/*
+ * Stats files: this library's own format for the calibrated statistics (the
+ * llama.cpp port's stats.bin layout is not documented, so it is not read).
+ * Little-endian, no padding:
+ *   offset  size  field
+ *   0       4     uint32 magic 0x54524941
+ *   4       4     uint32 version 1
+ *   8       24    int32 n_layers, n_q_heads, n_kv_heads, head_dim, pairing,
+ *                 offset_log2_max
+ *   32      8     float64 rope_theta
+ *   40      4     uint32 flags: bit 0 per-layer budget scales present, bit 1
+ *                 band mask present
+ *   44      4     uint32 0
+ *   48            float32 q_mean_re [n_layers][n_q_heads][head_dim/2], then
+ *                 q_mean_im and q_abs_mean (the same shape), then the
+ *                 per-layer budget scales [n_layers] and the band mask
+ *                 [head_dim/2] when their flags are set.
+ *
+ * tria_write_stats_file - write the statistics (host arrays, layouts as in
+ *   tria_load_stats; scales and mask nullable) to `path` (created or
+ *   truncated).  Errors: INVALID_ARG (null pointer, bad desc), IO.
+ * tria_read_stats_file - read the header into *desc_out and the flags into
+ *   *has_scales / *has_mask (each nullable), and, for every non-null array
+ *   pointer, the array (host memory the caller sized from *desc_out; asking
+ *   for scales or mask the file does not hold is INVALID_ARG).  Calling it
+ *   first with every array NULL gives the sizes.  Errors: INVALID_ARG, IO
+ *   (missing, short or foreign file), UNSUPPORTED (another version).
+ * Both are host-only: they make no CUDA call.
+ */
+tria_status tria_write_stats_file(const char *path, const tria_model_desc *desc,
+                                  const float *q_mean_re, const float *q_mean_im,
+                                  const float *q_abs_mean, const float *layer_budget_scales,
+                                  const float *band_mask);
+tria_status tria_read_stats_file(const char *path, tria_model_desc *desc_out, int *has_scales,
+                                 int *has_mask, float *q_mean_re, float *q_mean_im,
+                                 float *q_abs_mean, float *layer_budget_scales,
+                                 float *band_mask);
 
 /* Free a stats object (synchronises the device first).  NULL is allowed. */
 tria_status tria_free_stats(tria_stats *stats);

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libtria.so")
 
 TRIA_OK = 0
 STATUS_NAMES = {0: "TRIA_OK", 1: "TRIA_ERR_INVALID_ARG", 2: "TRIA_ERR_UNSUPPORTED",
-                3: "TRIA_ERR_WORKSPACE", 4: "TRIA_ERR_CUDA", 5: "TRIA_ERR_OOM"}
+                3: "TRIA_ERR_WORKSPACE", 4: "TRIA_ERR_CUDA", 5: "TRIA_ERR_OOM", 6: "TRIA_ERR_IO"}
 PAIR_NEOX = 0
 PAIR_INTERLEAVED = 1
 LAYOUT_CONTIGUOUS = 0
@@ -31,7 +31,8 @@ EXPORTS = ["tria_status_string", "tria_version", "tria_load_stats", "tria_free_s
            "tria_stats_desc", "tria_workspace_size", "tria_score", "tria_select", "tria_compact",
            "tria_compress_pass", "tria_read_device_status", "tria_set_pass_events",
            "tria_compress_pass_static", "tria_calib_accumulate", "tria_calib_finalize",
-           "tria_layer_budgets", "tria_decode_workspace_size", "tria_decode_attention"]
+           "tria_layer_budgets", "tria_decode_workspace_size", "tria_decode_attention",
+           "tria_write_stats_file", "tria_read_stats_file"]
 STATIC_SCRATCH_BYTES = 32 * 1024 * 1024   # TRIA_STATIC_SCRATCH_BYTES
 
 
@@ -113,6 +114,11 @@ def lib() -> ctypes.CDLL:
                                              ctypes.POINTER(ctypes.c_size_t)]
     L.tria_decode_attention.argtypes = [_VP, ctypes.POINTER(CacheView), _I, _VP, ctypes.c_float,
                                         _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP]
+    L.tria_write_stats_file.argtypes = [ctypes.c_char_p, ctypes.POINTER(ModelDesc), _VP, _VP, _VP,
+                                        _VP, _VP]
+    L.tria_read_stats_file.argtypes = [ctypes.c_char_p, ctypes.POINTER(ModelDesc),
+                                       ctypes.POINTER(_I), ctypes.POINTER(_I), _VP, _VP, _VP, _VP,
+                                       _VP]
     for name in EXPORTS:
         if name not in ("tria_status_string", "tria_version"):
             getattr(L, name).restype = _I
@@ -168,6 +174,49 @@ def model_desc(n_layers, n_q_heads, n_kv_heads, pairing, rope_theta, offset_log2
                head_dim=128) -> ModelDesc:
     return ModelDesc(n_layers, n_q_heads, n_kv_heads, head_dim, pairing, float(rope_theta),
                      offset_log2_max)
+
+
+def _f32(a):
+    import numpy as np
+
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float32)
+
+
+def tria_write_stats_file(path, desc: ModelDesc, q_mean_re, q_mean_im, q_abs_mean,
+                          layer_budget_scales=None, band_mask=None):
+    """Save the calibrated statistics (host arrays [L][Hq][F]) in the
+    library's stats file format."""
+    arrs = [_f32(a) for a in (q_mean_re, q_mean_im, q_abs_mean, layer_budget_scales, band_mask)]
+    n = desc.n_layers * desc.n_q_heads * (desc.head_dim // 2)
+    if any(a.size != n for a in arrs[:3]):
+        raise TriaError(1, "tria_write_stats_file: array sizes")
+    _check(lib().tria_write_stats_file(os.fsencode(path), ctypes.byref(desc),
+                                       *[None if a is None else a.ctypes.data for a in arrs]),
+           "tria_write_stats_file")
+
+
+def tria_read_stats_file(path):
+    """(desc, q_mean_re, q_mean_im, q_abs_mean, layer_budget_scales or None,
+    band_mask or None) from a stats file; arrays are numpy float32."""
+    import numpy as np
+
+    L = lib()
+    desc = ModelDesc()
+    sc, mk = _I(), _I()
+    _check(L.tria_read_stats_file(os.fsencode(path), ctypes.byref(desc), ctypes.byref(sc),
+                                  ctypes.byref(mk), None, None, None, None, None),
+           "tria_read_stats_file")
+    F = desc.head_dim // 2
+    shape = (desc.n_layers, desc.n_q_heads, F)
+    re, im, am = (np.empty(shape, np.float32) for _ in range(3))
+    scales = np.empty(desc.n_layers, np.float32) if sc.value else None
+    mask = np.empty(F, np.float32) if mk.value else None
+    _check(L.tria_read_stats_file(os.fsencode(path), ctypes.byref(desc), None, None,
+                                  re.ctypes.data, im.ctypes.data, am.ctypes.data,
+                                  None if scales is None else scales.ctypes.data,
+                                  None if mask is None else mask.ctypes.data),
+           "tria_read_stats_file")
+    return desc, re, im, am, scales, mask
 
 
 def tria_load_stats(desc: ModelDesc, q_mean_re, q_mean_im, q_abs_mean, band_mask=None,

@@ -371,6 +371,7 @@ const char *tria_status_string(tria_status s) {
     case TRIA_ERR_WORKSPACE: return "TRIA_ERR_WORKSPACE: workspace missing, misaligned or too small";
     case TRIA_ERR_CUDA: return "TRIA_ERR_CUDA: CUDA runtime error";
     case TRIA_ERR_OOM: return "TRIA_ERR_OOM: device allocation failed";
+    case TRIA_ERR_IO: return "TRIA_ERR_IO: stats file missing, unreadable or not in this format";
   }
   return "unknown tria_status";
 }

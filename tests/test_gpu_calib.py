@@ -116,3 +116,43 @@ def test_calibration_argument_checks():
     assert float(acc.abs().sum()) == 0.0
     with pytest.raises(T.TriaError):
         T.tria_calib_finalize(d, acc, 0, *[torch.empty((hq, 64), device="cuda") for _ in range(3)])
+
+
+def test_calibrated_stats_through_a_stats_file(tmp_path):
+    # calibrate on the device, save the statistics in the library's file
+    # format, read them back and load them: the pass keeps the same rows as
+    # with the statistics straight from the calibration
+    cfg = synth.CONFIGS[0]
+    hq = cfg.n_q_heads
+    bits = synth.calib_queries(2048, hq, seed=9, layer=0)
+    desc = T.model_desc(cfg.n_layers, hq, cfg.n_kv_heads, cfg.pairing, cfg.theta,
+                        cfg.offset_log2_max)
+    acc = torch.zeros((hq, 64, 3), dtype=torch.float64, device="cuda")
+    T.tria_calib_accumulate(desc, _device_bf16(bits), acc)
+    outs = [torch.empty((hq, 64), device="cuda") for _ in range(3)]
+    T.tria_calib_finalize(desc, acc, 2048, *outs)
+    torch.cuda.synchronize()
+    re, im, am = (o.cpu().numpy().reshape(1, hq, 64) for o in outs)
+    path = tmp_path / "calib.tria"
+    T.tria_write_stats_file(path, desc, re, im, am)
+    d2, re2, im2, am2, sc2, mk2 = T.tria_read_stats_file(path)
+    assert sc2 is None and mk2 is None and d2.n_q_heads == hq
+
+    kept = []
+    for arrays, dd in (((re, im, am), desc), ((re2, im2, am2), d2)):
+        w = synth.Workload(cfg)
+        st = T.tria_load_stats(dd, *arrays)
+        try:
+            cache = T.Cache.from_workload(w)
+            prm = T.params(cfg.budget, cfg.window, cfg.sinks)
+            ws = T.alloc_workspace(T.tria_workspace_size(st, cache, prm))
+            k = torch.full((cfg.n_seq, cfg.n_layers, cfg.n_kv_heads, cfg.budget), -7,
+                           dtype=torch.int32, device="cuda")
+            T.tria_compress_pass(st, cache, prm, k, ws)
+            torch.cuda.synchronize()
+            kept.append(k.cpu().numpy())
+        finally:
+            st.free()
+            del w
+    assert np.array_equal(kept[0], kept[1])
+    assert np.all(kept[0][..., -cfg.window:] >= 0)
