@@ -488,6 +488,11 @@ def pin_budget_variants_golden():
     assert O.freed_block_range(old, new_a, 16) == tuple(int(x) for x in g["freed_a"].split())
     new_b = O.pass_lengths(old[None], np.array([1024, 1024]), 128)[0]
     assert O.freed_block_range(old, new_b, 16) == tuple(int(x) for x in g["freed_b"].split())
+    # lengths that are not whole blocks, and a percentage that is not a whole row
+    assert O.freed_block_range(np.array([2100, 2100]), np.array([1000, 1030]), 16) == \
+        tuple(int(x) for x in g["freed_c"].split())
+    assert list(O.layer_budgets(1, 0, int(g["pct_cap"]), budget_pct=float(g["pct_odd"]))) == \
+        [int(g["pct_odd_budget"])]
 
 
 def pin_interval_unit_pipeline():

@@ -222,6 +222,19 @@ def _recall_of_dropped(logits, kept):
     return _orig["attention_recall"](logits, drop)
 
 
+def _freed_floor(old_lens, new_lens, block_size):
+    bs = int(block_size)
+    first = int(np.max(new_lens)) // bs
+    return first, max(first, int(np.max(old_lens)) // bs)
+
+
+def _budget_pct_rounded_up(n_layers, budget, capacity, budget_pct=0.0, scales=None):
+    pct = float(np.float32(budget_pct))
+    base = np.ceil(pct * float(capacity) / 100.0) if pct > 0.0 else float(budget)
+    sc = np.ones(int(n_layers)) if scales is None else np.asarray(scales, np.float32).astype(np.float64)
+    return np.floor(base * sc + 0.5).astype(np.int64)
+
+
 _orig = {name: getattr(O, name) for name in dir(O) if callable(getattr(O, name))}
 
 MUTATIONS = {
@@ -264,6 +277,8 @@ MUTATIONS = {
     "softmax over the heads": ("decode_attention", _attn_softmax_over_heads),
     "lse without the max": ("decode_attention", _attn_lse_without_max),
     "recall of the dropped rows": ("attention_recall", _recall_of_dropped),
+    "freed blocks rounded down": ("freed_block_range", _freed_floor),
+    "percentage budget rounded up": ("layer_budgets", _budget_pct_rounded_up),
 }
 
 
