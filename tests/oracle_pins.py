@@ -558,4 +558,13 @@ def pin_attention_recall():
     assert np.allclose(O.attention_recall(z, [1]), [0.75, 0.5])
 
 
+def pin_select_signed_zeros():
+    """-0.0 and +0.0 are equal numbers (IEEE 754), so they tie and the lower
+    slot wins either way round; NaN ranks below -inf."""
+    for agg, want in (([-0.0, 0.0, 1.0], [0, 2]), ([0.0, -0.0, 1.0], [0, 2]),
+                      ([np.nan, -np.inf, -0.0], [1, 2])):
+        kept = O.select_kept(np.array(agg), 3, 2, 0, 0)
+        assert list(kept) == want, (agg, kept)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -235,6 +235,12 @@ def _budget_pct_rounded_up(n_layers, budget, capacity, budget_pct=0.0, scales=No
     return np.floor(base * sc + 0.5).astype(np.int64)
 
 
+def _rank_negative_zero_below(agg):
+    a = np.asarray(agg, dtype=np.float64)
+    key = -a - np.where((a == 0) & np.signbit(a), 1e-300, 0.0)
+    return np.argsort(np.where(np.isnan(a), np.inf, key), kind="stable")
+
+
 _orig = {name: getattr(O, name) for name in dir(O) if callable(getattr(O, name))}
 
 MUTATIONS = {
@@ -279,6 +285,7 @@ MUTATIONS = {
     "recall of the dropped rows": ("attention_recall", _recall_of_dropped),
     "freed blocks rounded down": ("freed_block_range", _freed_floor),
     "percentage budget rounded up": ("layer_budgets", _budget_pct_rounded_up),
+    "-0.0 ranked below +0.0": ("rank_order", _rank_negative_zero_below),
 }
 
 
