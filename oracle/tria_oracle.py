@@ -270,10 +270,11 @@ def gqa_znorm_max(scores: np.ndarray, eps: float = NORM_EPS):
 
 def rank_order(agg: np.ndarray) -> np.ndarray:
     """Candidate indices by descending score; equal scores keep ascending
-    index order (stable sort); NaN last; -0.0 == +0.0."""
+    index order; NaN below every number (-inf included); -0.0 == +0.0.
+    Sorted by (is NaN, -score, index)."""
     a = np.asarray(agg, dtype=np.float64)
-    key = np.where(np.isnan(a), np.inf, -a)
-    return np.argsort(key, kind="stable")
+    nan = np.isnan(a)
+    return np.lexsort((np.arange(a.size), np.where(nan, 0.0, -a), nan))
 
 
 def select_kept(agg: np.ndarray, n_tokens: int, budget: int, window: int,
