@@ -260,7 +260,7 @@ def test_select_adversarial_agg():
         cmax = w.max_seq_len - cfg.window - cfg.sinks
         rng = np.random.default_rng(5)
         agg = np.zeros((cfg.n_seq, 1, cfg.n_kv_heads, cmax), dtype=np.float32)
-        kinds = ["int_ties", "all_equal", "zeros", "specials", "normal"]
+        kinds = ["int_ties", "all_equal", "zeros", "specials", "normal", "nan_neginf"]
         for s in range(cfg.n_seq):
             for h in range(cfg.n_kv_heads):
                 kind = kinds[(s * cfg.n_kv_heads + h) % len(kinds)]
@@ -277,6 +277,11 @@ def test_select_adversarial_agg():
                     a[r < 0.05] = np.inf
                     a[(r >= 0.05) & (r < 0.1)] = -np.inf
                     a[(r >= 0.1) & (r < 0.3)] = np.nan
+                elif kind == "nan_neginf":
+                    # only -inf and NaN: the K-th key falls among them, and
+                    # -inf must rank above NaN
+                    a = np.full(cmax, -np.inf, dtype=np.float32)
+                    a[rng.random(cmax) < 0.6] = np.nan
                 else:
                     a = rng.normal(size=cmax).astype(np.float32)
                 agg[s, 0, h] = a
