@@ -567,4 +567,27 @@ def pin_select_signed_zeros():
         assert list(kept) == want, (agg, kept)
 
 
+def pin_band_mask():
+    """The high-frequency band mask rescales |mu'_f| in the trigonometric
+    term only (article 2607.13051 sec. 7): the masked score equals the trig
+    term of the query center multiplied by the mask (with the norm term
+    zeroed by E|q| = |E q|) plus the unmasked norm term; an all-ones mask is
+    no mask and an all-zero mask leaves the norm term alone."""
+    rng = np.random.default_rng(41)
+    d, G, N, theta = 16, 2, 12, 1e4
+    qc, qa, k_pre, k_post, pos, p_q = _random_unit(rng, d, G, N, O.PAIR_NEOX, theta)
+    omega = O.band_frequencies(d, theta)
+    m = rng.random(d // 2)
+    got = O.unit_scores(k_post, pos, p_q, qc, qa, omega, O.PAIR_NEOX, band_mask=m)
+    trig = O.unit_scores(k_post, pos, p_q, qc * m, np.abs(qc * m), omega, O.PAIR_NEOX)
+    kb = O.to_bands(k_pre, O.PAIR_NEOX)
+    norm = np.stack([O.s_norm(qc[h], qa[h], kb) for h in range(G)])
+    assert np.allclose(got, trig + norm, rtol=0, atol=1e-10 * (1 + np.abs(got).max()))
+    plain = O.unit_scores(k_post, pos, p_q, qc, qa, omega, O.PAIR_NEOX)
+    ones = O.unit_scores(k_post, pos, p_q, qc, qa, omega, O.PAIR_NEOX, band_mask=np.ones(d // 2))
+    zero = O.unit_scores(k_post, pos, p_q, qc, qa, omega, O.PAIR_NEOX, band_mask=np.zeros(d // 2))
+    assert np.allclose(ones, plain, rtol=0, atol=1e-12 * (1 + np.abs(plain).max()))
+    assert np.allclose(zero, norm, rtol=0, atol=1e-12 * (1 + np.abs(norm).max()))
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -22,7 +22,7 @@ SCORE_RTOL = 1e-4
 
 
 def unit_oracle(w, s: int, layer: int, h: int, k_bits=None, positions=None, form="folded",
-                budget=None, interval=0, n=None):
+                budget=None, interval=0, n=None, band_mask=None):
     """Oracle of one unit of a synth.Workload (reads K rows back unless given).
     budget: the unit's budget (default: the configuration's); n: its length
     (default: the sequence's)."""
@@ -40,14 +40,16 @@ def unit_oracle(w, s: int, layer: int, h: int, k_bits=None, positions=None, form
     qa = am[layer, h * G:(h + 1) * G].astype(np.float64)
     omega = O.band_frequencies(cfg.head_dim, cfg.theta)
     p_q = int(w.query_pos[s].item())
+    mask = None if band_mask is None else np.asarray(band_mask, np.float32).astype(np.float64)
     res = O.compress_unit(k, positions, p_q, qc, qa, omega, cfg.pairing, B, cfg.window,
-                          cfg.sinks, cfg.offset_log2_max, form=form, interval=interval)
+                          cfg.sinks, cfg.offset_log2_max, band_mask=mask, form=form,
+                          interval=interval)
     N = len(k)
     res["B"] = B
     res["compressed"] = O.is_compressed(N, B, interval)
     if res["scores"] is not None:
         l1 = O.score_l1_scale(k, positions, qc, qa, omega, cfg.pairing, cfg.offset_log2_max,
-                              form="max" if form == "max" else "folded")
+                              band_mask=mask, form="max" if form == "max" else "folded")
         res["l1"] = l1[:, cfg.sinks:N - cfg.window]
     res["N"] = N
     return res

@@ -440,3 +440,30 @@ def test_offset_max_unsupported_shapes():
         assert ei.value.status == 1
     finally:
         st.free()
+
+
+# ---------------------------------------------------------------------------
+# the high-frequency band mask (article 2607.13051 sec. 7), folded into the
+# coefficients at load time
+# ---------------------------------------------------------------------------
+def test_band_mask_scores_and_selection():
+    cfg = synth.CONFIGS[2].scaled(n_layers=1, seq_len=3000)
+    w = synth.Workload(cfg)
+    mask = np.linspace(0.2, 1.0, 64).astype(np.float32)
+    desc = T.model_desc(cfg.n_layers, cfg.n_q_heads, cfg.n_kv_heads, cfg.pairing, cfg.theta,
+                        cfg.offset_log2_max)
+    st = T.tria_load_stats(desc, *w.stats, band_mask=mask)
+    try:
+        agg, sc, kept = score_layers(w, st, 0, 1)
+        C = int(w.lens[0]) - cfg.window - cfg.sinks
+        for h in (0, 3, 7):
+            ora = PH.unit_oracle(w, 0, 0, h, band_mask=mask)
+            where = f"{cfg.name} band mask h{h}"
+            PH.check_scores(sc[0, 0, h, :C], ora, where)
+            PH.check_agg(agg[0, 0, h, :C], ora, where)
+            PH.check_kept_same_precision(kept[0, 0, h], agg[0, 0, h, :C], ora["N"], cfg, where)
+            PH.check_kept_vs_oracle(kept[0, 0, h], ora, cfg, where)
+    finally:
+        st.free()
+        del w
+        torch.cuda.empty_cache()

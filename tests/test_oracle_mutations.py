@@ -241,6 +241,10 @@ def _rank_negative_zero_below(agg):
     return np.argsort(np.where(np.isnan(a), np.inf, key), kind="stable")
 
 
+def _mask_dropped(q_center, W, band_mask=None):
+    return q_center * W
+
+
 _orig = {name: getattr(O, name) for name in dir(O) if callable(getattr(O, name))}
 
 MUTATIONS = {
@@ -286,6 +290,7 @@ MUTATIONS = {
     "freed blocks rounded down": ("freed_block_range", _freed_floor),
     "percentage budget rounded up": ("layer_budgets", _budget_pct_rounded_up),
     "-0.0 ranked below +0.0": ("rank_order", _rank_negative_zero_below),
+    "band mask dropped": ("folded_center", _mask_dropped),
 }
 
 
