@@ -90,3 +90,25 @@ def test_reference_arm_line_on_rank0(capsys):
     assert line["impl"] == "reference" and line["value"] > 0 and line["steps"] == 2
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+
+
+def test_recorded_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
+    """bench.py reports the score kernel's DRAM traffic only while the
+    committed ncu record was taken on the current kernel source."""
+    import json
+
+    import bench
+
+    rec = {"score_kernel": {"source_hash": bench.kernel_source_hash(),
+                            "bytes_per_launch_full_size": 123}}
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(rec))
+    real_root = bench.ROOT
+    src = os.path.join(real_root, "key_retention_scoring_b200")
+    os.symlink(src, tmp_path / "key_retention_scoring_b200")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("score_kernel") == 123
+    rec["score_kernel"]["source_hash"] = "0" * 16
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(rec))
+    assert bench.recorded_traffic("score_kernel") is None
+    assert bench.recorded_traffic("other_kernel") is None
