@@ -49,7 +49,7 @@ def peaks():
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("tria_score_tc.cu", "tria_device.cuh", "tria_internal.h"):
+    for f in ("tria_score_tc.cu", "tria_tc.cuh", "tria_device.cuh", "tria_internal.h"):
         with open(os.path.join(ROOT, "key_retention_scoring_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -134,25 +134,65 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
-# oracle (CPU baseline and reference arm)
+# oracle (CPU baseline and reference arm): worker processes (spawned, one
+# numpy thread each) that time the fp64 oracle on whole units of a workload,
+# generated on the host with the same recipe
 # ---------------------------------------------------------------------------
-def oracle_unit_keys_per_s(cfg, seconds: float, max_units: int = 64, form: str = "folded"):
-    """Time the fp64 oracle (normalize-then-max and selection after the
-    scores in `form`: the folded Eq. 7 or the direct 17-offset Eq. 4) on
-    units of the workload generated on the host with the same recipe."""
+def _single_thread_env():
+    saved = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS",
+                                             "MKL_NUM_THREADS")}
+    for k in saved:
+        os.environ[k] = "1"
+    return saved
+
+
+def _restore_env(saved):
+    for k, v in saved.items():
+        if v is None:
+            os.environ.pop(k, None)
+        else:
+            os.environ[k] = v
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _oracle_units(task):
+    """Worker: the fp64 oracle (scores in `form`, normalize-then-max,
+    selection) on units of workload `cfg_idx` until `seconds` of compute (at
+    least one unit, at most `max_units`).  Returns (keys, seconds, units)."""
+    cfg_idx, form, seconds, max_units, seed = task
     import synth
     from oracle import tria_oracle as O
 
+    cfg = synth.CONFIGS[cfg_idx]
     re, im, am = synth.make_stats(cfg)
     centers = synth.make_centers(cfg)
     omega = O.band_frequencies(cfg.head_dim, cfg.theta)
     G = cfg.group
-    N = int(synth.seq_lengths(cfg)[0])
+    lens = synth.seq_lengths(cfg)
+    rng = np.random.default_rng(seed)
     spent, keys, units = 0.0, 0, 0
-    rng = np.random.default_rng(0)
-    while units == 0 or (spent < seconds and units < max_units):  # at least one unit
+    while units == 0 or (spent < seconds and units < max_units):
+        s = int(rng.integers(cfg.n_seq))
         l, h = int(rng.integers(cfg.n_layers)), int(rng.integers(cfg.n_kv_heads))
-        bits = synth.host_key_rows(cfg, centers, 0, l, h, np.arange(N))
+        N = int(lens[s])
+        bits = synth.host_key_rows(cfg, centers, s, l, h, np.arange(N))
         k = O.bf16_bits_to_f64(bits)
         qc = re[l, h * G:(h + 1) * G].astype(np.float64) + 1j * im[l, h * G:(h + 1) * G]
         qa = am[l, h * G:(h + 1) * G].astype(np.float64)
@@ -162,7 +202,64 @@ def oracle_unit_keys_per_s(cfg, seconds: float, max_units: int = 64, form: str =
         spent += time.perf_counter() - t0
         keys += N
         units += 1
-    return keys / spent, units, spent
+    return keys, spent, units
+
+
+def oracle_rate(cfg_idx: int, form: str, seconds: float, workers: int, max_units: int = 64,
+                seed: int = 0):
+    """keys/s of the oracle on `workers` processes in parallel (the sum of
+    their rates), with the sample it took."""
+    tasks = [(cfg_idx, form, seconds, max_units, seed * 1000 + i) for i in range(workers)]
+    if workers == 1:
+        saved = _single_thread_env()
+        try:
+            res = [_oracle_units(tasks[0])]
+        finally:
+            _restore_env(saved)
+    else:
+        import multiprocessing as mp
+
+        saved = _single_thread_env()
+        try:
+            with mp.get_context("spawn").Pool(workers) as pool:
+                res = pool.map(_oracle_units, tasks)
+        finally:
+            _restore_env(saved)
+    rate = sum(k / t for k, t, _ in res)
+    units = sum(u for _, _, u in res)
+    keys = sum(k for k, _, _ in res)
+    return rate, {"units": units, "keys": keys, "cpu_seconds": round(sum(t for _, t, _ in res), 2)}
+
+
+def cpu_baseline(args, cfg_main):
+    """The fp64 oracle on the host cores: the folded form (Eq. 7) on every
+    workload, and the direct 17-offset form (Eq. 4, the reference-style
+    scorer) on the two smallest both on all cores and on one."""
+    import synth
+
+    cores = host_cores()
+    per = max(2.0, args.cpu_seconds / 6)
+    out = {"kind": "oracle", "cores": cores, "cpu_model": cpu_model(), "unit": UNIT,
+           "workloads": {}}
+    for ci in sorted(synth.CONFIGS):
+        rate, smp = oracle_rate(ci, "folded", per, cores, seed=ci)
+        out["workloads"][synth.CONFIGS[ci].name] = {
+            "value": rate, "sample": f"{smp['units']} units ({smp['keys']} keys) on {cores} "
+                                     f"processes, {smp['cpu_seconds']} CPU s, folded form + z-norm "
+                                     f"+ selection"}
+    direct = {}
+    for ci in (0, 1):
+        r_all, s_all = oracle_rate(ci, "direct", per / 2, cores, max_units=1, seed=10 + ci)
+        r_one, s_one = oracle_rate(ci, "direct", per / 2, 1, max_units=1, seed=20 + ci)
+        direct[synth.CONFIGS[ci].name] = {"all_cores": r_all, "one_core": r_one,
+                                           "sample": f"{s_all['units']} units on {cores} processes; "
+                                                     f"{s_one['units']} unit on one",
+                                           "unit": UNIT}
+    out["direct_form"] = direct
+    main = out["workloads"][cfg_main.name]
+    out["value"] = main["value"]
+    out["sample"] = main["sample"]
+    return out
 
 
 def run_reference(args, rank, world):
@@ -171,22 +268,32 @@ def run_reference(args, rank, world):
     if rank != 0:
         return 0
     cfg = synth.CONFIGS[args.config]
-    per_step = []
-    for i in range(args.warmup + args.steps):
-        v, units, spent = oracle_unit_keys_per_s(cfg, 0.0, max_units=1)
-        if i >= args.warmup:
-            per_step.append(spent)
-    N = int(synth.seq_lengths(cfg)[0])
-    t = sum(per_step)
-    value = args.steps * N / t
+    cores = host_cores()
+    N = int(synth.seq_lengths(cfg).max())
+    # warm-up units, then K units (one per step) spread over the host cores
+    if args.warmup:
+        oracle_rate(args.config, "folded", 0.0, min(cores, args.warmup), max_units=1, seed=1)
+    t0 = time.perf_counter()
+    done, step = 0, 0
+    keys = 0
+    while done < args.steps:
+        n = min(cores, args.steps - done)
+        _, smp = oracle_rate(args.config, "folded", 0.0, n, max_units=1, seed=100 + step)
+        keys += smp["keys"]
+        done += n
+        step += 1
+    wall = time.perf_counter() - t0
+    value = keys / wall
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wall / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_desc(cfg, "one unit (1 layer x 1 KV head) per step"),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"{args.steps} units of {N} keys (G={cfg.group}), fp64 numpy, "
-                                   "folded form + z-norm + selection"},
+        "data": "synthetic", "config": config_desc(cfg, f"one unit (1 layer x 1 KV head, {N} keys) "
+                                                        f"per step, {cores} steps at a time"),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "cpu_model": cpu_model(),
+                         "sample": f"{args.steps} units of {N} keys (G={cfg.group}) on {cores} "
+                                   "processes, fp64 numpy, folded form + z-norm + selection"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -344,12 +451,8 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    pass_ms = [e[0].elapsed_time(e[4]) for e in all_evs]
-    coef_ms = [e[0].elapsed_time(e[1]) for e in all_evs]
-    score_ms = [e[1].elapsed_time(e[2]) for e in all_evs]
-    tail_ms = [e[2].elapsed_time(e[3]) for e in all_evs]
-    compact_ms = [e[3].elapsed_time(e[4]) for e in all_evs]
-    ms = statistics.mean(pass_ms)
+    seg = split_events(all_evs)
+    ms = seg["pass"]
     if world > 1:
         ms = max_over_ranks(ms, dist, "cuda")
 
@@ -357,52 +460,47 @@ def main():
     units = cfg.n_seq * cfg.n_layers * cfg.n_kv_heads
     keys = units * N
     C = N - cfg.window - cfg.sinks
-    score_bytes = units * C * 256
+    k_bytes = units * C * 256
     compact_bytes = moved * 1024
     hbm, peak_kind = peaks()
-    score_avg = statistics.mean(score_ms)
-    tail_avg = statistics.mean(tail_ms)
-    compact_avg = statistics.mean(compact_ms)
-    # the library runs the compaction inside the tail kernel (one block per
-    # unit) when a unit's candidates fit in shared memory: then the last
-    # event segment is empty and the pass has three launches
-    fused = compact_avg < 0.02
-    move_ms = tail_avg + compact_avg if fused else compact_avg
-    raw_bytes = units * C * cfg.group * 4
-    achieved = score_bytes / (score_avg * 1e-3) / 1e9
+    score_ms = seg["score"]
     line = {
         "metric": METRIC, "value": keys * world / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": config_desc(cfg),
+        "numerics": "bf16 K/V cache; scores accumulate in fp32 (tensor cores, bf16 hi/lo "
+                    "operands), moments in fp64, selection on fp32 agg",
         "us_per_pass": ms * 1e3,
-        "pass_gbs": (score_bytes + compact_bytes) / (ms * 1e-3) / 1e9,
         "keys_per_s_per_query_head": keys * world * cfg.group / (ms * 1e-3),
-        "kernels_us": ({"coef": 1e3 * statistics.mean(coef_ms), "score": 1e3 * score_avg,
-                        "normalize_select_compact": 1e3 * tail_avg} if fused else
-                       {"coef": 1e3 * statistics.mean(coef_ms), "score": 1e3 * score_avg,
-                        "normalize_select": 1e3 * tail_avg, "compact": 1e3 * compact_avg}),
-        "roofline": {"bound": "hbm", "kernel": "score_tc_kernel (scores of every candidate key)",
-                     "achieved": achieved, "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": recorded_traffic("score_kernel"),
-                     "algorithmic_bytes": score_bytes},
+        "kernels_us": {"coef": 1e3 * seg["coef"], "score_select": 1e3 * score_ms,
+                       "compact": 1e3 * seg["compact"]},
+        # the dominant kernel: scoring with each unit's normalize-then-max and
+        # selection fused; its algorithmic bytes are the K rows it reads once
+        "roofline": {"bound": "hbm",
+                     "kernel": "score_tc_kernel (scores of every candidate key; each unit's "
+                               "normalize-then-max and selection fused)",
+                     "achieved": k_bytes / (score_ms * 1e-3) / 1e9, "peak": hbm,
+                     "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": k_bytes / (score_ms * 1e-3) / 1e9 / hbm,
+                     "traffic": recorded_traffic("score_kernel"), "algorithmic_bytes": k_bytes,
+                     "pass": pass_roofline(k_bytes, compact_bytes, ms, hbm)},
+        "pass_roofline": pass_roofline(k_bytes, compact_bytes, ms, hbm),
         "compact_roofline": {
-            "kernel": "tail_compact_kernel (selection + compaction; raw-score reads included)"
-                      if fused else "compact_kernel",
-            "achieved": (compact_bytes + (raw_bytes if fused else 0)) / (move_ms * 1e-3) / 1e9,
+            "kernel": "compact_kernel", "achieved": compact_bytes / (seg["compact"] * 1e-3) / 1e9,
             "peak": hbm, "unit": "GB/s",
-            "frac": (compact_bytes + (raw_bytes if fused else 0)) / (move_ms * 1e-3) / 1e9 / hbm,
-            "algorithmic_bytes": compact_bytes, "raw_score_bytes": raw_bytes if fused else 0,
-            "moved_rows": moved},
+            "frac": compact_bytes / (seg["compact"] * 1e-3) / 1e9 / hbm,
+            "algorithmic_bytes": compact_bytes, "moved_rows": moved},
         "bracket_ms_per_step": br0.elapsed_time(br1) / args.steps,
         "clocks": clk.summary(),
-        "gpu_launches": (3 if fused else 4) * args.steps,
+        # coefficients, fused scoring + selection, compaction
+        "gpu_launches": 3 * args.steps,
     }
 
     if not args.no_extras:
         line["decode_attention"] = decode_attention(T, torch, w, st, cache, prm, ws, kept, restore,
                                                     cfg, hbm)
-        line["run16"] = run16(T, w, st, cache, prm, ws, kept, restore)
+        line["run16"] = run16(T, w, st, cache, prm, ws, kept, restore, hbm)
         line["calibration"] = calibration(T, torch, hbm)
         line["offset_max"] = offset_max(T, torch, st, cache, cfg, kept, restore, hbm)
         line["layer_budgets"] = layer_budgets(T, torch, w, st, cfg, restore, hbm)
@@ -413,26 +511,155 @@ def main():
             ms_e2e = max_over_ranks(line["e2e"]["ms_per_step"], dist, "cuda")
             line["e2e"]["ms_per_step"] = ms_e2e
             line["e2e"]["value"] = keys * world / (ms_e2e * 1e-3)
-        if rank == 0 and world == 1:
-            v, n_units, spent = oracle_unit_keys_per_s(cfg, args.cpu_seconds)
-            # the direct 17-offset form (Eq. 4), the reference-style scorer,
-            # on a bounded sample of the same workload
-            vd, nd_units, spent_d = oracle_unit_keys_per_s(cfg, 0.0, max_units=1, form="direct")
-            line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
-                                    "direct_form": {"value": vd, "unit": UNIT, "cores": 1,
-                                                    "sample": f"{nd_units} unit of {N} keys, "
-                                                              f"{spent_d:.1f} s, 17 offsets per band"},
-                                    "sample": f"{n_units} units of {N} keys (G={cfg.group}), "
-                                              f"{spent:.1f} s, fp64 numpy (single thread), "
-                                              "folded form + z-norm + selection"}
     T.tria_set_pass_events(None)
     st.free()
+    del w, kb, vb, pb, ws, kept, cache, flush
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    if not args.no_extras and world == 1:
+        # the other workload shapes, each timed on its own (one GPU)
+        line["workloads"] = {}
+        for ci in (1, 4, 3):
+            if ci == args.config:
+                continue
+            try:
+                line["workloads"][synth.CONFIGS[ci].name] = workload_pass(T, torch, ci, hbm)
+            except torch.cuda.OutOfMemoryError as e:
+                line["workloads"][synth.CONFIGS[ci].name] = {"error": f"out of memory: {e}"}
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+        if rank == 0:
+            line["cpu_baseline"] = cpu_baseline(args, cfg)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def split_events(all_evs):
+    """Mean per-kernel times (ms) of a list of tria_set_pass_events records:
+    coefficients, scoring (+ fused selection), a separate selection kernel
+    (modes without the fused tail), compaction, and the whole pass."""
+    seg = [statistics.mean(e[k].elapsed_time(e[k + 1]) for e in all_evs) for k in range(4)]
+    return {"coef": seg[0], "score": seg[1], "select": seg[2], "compact": seg[3],
+            "pass": statistics.mean(e[0].elapsed_time(e[4]) for e in all_evs)}
+
+
+def pass_roofline(k_bytes, compact_bytes, ms, hbm):
+    """The whole pass against the HBM bandwidth: K rows read once plus the
+    moved K/V rows read and written, over the pass time."""
+    tot = k_bytes + compact_bytes
+    return {"bound": "hbm", "achieved": tot / (ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+            "frac": tot / (ms * 1e-3) / 1e9 / hbm, "algorithmic_bytes": tot, "k_bytes": k_bytes,
+            "compact_bytes": compact_bytes, "us": ms * 1e3}
+
+
+def workload_pass(T, torch, ci, hbm, passes=None):
+    """One full compression pass of workload `ci` (the other shapes of the
+    pages' workloads), timed with the pass's own CUDA events.  Contiguous
+    caches restore the rows compaction overwrites between passes; the paged
+    batch (157.5 GB of K + V, no room for backups) is generated afresh
+    before each pass, after a warm-up pass of the same kernels on a small
+    instance of it."""
+    import synth
+
+    cfg = synth.CONFIGS[ci]
+    paged = cfg.layout == synth.LAYOUT_PAGED
+    passes = passes or (2 if paged else 5)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+
+    def load(wl):
+        re, im, am = wl.stats
+        return T.tria_load_stats(T.model_desc(wl.cfg.n_layers, wl.cfg.n_q_heads, wl.cfg.n_kv_heads,
+                                              wl.cfg.pairing, wl.cfg.theta,
+                                              wl.cfg.offset_log2_max), re, im, am)
+
+    if paged:
+        small = synth.Workload(cfg.scaled(n_layers=1, n_seq=2, len_range=(4096, 6000)),
+                               with_positions=False)
+        sst = load(small)
+        scache = T.Cache.from_workload(small)
+        sprm = T.params(small.cfg.budget, small.cfg.window, small.cfg.sinks)
+        sws = T.alloc_workspace(T.tria_workspace_size(sst, scache, sprm))
+        T.tria_compress_pass(sst, scache, sprm, None, sws)
+        torch.cuda.synchronize()
+        sst.free()
+        del small, scache, sws
+        torch.cuda.empty_cache()
+    w = synth.Workload(cfg, with_positions=not paged)
+    st = load(w)
+    try:
+        cache = T.Cache.from_workload(w)
+        prm = T.params(cfg.budget, cfg.window, cfg.sinks)
+        ws_bytes = T.tria_workspace_size(st, cache, prm)
+        ws = T.alloc_workspace(ws_bytes)
+        T.tria_read_device_status(ws)
+        B = cfg.budget
+        kept = torch.empty((cfg.n_seq, cfg.n_layers, cfg.n_kv_heads, B), dtype=torch.int32,
+                           device="cuda")
+        lens = w.seq_lens.clone()
+        if not paged:
+            kb = [t[:, :, :B].clone() for t in w.k]
+            vb = [t[:, :, :B].clone() for t in w.v]
+        zero = np.zeros(cfg.n_seq, dtype=np.int64)
+
+        def reset():
+            if paged:
+                w._fill(zero.astype(np.int32), w.lens.astype(np.int32), zero)
+            else:
+                for l in range(cfg.n_layers):
+                    w.k[l][:, :, :B].copy_(kb[l])
+                    w.v[l][:, :, :B].copy_(vb[l])
+            w.seq_lens.copy_(lens)
+            flush.zero_()
+
+        evs_all, moved = [], 0
+        for i in range(passes + (0 if paged else 2)):
+            reset()
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+            T.tria_set_pass_events(evs)
+            T.tria_compress_pass(st, cache, prm, kept, ws)
+            T.tria_set_pass_events(None)
+            if paged or i >= 2:
+                evs_all.append(evs)
+        torch.cuda.synchronize()
+        if T.tria_read_device_status(ws) != 0:
+            raise RuntimeError(f"device status flags set ({cfg.name})")
+        kh = kept.cpu().numpy()
+        moved = int(np.sum((kh >= 0) & (kh != np.arange(B)[None, None, None, :])))
+        seg = split_events(evs_all)
+        ms = seg["pass"]
+        lens_h = w.lens.astype(np.int64)
+        units = cfg.n_layers * cfg.n_kv_heads
+        keys = int(lens_h.sum()) * units
+        comp = lens_h > B
+        k_bytes = int(np.sum(lens_h[comp] - cfg.window - cfg.sinks)) * units * 256
+        compact_bytes = moved * 1024
+        out = {"workload": cfg.name, "us_per_pass": ms * 1e3, "keys_per_s": keys / (ms * 1e-3),
+               "keys": keys, "passes": passes,
+               "kernels_us": {"coef": 1e3 * seg["coef"], "score_select": 1e3 * seg["score"],
+                              "compact": 1e3 * seg["compact"]},
+               "roofline": {"bound": "hbm", "kernel": "score_tc_kernel (fused selection)",
+                            "achieved": k_bytes / (seg["score"] * 1e-3) / 1e9, "peak": hbm,
+                            "unit": "GB/s",
+                            "frac": k_bytes / (seg["score"] * 1e-3) / 1e9 / hbm,
+                            "algorithmic_bytes": k_bytes},
+               "pass_roofline": pass_roofline(k_bytes, compact_bytes, ms, hbm),
+               "moved_rows": moved,
+               "footprint_bytes": {"kv_cache": w.footprint_bytes(), "workspace": ws_bytes},
+               "restore": "cache generated afresh before each pass" if paged else
+                          "overwritten rows restored between passes, outside the events"}
+        if paged:
+            out["lengths"] = {"sum": int(lens_h.sum()), "min": int(lens_h.min()),
+                              "max": int(lens_h.max())}
+        return out
+    finally:
+        st.free()
+        del w
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
 
 
 def calibration(T, torch, hbm, reps=5):
@@ -545,8 +772,7 @@ def layer_budgets(T, torch, w, st, cfg, restore, hbm, passes=5):
     return {"workload": f"scales 0.5 .. 1.5 linear over {L} layers (budgets {min(budgets)} .. "
                         f"{max(budgets)}), lengths per (sequence, layer)",
             "us_per_pass": 1e3 * ms, "keys_per_s": units * cfg.seq_len / (ms * 1e-3),
-            "kernels_us": {"coef": 1e3 * statistics.mean(seg[0]), "score": 1e3 * score_ms,
-                           "normalize_select": 1e3 * statistics.mean(seg[2]),
+            "kernels_us": {"coef": 1e3 * statistics.mean(seg[0]), "score_select": 1e3 * score_ms,
                            "compact_and_lengths": 1e3 * statistics.mean(seg[3])},
             "score_roofline": {"bound": "hbm", "achieved": units * C * 256 / (score_ms * 1e-3) / 1e9,
                                "peak": hbm, "unit": "GB/s",
@@ -645,14 +871,19 @@ def decode_attention(T, torch, w, st, cache, prm, ws, kept, restore, cfg, hbm, r
             "sampled_layers": sample, "reps": reps}
 
 
-def run16(T, w, st, cache, prm, ws, kept, restore):
+def run16(T, w, st, cache, prm, ws, kept, restore, hbm):
     """The decode run: a first pass at 32K, then 15 passes each after 128
-    appended tokens (append excluded from the pass times)."""
+    appended tokens (append excluded from the pass times).  The steady
+    passes see N = budget + 128 rows per unit: their algorithmic bytes are
+    the candidates' K rows plus the moved K/V rows (read and written)."""
     import torch
 
     restore()
     torch.cuda.synchronize()
-    pass_us, append_ms = [], []
+    cfg = w.cfg
+    B = cfg.budget
+    units = cfg.n_seq * cfg.n_layers * cfg.n_kv_heads
+    pass_us, append_ms, moved, kbytes = [], [], [], []
     for i in range(16):
         if i:
             a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -661,16 +892,27 @@ def run16(T, w, st, cache, prm, ws, kept, restore):
             a1.record()
             torch.cuda.synchronize()
             append_ms.append(a0.elapsed_time(a1))
+        n = int(w.seq_lens[0].item())
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         T.tria_compress_pass(st, cache, prm, kept, ws)
         e1.record()
         torch.cuda.synchronize()
         pass_us.append(1e3 * e0.elapsed_time(e1))
+        kh = kept.cpu().numpy()
+        moved.append(int(np.sum((kh >= 0) & (kh != np.arange(B)[None, None, None, :]))))
+        kbytes.append(units * (n - cfg.window - cfg.sinks) * 256)
     w.next_pos = w.lens.astype(np.int64).copy()
     restore()
-    return {"first_pass_us": pass_us[0], "steady_pass_us_mean": statistics.mean(pass_us[1:]),
-            "steady_keys_per_pass": int(w.cfg.n_layers * w.cfg.n_kv_heads * (w.cfg.budget + 128)),
+    steady_us = statistics.mean(pass_us[1:])
+    steady_bytes = statistics.mean(kb + 1024 * m for kb, m in zip(kbytes[1:], moved[1:]))
+    return {"first_pass_us": pass_us[0], "steady_pass_us_mean": steady_us,
+            "steady_keys_per_pass": int(units * (B + 128)),
+            "steady_moved_rows_mean": statistics.mean(moved[1:]),
+            "steady_roofline": {"bound": "hbm", "algorithmic_bytes": steady_bytes,
+                                "achieved": steady_bytes / (steady_us * 1e-6) / 1e9, "peak": hbm,
+                                "unit": "GB/s",
+                                "frac": steady_bytes / (steady_us * 1e-6) / 1e9 / hbm},
             "total_pass_ms": sum(pass_us) / 1e3, "append_ms_mean": statistics.mean(append_ms)}
 
 

@@ -178,6 +178,13 @@ typedef struct {
                                         NULL = 1.0 for every layer                   */
   int interval;       /* compression interval beta >= 0 (0 and 1: compress whenever
                          N > B_l)                                                   */
+  int64_t wait_limit_ns; /* >= 0: bound, in ns, of every wait of the scoring kernel on
+                            its pipeline (tile loads, MMA results, hand-offs between
+                            its warps); 0 = 2 s.  A wait that runs out sets status
+                            bit 1 (tria_read_device_status), the kernel lets its own
+                            loads and MMAs land and returns; the call's results are
+                            then undefined.  A limit far below a kernel's run time
+                            makes that happen on purpose (tests of the abort path). */
 } tria_params;
 
 /* Human-readable name of a status code (static string). */
@@ -359,11 +366,13 @@ tria_status tria_compress_pass(const tria_stats *stats, const tria_cache_view *c
  *
  * Scratch: TRIA_STATIC_SCRATCH_BYTES (32 MiB, 256-byte aligned) of device
  * memory per device, held for as long as the library is loaded.  The first
- * call made while a given device is current looks up that device's address
- * of the array (cudaGetSymbolAddress, which may load the library's device
- * code on that device) and keeps it; make that first call on each device
- * before any stream capture begins.  The current device's array is used:
- * `stream` must belong to the current device.
+ * call made in a given CUDA context (per device; the context that follows a
+ * cudaDeviceReset counts as a new one) looks up that context's address of
+ * the array (cudaGetSymbolAddress, which may load the library's device code
+ * on that device) and keeps it, keyed by the context's id; make that first
+ * call on each device, and again after a reset, before any stream capture
+ * begins.  The current device's array is used: `stream` must belong to the
+ * current device.
  * Limit: the pass over all layers must need at most TRIA_STATIC_SCRATCH_BYTES
  * of workspace (tria_workspace_size with layers [0, n_layers)); a larger one
  * returns TRIA_ERR_WORKSPACE with nothing enqueued.  32 MiB holds, for
@@ -423,10 +432,12 @@ tria_status tria_calib_finalize(const tria_model_desc *desc, const double *acc, 
                                 tria_stream_t stream);
 
 /*
- * tria_read_device_status - errors the kernels found in device-resident
- * inputs during the calls that used this workspace (bit 0: a seq_lens entry
- * outside [0, max_seq_len]; such a unit is skipped and its kept row is all
- * -1), then clears them.  Synchronises `stream`.  *flags_out = 0 means none.
+ * tria_read_device_status - errors the kernels found during the calls that
+ * used this workspace, then clears them.  Bit 0: a seq_lens entry outside
+ * [0, max_seq_len] (such a unit is skipped and its kept row is all -1).
+ * Bit 1: a wait of the scoring kernel ran out (tria_params.wait_limit_ns);
+ * the kernel stopped early and the call's scores, kept rows and compaction
+ * are undefined.  Synchronises `stream`.  *flags_out = 0 means none.
  * The flags start undefined in a fresh workspace: read (and so clear) them
  * once before the first call.
  */

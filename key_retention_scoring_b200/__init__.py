@@ -66,7 +66,7 @@ class Params(ctypes.Structure):
     _fields_ = [("budget", ctypes.c_int), ("window", ctypes.c_int), ("sinks", ctypes.c_int),
                 ("offset_reduce", ctypes.c_int), ("budget_pct", ctypes.c_float),
                 ("layer_budget_scales", ctypes.POINTER(ctypes.c_float)),
-                ("interval", ctypes.c_int)]
+                ("interval", ctypes.c_int), ("wait_limit_ns", ctypes.c_int64)]
 
 
 _lib = None
@@ -280,12 +280,14 @@ class Cache:
 
 
 def params(budget, window, sinks, offset_reduce=0, budget_pct=0.0, layer_budget_scales=None,
-           interval=0) -> Params:
+           interval=0, wait_limit_ns=0) -> Params:
     """offset_reduce: OFFSET_MEAN (the published average over D) or OFFSET_MAX.
     budget_pct > 0: the budget is that percentage of the cache capacity;
     layer_budget_scales: per-layer multipliers of the budget (None: 1.0);
-    interval: a unit is compressed only once it is that many rows past its budget."""
-    prm = Params(budget, window, sinks, offset_reduce, float(budget_pct), None, int(interval))
+    interval: a unit is compressed only once it is that many rows past its budget;
+    wait_limit_ns: bound of each wait of the scoring kernel (0: 2 s)."""
+    prm = Params(budget, window, sinks, offset_reduce, float(budget_pct), None, int(interval),
+                 int(wait_limit_ns))
     if layer_budget_scales is not None:
         arr = (ctypes.c_float * len(layer_budget_scales))(*[float(x) for x in layer_budget_scales])
         prm._scales = arr  # kept alive with the parameters

@@ -47,7 +47,8 @@ tria_status make_geom(const tria_stats *stats, const tria_cache_view *cache,
   if (layer0 < 0 || layer1 <= layer0 || layer1 > d.n_layers) return TRIA_ERR_INVALID_ARG;
   if (cache->n_seq < 1 || cache->n_seq > TRIA_MAX_SEQS) return TRIA_ERR_INVALID_ARG;
   if (cache->max_seq_len < 1) return TRIA_ERR_INVALID_ARG;
-  if (params->window < 0 || params->sinks < 0 || params->interval < 0) return TRIA_ERR_INVALID_ARG;
+  if (params->window < 0 || params->sinks < 0 || params->interval < 0 || params->wait_limit_ns < 0)
+    return TRIA_ERR_INVALID_ARG;
   const double pct = params->budget_pct;  // the fp32 value, exactly
   if (!std::isfinite(pct) || pct < 0.0 || pct > 100.0) return TRIA_ERR_INVALID_ARG;
   if (cache->layout != TRIA_LAYOUT_CONTIGUOUS && cache->layout != TRIA_LAYOUT_PAGED)
@@ -276,8 +277,8 @@ CoefParams make_coef(const tria_stats *st, const Geom &g, const tria_cache_view 
   return cp;
 }
 
-tria_status make_score(const Geom &g, const tria_cache_view *c, int layer0, int layer1, void *ws,
-                       const WsLayout &wl, ScoreParams &sp) {
+tria_status make_score(const Geom &g, const tria_cache_view *c, const tria_params *prm, int layer0,
+                       int layer1, void *ws, const WsLayout &wl, ScoreParams &sp) {
   std::memset(&sp, 0, sizeof(sp));
   for (int l = layer0; l < layer1; ++l) {
     const tria_status st = k_tensor_map(c, g.hkv, c->k_layers[l], &sp.kmap[l - layer0]);
@@ -293,6 +294,13 @@ tria_status make_score(const Geom &g, const tria_cache_view *c, int layer0, int 
   sp.moments = at<double>(ws, wl.moments);
   sp.raw = at<float>(ws, wl.raw);
   sp.raw_stride = wl.raw_stride;
+  sp.wait_ns = (uint64_t)prm->wait_limit_ns;
+  // the fused tail's scratch (used only by the fused pass)
+  sp.unit_done = at<uint32_t>(ws, wl.unit_done);
+  sp.keys = at<uint32_t>(ws, wl.agg);
+  sp.keys_stride = wl.agg_stride;
+  sp.kept = nullptr;
+  sp.discard = 1;
   return TRIA_OK;
 }
 
@@ -517,7 +525,7 @@ tria_status tria_score(const tria_stats *stats, const tria_cache_view *cache,
   if ((st = check_workspace(g, ws, ws_bytes, &wl)) != TRIA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   static thread_local ScoreParams sp;
-  if ((st = make_score(g, cache, layer0, layer1, ws, wl, sp)) != TRIA_OK) return st;
+  if ((st = make_score(g, cache, params, layer0, layer1, ws, wl, sp)) != TRIA_OK) return st;
   TailParams tp = make_tail(g, cache, ws, wl);
   if (scores_out != nullptr) {
     sp.raw = scores_out;
@@ -531,7 +539,7 @@ tria_status tria_score(const tria_stats *stats, const tria_cache_view *cache,
   tp.discard_agg = 0;
   if (launch_coef(make_coef(stats, g, cache, ws, wl, nullptr, false), s) != cudaSuccess)
     return TRIA_ERR_CUDA;
-  if (launch_score(sp, s) != cudaSuccess) return TRIA_ERR_CUDA;
+  if (launch_score(sp, false, s) != cudaSuccess) return TRIA_ERR_CUDA;
   return cuda_status(launch_tail(tp, s));
 }
 
@@ -605,19 +613,26 @@ tria_status tria_compress_pass(const tria_stats *stats, const tria_cache_view *c
   int32_t *kept = kept_idx != nullptr ? kept_idx : at<int32_t>(ws, wl.kept);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   static thread_local ScoreParams sp;
-  if ((st = make_score(g, cache, 0, L, ws, wl, sp)) != TRIA_OK) return st;
+  if ((st = make_score(g, cache, params, 0, L, ws, wl, sp)) != TRIA_OK) return st;
+  sp.kept = kept;
+  // offset-mean mode: the scoring kernel also runs each unit's
+  // normalize-then-max and selection (its raw scores stay in L2); the
+  // max-over-offsets mode runs them in a separate kernel: one block per unit
+  // when the candidates' keys fit in shared memory, else blocks over
+  // candidate chunks with a histogram in the workspace
+  const bool fused = g.mode == TRIA_OFFSET_MEAN;
   TailParams tp = make_tail(g, cache, ws, wl);
   tp.kept = kept;
-  // one block per unit when its candidates' keys fit in shared memory, else
-  // blocks over candidate chunks with a histogram in the workspace
   const bool per_unit = unit_tail_fits(g);
   if (mark(0, s) != cudaSuccess) return TRIA_ERR_CUDA;
-  if (launch_coef(make_coef(stats, g, cache, ws, wl, kept, !per_unit), s) != cudaSuccess)
+  if (launch_coef(make_coef(stats, g, cache, ws, wl, kept, !fused && !per_unit), s) != cudaSuccess)
     return TRIA_ERR_CUDA;
   if (mark(1, s) != cudaSuccess) return TRIA_ERR_CUDA;
-  if (launch_score(sp, s) != cudaSuccess) return TRIA_ERR_CUDA;
+  if (launch_score(sp, fused, s) != cudaSuccess) return TRIA_ERR_CUDA;
   if (mark(2, s) != cudaSuccess) return TRIA_ERR_CUDA;
-  if ((per_unit ? launch_unit_tail(tp, s) : launch_tail(tp, s)) != cudaSuccess) return TRIA_ERR_CUDA;
+  if (!fused &&
+      (per_unit ? launch_unit_tail(tp, s) : launch_tail(tp, s)) != cudaSuccess)
+    return TRIA_ERR_CUDA;
   if (mark(3, s) != cudaSuccess) return TRIA_ERR_CUDA;
   CompactParams cp{};
   cp.geo = g;

@@ -8,18 +8,20 @@
 // depends only on the rotations already applied to q and k).
 //
 // Split-K flash decoding.  The rows of every (sequence, KV head) are shared
-// evenly by splits x 4 warps (about one block of 4 warps per SM in all); each
-// warp streams its range through a 3-deep ring of 32-row K/V tiles (cp.async)
-// and runs the two contractions on the tensor cores with warp-level
-// mma.sync (m16n8k16, bf16 inputs, fp32 accumulation), the G query heads
-// on the M side: S^T = Q K^T, an online softmax in base 2 in registers, and
-// O += P V with the weights split into bf16 hi + lo.  The block's warps merge their
-// (o, m, l) per head into the block's partial; the last block of each
-// (sequence, KV head) to finish rescales the partials to their common
-// maximum (an arrival count per unit in the workspace, reset by that block).  Decode attention at G <= 16 reads 512 bytes per row for 4 G
-// multiply-adds per byte, well below the tensor cores' balance point, so
-// the warp-level MMA (not the 128-row tcgen05 tile) is enough to leave the
-// kernel bound by HBM.
+// evenly by splits x 8 warps (about one block of 8 warps per SM in all); each
+// warp streams its range through a 3-deep ring of 16-row K/V tiles (cp.async
+// into XOR-swizzled shared memory, read with ldmatrix) and runs the two
+// contractions on the tensor cores with warp-level mma.sync (m16n8k16, bf16
+// inputs, fp32 accumulation), the 16 rows on the M side: S = K Q^T (heads as
+// N), an online softmax in base 2 in registers, and O^T += V^T P^T (the 128
+// dims as M) with each 8x8 block of P transposed in registers (movmatrix)
+// and split into bf16 hi + lo.  The block's warps merge their (o, m, l) per
+// head into the block's partial; the last block of each (sequence, KV head)
+// to finish rescales the partials to their common maximum (an arrival count
+// per unit in the workspace, reset by that block).  Decode attention at
+// G <= 16 reads 512 bytes per row for 4 G multiply-adds per byte, well below
+// the tensor cores' balance point, so the warp-level MMA (not the 128-row
+// tcgen05 tile) is enough to leave the kernel bound by HBM.
 #include <cmath>
 #include <cstdint>
 

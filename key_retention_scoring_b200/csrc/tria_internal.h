@@ -111,6 +111,14 @@ struct ScoreParams {
   double *moments;
   float *raw;           // [unit][raw_stride], per candidate G floats
   int64_t raw_stride;
+  uint64_t wait_ns;     // bound of every wait in the kernel (0: 2 s)
+  // the pass with its tail fused (the scoring kernel also runs, per unit,
+  // normalize-then-max and the selection once its last item is scored)
+  uint32_t *unit_done;  // [unit] items scored (zeroed by the coefficient kernel)
+  uint32_t *keys;       // [unit][keys_stride] order keys of agg (scratch)
+  int64_t keys_stride;  // multiple of 32
+  int32_t *kept;        // [unit][budget]
+  int discard;          // raw scores and keys are scratch: drop their L2 lines after use
 };
 
 // Normalize-then-max (and selection) kernel parameters.
@@ -176,7 +184,12 @@ struct LensParams {
 
 // Launchers (tria_kernels.cu).  Return cudaGetLastError() of the launch.
 cudaError_t launch_coef(const CoefParams &p, cudaStream_t st);
-cudaError_t launch_score(const ScoreParams &p, cudaStream_t st);
+// Scoring (tria_score_tc.cu): raw scores and moment partials of every
+// candidate; with fused != 0 (offset-mean mode) also the selection of every
+// compressed unit into p.kept.  The max-over-offsets mode is launched by
+// launch_score_max (tria_score_max.cu) and is never fused.
+cudaError_t launch_score(const ScoreParams &p, bool fused, cudaStream_t st);
+cudaError_t launch_score_max(const ScoreParams &p, cudaStream_t st);
 cudaError_t launch_tail(const TailParams &p, cudaStream_t st);
 cudaError_t launch_select(const SelectParams &p, cudaStream_t st);
 // Normalize-then-max + selection with one block per unit (kept != null);

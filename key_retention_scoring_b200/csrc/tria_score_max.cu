@@ -1,0 +1,338 @@
+// Scoring kernel of the max-over-offsets mode (tria_params.offset_reduce =
+// TRIA_OFFSET_MAX), the non-default variant named at the end of sec. 4 of
+// the academ.us article 2607.13051: the trigonometric term takes the
+// maximum over the future offsets delta_j in D instead of their mean.
+//
+// S_g(k) = max_j S_trig,g(k, Delta + delta_j) + S_norm,g(k).  The maximum is
+// not linear, so nothing folds: per (head g, offset delta_j) the coefficient
+// vector c_gj = E[q_g] mask e^{i omega (p_q + delta_j)} is its own bf16 hi/lo
+// column pair (2 |D| G columns, written by the coefficient kernel) and the
+// norm weights a separate 2G-column operand.  Per tile two contractions,
+// [k] (128 x 128) . Btrig (128 x 2 |D| G) into a trig accumulator (one or two
+// MMAs per K-step, N <= 256 each) and [m_hi | m_lo] . Bnorm (128 x 2G) into
+// a norm accumulator, then a max over the offset pairs in the epilogue.
+// Tensor memory holds one buffer of each (trig 0..271, norm 288.., magnitudes
+// 320..383), so a tile's epilogue runs before the next tile's MMAs; the
+// compute warps hide it behind the next tile's magnitude math (computed into
+// registers first, stored to tensor memory after the epilogue).
+//
+// Roles as in the offset-mean kernel (tria_score_tc.cu): warps 0-7 compute
+// (magnitudes, epilogue), warp 8 producer (TMA), warp 9 MMA issuer.  Bounded
+// waits and the abort path as described in tria_tc.cuh.
+#include "tria_tc.cuh"
+
+namespace tria {
+namespace {
+
+using namespace dev;
+using namespace tc;
+
+constexpr int kBandGroups = 2;
+constexpr int kBandsPerThread = kBands / kBandGroups;
+constexpr int kComputeWarps = 4 * kBandGroups;
+constexpr int kProducerWarp = kComputeWarps;
+constexpr int kMmaWarp = kComputeWarps + 1;
+constexpr int kThreads = 32 * (kComputeWarps + 2);
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kMaxNormCol = 288, kMaxMagCol = 320;
+
+template <int G>
+struct MaxCfg {
+  static constexpr int NN = (2 * G < 16) ? 16 : 2 * G;                  // norm columns
+  static constexpr int NT_MAX = ((2 * 17 * G + 15) / 16) * 16;          // trig columns at |D| = 17
+  static constexpr int STAGES = (G >= 8) ? 2 : 4;
+  static constexpr int BMAX = (NT_MAX + NN) * 256;                       // coefficient image bytes
+  static constexpr int GQ = (G >= kBandGroups) ? G / kBandGroups : 1;
+};
+
+template <int G>
+struct MaxSmem {
+  alignas(1024) uint8_t k[MaxCfg<G>::STAGES][2][kHalfBlock];
+  alignas(1024) uint8_t b[2][MaxCfg<G>::BMAX];
+  alignas(8) uint64_t full[MaxCfg<G>::STAGES];
+  alignas(8) uint64_t kempty[MaxCfg<G>::STAGES];
+  alignas(8) uint64_t aready;
+  alignas(8) uint64_t accfull;
+  alignas(8) uint64_t bempty[2];
+  SubRec rec[MaxCfg<G>::STAGES];
+  alignas(16) int seq_items[kMaxSeqTable];
+  int seq_len[kMaxSeqTable];
+  uint32_t tmem_base;
+  volatile int abort_flag;
+  __device__ __forceinline__ uint8_t *bbuf(int i) { return &b[i][0]; }
+};
+
+template <int G>
+__device__ void mma_issuer_max(const ScoreParams &p, MaxSmem<G> &sm, uint32_t tmem,
+                               const WaitCtl &wc) {
+  using Cfg = MaxCfg<G>;
+  constexpr int ST = Cfg::STAGES, NN = Cfg::NN;
+  const int NT = p.geo.ncol_t;
+  const int N1 = NT < 256 ? NT : 256, N2 = NT - N1;
+  const uint32_t id1 = idesc_bf16_m128_n(N1), id2 = idesc_bf16_m128_n(N2 > 0 ? N2 : 16);
+  constexpr uint32_t idn = idesc_bf16_m128_n(NN);
+  const uint64_t da0 = sw128_desc(smem_u32(&sm.k[0][0][0]));
+  const uint64_t db0 = sw128_desc(smem_u32(&sm.b[0][0]));
+  constexpr uint32_t kStageBytes = 2 * kHalfBlock;
+  const uint32_t nbase = 2u * NT * 128u;  // norm image after the trig image
+  int i = 0;
+  for (;; ++i) {
+    if (!mbar_wait(&sm.aready, i & 1, wc)) break;
+    tc_fence_after();
+    const int stage = i % ST;
+    const SubRec &rec = sm.rec[stage];
+    const int flags = rec.flags, bpar = rec.bpar;
+    if (flags & kFlagEnd) break;
+    const uint64_t da = da0 + (uint64_t)((stage * kStageBytes) >> 4);
+    const uint64_t db = db0 + (uint64_t)(((uint32_t)bpar * (uint32_t)Cfg::BMAX) >> 4);
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const uint32_t ao = (s >> 2) * kHalfBlock + (s & 3) * 32;
+      const uint32_t bo = (uint32_t)(s >> 2) * (uint32_t)NT * 128u + (s & 3) * 32;
+      mma_bf16(tmem, da + (ao >> 4), db + (bo >> 4), id1, s > 0 ? 1u : 0u);
+      if (N2 > 0)
+        mma_bf16(tmem + (uint32_t)N1, da + (ao >> 4), db + ((bo + (uint32_t)N1 * 128u) >> 4), id2,
+                 s > 0 ? 1u : 0u);
+    }
+    mma_commit(&sm.kempty[stage]);  // the K tile is consumed
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const uint32_t bo = nbase + (uint32_t)(s >> 2) * NN * 128u + (s & 3) * 32;
+      mma_bf16_ta(tmem + kMaxNormCol, tmem + kMaxMagCol + (uint32_t)(s * 8), db + (bo >> 4), idn,
+                  s > 0 ? 1u : 0u);
+    }
+    if (flags & kFlagLast) mma_commit(&sm.bempty[bpar]);
+    mma_commit(&sm.accfull);
+  }
+  if (i > 0) mbar_drain(&sm.accfull, (i - 1) & 1, wc.status);
+}
+
+// Raw scores, fp64 moment sums and the item's moment partials of one tile.
+template <int G>
+__device__ __forceinline__ void emit_scores(const ScoreParams &p, const EpRec &pr,
+                                            const float (&sc)[MaxCfg<G>::GQ], bool active, int q,
+                                            int rg, int lane, double (&msum)[MaxCfg<G>::GQ],
+                                            double (&msq)[MaxCfg<G>::GQ]) {
+  constexpr int GQ = MaxCfg<G>::GQ;
+  const Geom &geo = p.geo;
+  if (pr.flags & kFlagFirst) {
+#pragma unroll
+    for (int g = 0; g < GQ; ++g) msum[g] = msq[g] = 0.0;
+  }
+  if (active) {
+    const int slot = pr.slot0 + rg * 32 + lane;
+    if (slot >= geo.sinks && slot < pr.N - geo.window) {
+#pragma unroll
+      for (int g = 0; g < GQ; ++g) {
+        msum[g] += (double)sc[g];
+        msq[g] = fma((double)sc[g], (double)sc[g], msq[g]);
+      }
+      float *dst = ep_raw(p, pr) + (slot - geo.sinks) * G + q * GQ;
+#pragma unroll
+      for (int g = 0; g < GQ; ++g) dst[g] = sc[g];
+    }
+  }
+  if ((pr.flags & kFlagLast) && active) {
+#pragma unroll
+    for (int g = 0; g < GQ; ++g) {
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) {
+        msum[g] += __shfl_xor_sync(kFull, msum[g], o);
+        msq[g] += __shfl_xor_sync(kFull, msq[g], o);
+      }
+    }
+    if (lane == 0) {
+      double *m = ep_mom(p, pr) + (rg * G + q * GQ) * 2;
+#pragma unroll
+      for (int g = 0; g < GQ; ++g) {
+        m[2 * g] = msum[g];
+        m[2 * g + 1] = msq[g];
+      }
+    }
+  }
+}
+
+// Maximum that returns NaN when either operand is NaN.
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
+// Epilogue of the previous tile: per head of this thread's band group,
+// S = max_j (hi_j + lo_j) + (norm hi + norm lo).
+template <int G>
+__device__ __forceinline__ void epilogue_max(const ScoreParams &p, uint32_t tmem, const EpRec &pr,
+                                             int q, int rg, int lane, double (&msum)[MaxCfg<G>::GQ],
+                                             double (&msq)[MaxCfg<G>::GQ]) {
+  constexpr int GQ = MaxCfg<G>::GQ;
+  const bool active = (G >= kBandGroups) || q < G;
+  const int nd = p.geo.n_off;
+  float sc[GQ];
+  if (active) {
+    const uint32_t lb = tmem + ((uint32_t)(32 * rg) << 16);
+#pragma unroll
+    for (int gi = 0; gi < GQ; ++gi) {
+      const int g = q * GQ + gi;
+      // the head's 2 nd columns: one 32-column load (offsets 0..15; beyond
+      // 2 nd it reads the next head's columns, unused) and one 2-column load
+      // for offset 16
+      uint32_t t[32], t16[2], nv[2];
+      const uint32_t c0 = lb + (uint32_t)(g * nd * 2);
+      tmem_ld_nowait<32>(c0, t);
+      if (nd == 17) tmem_ld_nowait<2>(c0 + 32, t16);
+      tmem_ld_nowait<2>(lb + kMaxNormCol + (uint32_t)(2 * g), nv);
+      tmem_wait_ld();
+      // offsets past |D| read as -inf; a pairwise tree of NaN-propagating
+      // maxes, built in place over the loaded words
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        t[j] = __float_as_uint((j < nd) ? __uint_as_float(t[2 * j]) + __uint_as_float(t[2 * j + 1])
+                                        : -INFINITY);
+      const float v16 = (nd == 17) ? __uint_as_float(t16[0]) + __uint_as_float(t16[1]) : -INFINITY;
+#pragma unroll
+      for (int w = 1; w < 16; w *= 2) {
+#pragma unroll
+        for (int j = 0; j + w < 16; j += 2 * w)
+          t[j] = __float_as_uint(max_nan(__uint_as_float(t[j]), __uint_as_float(t[j + w])));
+      }
+      const float m = max_nan(__uint_as_float(t[0]), v16);
+      sc[gi] = m + (__uint_as_float(nv[0]) + __uint_as_float(nv[1]));
+    }
+  } else {
+#pragma unroll
+    for (int gi = 0; gi < GQ; ++gi) sc[gi] = 0.0f;
+  }
+  tc_fence_before();
+  emit_scores<G>(p, pr, sc, active, q, rg, lane, msum, msq);
+}
+
+template <int G, int PAIR>
+__device__ void compute_max(const ScoreParams &p, MaxSmem<G> &sm, uint32_t tmem, int tid,
+                            const WaitCtl &wc) {
+  constexpr int ST = MaxCfg<G>::STAGES, GQ = MaxCfg<G>::GQ, W = kBandsPerThread / 2;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int q = warp >> 2, rg = warp & 3, r = rg * 32 + lane;
+  const uint32_t mag = tmem + ((uint32_t)(32 * rg) << 16) + kMaxMagCol;
+  double msum[GQ], msq[GQ];
+#pragma unroll
+  for (int g = 0; g < GQ; ++g) msum[g] = msq[g] = 0.0;
+  EpRec prev{};
+  for (int i = 0;; ++i) {
+    const int stage = i % ST;
+    if (!warp_wait(&sm.full[stage], (i / ST) & 1, wc, lane)) return;
+    const SubRec &rc = sm.rec[stage];
+    const int flags = rc.flags;
+    const bool end = (flags & kFlagEnd) != 0;
+    EpRec cur{};
+    uint32_t hi[W], lo[W];
+    if (!end) {
+      cur = ep_of(rc);
+      mags_regs<PAIR, kBandsPerThread>(&sm.k[stage][0][0], r, q, hi, lo);
+    }
+    if (i >= 1) {
+      // the previous tile's MMAs are done: its scores, and its magnitude
+      // buffer may be overwritten
+      if (!warp_wait(&sm.accfull, (i - 1) & 1, wc, lane)) return;
+      tc_fence_after();
+      epilogue_max<G>(p, tmem, prev, q, rg, lane, msum, msq);
+    }
+    if (!end) {
+      tmem_st<W>(mag + (uint32_t)(W * q), hi);
+      tmem_st<W>(mag + (uint32_t)(32 + W * q), lo);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.aready);
+    if (end) return;
+    prev = cur;
+  }
+}
+
+template <int G, int PAIR, int LAYOUT>
+__global__ void __launch_bounds__(kThreads, 1) score_max_kernel(const __grid_constant__ ScoreParams p) {
+  using Cfg = MaxCfg<G>;
+  extern __shared__ uint8_t smem_dyn[];
+  MaxSmem<G> &sm = *reinterpret_cast<MaxSmem<G> *>(
+      (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
+  const Geom &geo = p.geo;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  for (int i = tid; i <= geo.n_seq; i += kThreads) sm.seq_items[i] = p.seq_items[i];
+  for (int i = tid; i < geo.n_seq; i += kThreads) sm.seq_len[i] = unit_len(geo, i, 0);
+  if (tid == 0) {
+    for (int i = 0; i < Cfg::STAGES; ++i) {
+      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.kempty[i], 1);
+    }
+    mbar_init(&sm.aready, kComputeWarps);
+    mbar_init(&sm.accfull, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&sm.bempty[i], 1);
+    sm.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == kMmaWarp) tmem_alloc(&sm.tmem_base, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const int n_items = sm.seq_items[geo.n_seq];
+  const WaitCtl wc = wait_ctl(&sm.abort_flag, p.status, p.wait_ns);
+
+  if (warp < kComputeWarps) {
+    compute_max<G, PAIR>(p, sm, tmem, tid, wc);
+  } else if (warp == kProducerWarp) {
+    producer<Cfg::STAGES, LAYOUT>(p, sm, n_items, lane, wc);
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) mma_issuer_max<G>(p, sm, tmem, wc);
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int G, int PAIR, int LAYOUT>
+cudaError_t launch_max_t(const ScoreParams &p, cudaStream_t st) {
+  auto kern = score_max_kernel<G, PAIR, LAYOUT>;
+  const int smem = (int)sizeof(MaxSmem<G>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  kern<<<sms, kThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int G>
+cudaError_t launch_max_g(const ScoreParams &p, cudaStream_t st) {
+  const bool paged = p.cache.layout == TRIA_LAYOUT_PAGED;
+  if (p.geo.pairing == TRIA_PAIR_NEOX)
+    return paged ? launch_max_t<G, TRIA_PAIR_NEOX, TRIA_LAYOUT_PAGED>(p, st)
+                 : launch_max_t<G, TRIA_PAIR_NEOX, TRIA_LAYOUT_CONTIGUOUS>(p, st);
+  return paged ? launch_max_t<G, TRIA_PAIR_INTERLEAVED, TRIA_LAYOUT_PAGED>(p, st)
+               : launch_max_t<G, TRIA_PAIR_INTERLEAVED, TRIA_LAYOUT_CONTIGUOUS>(p, st);
+}
+
+static_assert(sizeof(MaxSmem<8>) + 1024 <= 232448, "shared memory of the G=8 max-mode kernel");
+static_assert(sizeof(MaxSmem<4>) + 1024 <= 232448, "shared memory of the G=4 max-mode kernel");
+static_assert(MaxCfg<8>::NT_MAX <= 288 - 16, "max-mode trig columns");
+
+}  // namespace
+
+cudaError_t launch_score_max(const ScoreParams &p, cudaStream_t st) {
+  switch (p.geo.g) {
+    case 1: return launch_max_g<1>(p, st);
+    case 2: return launch_max_g<2>(p, st);
+    case 4: return launch_max_g<4>(p, st);
+    case 8: return launch_max_g<8>(p, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace tria

@@ -11,6 +11,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/tria.h"
@@ -22,21 +23,62 @@ static __device__ __align__(256) unsigned char g_scratch[TRIA_STATIC_SCRATCH_BYT
 constexpr int kMaxDevices = 64;
 constexpr size_t kHeaderBytes = 256;  // work counter (bytes 0..3), status flags (4..7)
 
-std::mutex g_mu;
-void *g_scratch_ptr[kMaxDevices] = {};
+// The array's device address belongs to a CUDA context: after a device reset
+// the next context loads the library's device code again, possibly at
+// another address.  So the cached address is keyed by the id of the context
+// it was looked up in (cuCtxGetId: unique for the life of the process).
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  void *ptr;
+};
 
-// Address of the array on the current device; looked up once per device.
+std::mutex g_mu;
+ScratchEntry g_scratch_of[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Id of the calling thread's current context; false if there is none yet.
+bool current_ctx_id(unsigned long long *id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *a = nullptr, *b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+        qa == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+        qb == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+      get_id = reinterpret_cast<CtxGetIdFn>(b);
+    }
+  });
+  if (get_current == nullptr || get_id == nullptr) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Address of the array in the current device's context: looked up once per
+// context (cudaGetSymbolAddress, which also makes the device's primary
+// context current if no context is yet).
 tria_status scratch_of_current_device(void **out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return TRIA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return TRIA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  unsigned long long id = 0;
+  const bool have_id = current_ctx_id(&id);
+  ScratchEntry &e = g_scratch_of[dev];
+  if (!have_id || e.ptr == nullptr || e.ctx_id != id) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return TRIA_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
+    if (!current_ctx_id(&id)) return TRIA_ERR_CUDA;
+    e.ctx_id = id;
+    e.ptr = p;
   }
-  *out = g_scratch_ptr[dev];
+  *out = e.ptr;
   return TRIA_OK;
 }
 
