@@ -274,6 +274,8 @@ CoefParams make_coef(const tria_stats *st, const Geom &g, const tria_cache_view 
   cp.row_items = at<int32_t>(ws, wl.row_items);
   cp.kept = kept;
   cp.hist = with_hist ? at<uint32_t>(ws, wl.hist) : nullptr;
+  cp.tailq = at<int32_t>(ws, wl.tailq);
+  cp.tq = at<uint32_t>(ws, wl.hdr + 8);
   return cp;
 }
 
@@ -301,6 +303,8 @@ tria_status make_score(const Geom &g, const tria_cache_view *c, const tria_param
   sp.keys_stride = wl.agg_stride;
   sp.kept = nullptr;
   sp.discard = 1;
+  sp.tailq = at<int32_t>(ws, wl.tailq);
+  sp.tq = at<uint32_t>(ws, wl.hdr + 8);
   return TRIA_OK;
 }
 
@@ -361,6 +365,7 @@ WsLayout ws_layout(const Geom &g) {
   w.raw = take((size_t)g.n_units * w.raw_stride * 4);
   w.agg = take((size_t)g.n_units * w.agg_stride * 4);
   w.kept = take((size_t)g.n_units * g.budget * 4);
+  w.tailq = take((size_t)g.n_units * 4);
   w.total = off;
   return w;
 }

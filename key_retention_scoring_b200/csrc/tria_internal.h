@@ -73,7 +73,8 @@ struct CacheDev {
 
 // Workspace carve-up (byte offsets from the workspace base).
 struct WsLayout {
-  size_t hdr;         // 256 B: u32 item counter, i32 status flags
+  size_t hdr;         // 256 B: u32 item counter, i32 status flags, u32 tail queue
+                      // [put, get, units to compress]
   size_t unit_done;   // n_units x u32: finished normalization chunks per unit
   size_t seq_items;   // (n_seq + 1) x i32 prefix of scheduling items per sequence
   size_t row_items;   // (n_seq x nl + 1) x i32 prefix per (sequence, layer) (per-layer lengths)
@@ -83,6 +84,7 @@ struct WsLayout {
   size_t raw;         // n_units x raw_stride fp32
   size_t agg;         // n_units x agg_stride fp32
   size_t kept;        // n_units x budget i32
+  size_t tailq;       // n_units x i32: units whose tails are due, in completion order
   size_t total;
   int64_t raw_stride; // floats per unit, multiple of 32
   int64_t agg_stride; // floats per unit, multiple of 32
@@ -119,6 +121,9 @@ struct ScoreParams {
   int64_t keys_stride;  // multiple of 32
   int32_t *kept;        // [unit][budget]
   int discard;          // raw scores and keys are scratch: drop their L2 lines after use
+  int32_t *tailq;       // [unit] completed units in order (-1: not yet), any block's tail
+                        // warps take the next one
+  uint32_t *tq;         // [0] units queued, [1] units taken, [2] units compressed by the pass
 };
 
 // Normalize-then-max (and selection) kernel parameters.
@@ -152,6 +157,8 @@ struct CoefParams {
   int32_t *status;
   int32_t *kept;      // identity rows for units that are not compressed (may be null)
   uint32_t *hist;     // zeroed per unit (may be null)
+  int32_t *tailq;     // set to -1 per unit
+  uint32_t *tq;       // reset; [2] = units the pass compresses
 };
 
 struct SelectParams {

@@ -36,13 +36,19 @@
 //   warp 10     item warp: when the compute warps finish an item (all its
 //               raw scores and moment partials written) it counts the item
 //               in the unit's device-wide counter; the block that completes
-//               a unit queues the unit's tail for its tail warps;
-//   warps 11-14 tail warps: per queued unit, the mean and std of each head
-//               from the moment partials, the aggregated order keys (read
-//               from the raw scores, which are still in L2), and the radix
-//               selection over the keys into the ascending kept list.  They
-//               run next to the scoring roles, on the issue slots those
-//               leave free.
+//               a unit appends it to a device-wide queue of due tails;
+//   warps 11-14 tail warps: take the next due unit from that queue, whichever
+//               block completed it, and run its tail: the mean and std of
+//               each head from the moment partials, the aggregated order
+//               keys (read from the raw scores, which are still in L2), and
+//               the radix selection over the keys into the ascending kept
+//               list.  They run next to the scoring roles, on the issue
+//               slots those leave free.  Taking units from one queue keeps
+//               the tails spread over the blocks: a block slowed by its
+//               tails would otherwise finish the last items of more units
+//               and draw still more tails.  The tail warps wait on other
+//               blocks, so the kernel is launched cooperatively (every block
+//               resident).
 // The raw scores then never need to reach HBM: the tail reads them back
 // from L2 within microseconds of their writing and drops the lines.
 // Every wait is bounded (ScoreParams::wait_ns); on expiry the kernel flags
@@ -68,7 +74,6 @@ constexpr int kTailThreads = 32 * kTailWarps;
 constexpr int kTailBar = 2;                 // named barrier of the tail warps
 constexpr int kTailLoads = 8;               // float4 raw-score loads in flight per tail thread
 constexpr int kItemRing = 8;                // finished-item records in flight
-constexpr int kTailRing = 8;                // queued unit tails
 template <bool FUSED>
 __host__ __device__ constexpr int tc_threads() {
   return 32 * (kComputeWarps + 2 + (FUSED ? 1 + kTailWarps : 0));
@@ -97,8 +102,7 @@ struct TcCfg {
   static_assert(kNB * NACC * NCOL <= 256, "accumulator columns");
 };
 
-// A finished item, from the compute warps to the item warp, and a unit
-// whose tail is due, from the item warp to the tail warps.
+// A finished item, from the compute warps to the item warp.
 struct ItemPost {
   long long u;
   int N, end;
@@ -109,13 +113,9 @@ struct TailArea {
   uint2 list[kListCap];
   GroupScalars<kTailWarps> sc;
   ItemPost irec[kItemRing];
-  ItemPost tjob[kTailRing];
-  ItemPost act_job[2];
-  int act[2];
+  int act[2];                               // the unit the tail group takes next (-1: none)
   alignas(8) uint64_t idone[kItemRing];
   alignas(8) uint64_t ifree[kItemRing];
-  alignas(8) uint64_t tready[kTailRing];
-  alignas(8) uint64_t tfree[kTailRing];
 };
 
 template <bool FUSED>
@@ -353,60 +353,79 @@ __device__ void compute(const ScoreParams &p, TcSmem<G, FUSED> &sm, uint32_t tme
 // ---------------------------------------------------------------------------
 // fused pass: item warp and tail warps
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ int ld_acquire(const int32_t *a) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release(int32_t *a, int v) {
+  asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
+}
+
 template <int G>
 __device__ void item_warp(const ScoreParams &p, TailArea &ta, int lane, const WaitCtl &wc) {
   const Geom &geo = p.geo;
-  int queued = 0;
-  auto queue = [&](const ItemPost &job) -> bool {
-    const int slot = queued % kTailRing;
-    if (queued >= kTailRing &&
-        !warp_wait(&ta.tfree[slot], ((queued / kTailRing) - 1) & 1, wc, lane))
-      return false;
-    if (lane == 0) {
-      ta.tjob[slot] = job;
-      mbar_arrive(&ta.tready[slot]);
-    }
-    __syncwarp();
-    ++queued;
-    return true;
-  };
   for (int j = 0;; ++j) {
     const int slot = j % kItemRing;
     if (!warp_wait(&ta.idone[slot], (j / kItemRing) & 1, wc, lane)) return;
     const ItemPost ip = ta.irec[slot];
     __syncwarp();
     if (lane == 0) mbar_arrive(&ta.ifree[slot]);  // the record is copied
-    if (ip.end) {
-      queue(ip);
-      return;
-    }
+    if (ip.end) return;
     // Count the item in the unit's device-wide counter.  The compute warps'
     // raw-score and moment writes precede their arrivals on idone (release,
     // block scope), this warp acquired them by its wait, and the fence
     // below (cumulative) orders them before the count at device scope; the
-    // block that takes the last count fences again before its tail reads.
-    int last = 0;
+    // block that takes the last count fences again and publishes the unit
+    // with a release store, which the tail warps that take it acquire.
     if (lane == 0) {
       const int ntiles = unit_tiles(ip.N, geo.window, geo.sinks);
       __threadfence();
       const uint32_t old = atomicAdd(p.unit_done + ip.u, 1u);
       if (old + 1u == (uint32_t)ntiles) {
         __threadfence();
-        last = 1;
+        const uint32_t at = atomicAdd(p.tq, 1u);
+        st_release(p.tailq + at, (int)ip.u);
       }
     }
-    last = __shfl_sync(kFull, last, 0);
-    if (last && !queue(ip)) return;
+    __syncwarp();
   }
 }
 
+// Tail warp 0: the next due unit (device-wide order), or -1 when every unit
+// the pass compresses has been taken, or on abort or expiry.  Lane 0 claims
+// the next queue position and waits (bounded) until a block publishes the
+// unit that completes there.
+__device__ int claim_tail(const ScoreParams &p, int lane, const WaitCtl &wc) {
+  int u = -1;
+  if (lane == 0) {
+    const uint32_t at = atomicAdd(p.tq + 1, 1u);
+    if (at < __ldcg(p.tq + 2)) {
+      const uint64_t t0 = global_timer();
+      for (;;) {
+        u = ld_acquire(p.tailq + at);
+        if (u >= 0) break;
+        if (*wc.abort_flag) break;
+        if (global_timer() - t0 > wc.limit_ns) {
+          flag_expiry(wc);
+          break;
+        }
+        __nanosleep(500);
+      }
+    }
+  }
+  return __shfl_sync(kFull, u, 0);
+}
+
 template <int G>
-__device__ void run_tail(const ScoreParams &p, TailArea &ta, const ItemPost &job, int tt) {
+__device__ void run_tail(const ScoreParams &p, TailArea &ta, long long u, int tt) {
   const Geom &geo = p.geo;
-  const long long u = job.u;
-  const int N = job.N;
+  const int s = (int)(u / ((int64_t)geo.nl * geo.hkv));
+  const int lrel = (int)((u / geo.hkv) % geo.nl);
+  const int N = unit_len(geo, s, lrel);
   const int C = N - geo.window - geo.sinks;
-  const int B = geo.lbudget[(int)((u / geo.hkv) % geo.nl)];
+  const int B = geo.lbudget[lrel];
   unit_norm<G, kTailBar, kTailThreads>(p.moments + u * geo.tiles_max * kRowGroups * G * 2,
                                        unit_tiles(N, geo.window, geo.sinks), C, tt, ta.sc);
   clear_words<kTailThreads>(ta.hist, kHistBins, tt);
@@ -432,29 +451,18 @@ __device__ void run_tail(const ScoreParams &p, TailArea &ta, const ItemPost &job
 template <int G>
 __device__ void tail_warps(const ScoreParams &p, TailArea &ta, int tt, const WaitCtl &wc) {
   const int lane = tt & 31;
-  // tail warp 0 takes each queued unit and hands it to the group through
+  // tail warp 0 takes each due unit and hands it to the group through
   // shared memory (the other tail warps wait at the group barrier only, so
   // no tail warp is left waiting for one that stopped)
   for (int j = 0;; ++j) {
-    const int slot = j % kTailRing;
     if (tt < 32) {
-      int act = 0;  // 0: stop, 1: run the unit's tail
-      ItemPost job{};
-      if (warp_wait(&ta.tready[slot], (j / kTailRing) & 1, wc, lane)) {
-        job = ta.tjob[slot];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ta.tfree[slot]);
-        act = job.end ? 0 : 1;
-      }
-      if (lane == 0) {
-        ta.act[j & 1] = act;
-        ta.act_job[j & 1] = job;
-      }
+      const int u = claim_tail(p, lane, wc);
+      if (lane == 0) ta.act[j & 1] = u;
     }
     csync<kTailBar, kTailThreads>();
-    if (ta.act[j & 1] == 0) return;
-    const ItemPost job = ta.act_job[j & 1];
-    run_tail<G>(p, ta, job, tt);
+    const int u = ta.act[j & 1];
+    if (u < 0) return;
+    run_tail<G>(p, ta, u, tt);
   }
 }
 
@@ -486,10 +494,6 @@ __global__ void __launch_bounds__(tc_threads<FUSED>(), 1)
       for (int i = 0; i < kItemRing; ++i) {
         mbar_init(&ta.idone[i], kComputeWarps);
         mbar_init(&ta.ifree[i], 1);
-      }
-      for (int i = 0; i < kTailRing; ++i) {
-        mbar_init(&ta.tready[i], 1);
-        mbar_init(&ta.tfree[i], 1);
       }
     }
     sm.abort_flag = 0;
@@ -531,8 +535,23 @@ cudaError_t launch_t(const ScoreParams &p, cudaStream_t st) {
   int dev = 0, sms = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  kern<<<sms, tc_threads<FUSED>(), smem, st>>>(p);
-  return cudaGetLastError();
+  if constexpr (FUSED) {
+    // the tail warps wait on other blocks: every block must be resident
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)sms);
+    cfg.blockDim = dim3((unsigned)tc_threads<FUSED>());
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
+  } else {
+    kern<<<sms, tc_threads<FUSED>(), smem, st>>>(p);
+    return cudaGetLastError();
+  }
 }
 
 template <int G, bool FUSED>

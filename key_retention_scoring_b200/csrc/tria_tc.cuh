@@ -447,13 +447,19 @@ __device__ void producer(const ScoreParams &p, Smem &sm, int n_items, int lane, 
         if (sm.seq_items[mid] <= it) lo = mid; else hi = mid - 1;
       }
       s = lo;
+      // Items of a (sequence, layer) row take the row's KV heads in turn
+      // (item k of the row: tile k / hkv of head k % hkv), so the last items
+      // of the row's units are claimed one after another by different
+      // blocks: the blocks that complete units, and run their tails, rotate
+      // over the whole grid instead of repeating with the item count.
       if (!geo.per_layer) {
         ntiles = (sm.seq_items[s + 1] - sm.seq_items[s]) / units_per_seq;
         const int rem = it - sm.seq_items[s];
-        const int ul = rem / ntiles;
-        tile = rem % ntiles;
-        lrel = ul / geo.hkv;
-        h = ul % geo.hkv;
+        const int row_n = geo.hkv * ntiles;
+        lrel = rem / row_n;
+        const int idx = rem - lrel * row_n;
+        tile = idx / geo.hkv;
+        h = idx - tile * geo.hkv;
         N = sm.seq_len[s];
       } else {
         // a length per (sequence, layer): the layer is the last row of the
@@ -469,8 +475,8 @@ __device__ void producer(const ScoreParams &p, Smem &sm, int n_items, int lane, 
         N = unit_len(geo, s, lrel);
         ntiles = unit_tiles(N, W, S);
         const int rem = it - __ldcg(ri + lrel);
-        h = rem / ntiles;
-        tile = rem % ntiles;
+        tile = rem / geo.hkv;
+        h = rem - tile * geo.hkv;
       }
       u = (long long)s * units_per_seq + lrel * geo.hkv + h;
       tbase = (S / kTileKeys + tile) * kTileKeys;
