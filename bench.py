@@ -473,13 +473,12 @@ def main():
                     "operands), moments in fp64, selection on fp32 agg",
         "us_per_pass": ms * 1e3,
         "keys_per_s_per_query_head": keys * world * cfg.group / (ms * 1e-3),
-        "kernels_us": {"coef": 1e3 * seg["coef"], "score_select": 1e3 * score_ms,
-                       "compact": 1e3 * seg["compact"]},
-        # the dominant kernel: scoring with each unit's normalize-then-max and
-        # selection fused; its algorithmic bytes are the K rows it reads once
+        "kernels_us": {"coef": 1e3 * seg["coef"], "score": 1e3 * score_ms,
+                       "normalize_select": 1e3 * seg["select"], "compact": 1e3 * seg["compact"]},
+        # the dominant kernel: scoring; its algorithmic bytes are the K rows
+        # it reads once
         "roofline": {"bound": "hbm",
-                     "kernel": "score_tc_kernel (scores of every candidate key; each unit's "
-                               "normalize-then-max and selection fused)",
+                     "kernel": "score_tc_kernel (scores of every candidate key)",
                      "achieved": k_bytes / (score_ms * 1e-3) / 1e9, "peak": hbm,
                      "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": k_bytes / (score_ms * 1e-3) / 1e9 / hbm,
@@ -493,8 +492,8 @@ def main():
             "algorithmic_bytes": compact_bytes, "moved_rows": moved},
         "bracket_ms_per_step": br0.elapsed_time(br1) / args.steps,
         "clocks": clk.summary(),
-        # coefficients, fused scoring + selection, compaction
-        "gpu_launches": 3 * args.steps,
+        # coefficients, scoring, normalize-then-max + selection, compaction
+        "gpu_launches": 4 * args.steps,
     }
 
     if not args.no_extras:
@@ -540,8 +539,8 @@ def main():
 
 def split_events(all_evs):
     """Mean per-kernel times (ms) of a list of tria_set_pass_events records:
-    coefficients, scoring (+ fused selection), a separate selection kernel
-    (modes without the fused tail), compaction, and the whole pass."""
+    coefficients, scoring, normalize-then-max + selection, compaction, and
+    the whole pass."""
     seg = [statistics.mean(e[k].elapsed_time(e[k + 1]) for e in all_evs) for k in range(4)]
     return {"coef": seg[0], "score": seg[1], "select": seg[2], "compact": seg[3],
             "pass": statistics.mean(e[0].elapsed_time(e[4]) for e in all_evs)}
@@ -639,9 +638,10 @@ def workload_pass(T, torch, ci, hbm, passes=None):
         compact_bytes = moved * 1024
         out = {"workload": cfg.name, "us_per_pass": ms * 1e3, "keys_per_s": keys / (ms * 1e-3),
                "keys": keys, "passes": passes,
-               "kernels_us": {"coef": 1e3 * seg["coef"], "score_select": 1e3 * seg["score"],
+               "kernels_us": {"coef": 1e3 * seg["coef"], "score": 1e3 * seg["score"],
+                              "normalize_select": 1e3 * seg["select"],
                               "compact": 1e3 * seg["compact"]},
-               "roofline": {"bound": "hbm", "kernel": "score_tc_kernel (fused selection)",
+               "roofline": {"bound": "hbm", "kernel": "score_tc_kernel",
                             "achieved": k_bytes / (seg["score"] * 1e-3) / 1e9, "peak": hbm,
                             "unit": "GB/s",
                             "frac": k_bytes / (seg["score"] * 1e-3) / 1e9 / hbm,
@@ -772,7 +772,8 @@ def layer_budgets(T, torch, w, st, cfg, restore, hbm, passes=5):
     return {"workload": f"scales 0.5 .. 1.5 linear over {L} layers (budgets {min(budgets)} .. "
                         f"{max(budgets)}), lengths per (sequence, layer)",
             "us_per_pass": 1e3 * ms, "keys_per_s": units * cfg.seq_len / (ms * 1e-3),
-            "kernels_us": {"coef": 1e3 * statistics.mean(seg[0]), "score_select": 1e3 * score_ms,
+            "kernels_us": {"coef": 1e3 * statistics.mean(seg[0]), "score": 1e3 * score_ms,
+                           "normalize_select": 1e3 * statistics.mean(seg[2]),
                            "compact_and_lengths": 1e3 * statistics.mean(seg[3])},
             "score_roofline": {"bound": "hbm", "achieved": units * C * 256 / (score_ms * 1e-3) / 1e9,
                                "peak": hbm, "unit": "GB/s",

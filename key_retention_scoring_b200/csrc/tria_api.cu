@@ -274,8 +274,6 @@ CoefParams make_coef(const tria_stats *st, const Geom &g, const tria_cache_view 
   cp.row_items = at<int32_t>(ws, wl.row_items);
   cp.kept = kept;
   cp.hist = with_hist ? at<uint32_t>(ws, wl.hist) : nullptr;
-  cp.tailq = at<int32_t>(ws, wl.tailq);
-  cp.tq = at<uint32_t>(ws, wl.hdr + 8);
   return cp;
 }
 
@@ -297,14 +295,6 @@ tria_status make_score(const Geom &g, const tria_cache_view *c, const tria_param
   sp.raw = at<float>(ws, wl.raw);
   sp.raw_stride = wl.raw_stride;
   sp.wait_ns = (uint64_t)prm->wait_limit_ns;
-  // the fused tail's scratch (used only by the fused pass)
-  sp.unit_done = at<uint32_t>(ws, wl.unit_done);
-  sp.keys = at<uint32_t>(ws, wl.agg);
-  sp.keys_stride = wl.agg_stride;
-  sp.kept = nullptr;
-  sp.discard = 1;
-  sp.tailq = at<int32_t>(ws, wl.tailq);
-  sp.tq = at<uint32_t>(ws, wl.hdr + 8);
   return TRIA_OK;
 }
 
@@ -365,7 +355,6 @@ WsLayout ws_layout(const Geom &g) {
   w.raw = take((size_t)g.n_units * w.raw_stride * 4);
   w.agg = take((size_t)g.n_units * w.agg_stride * 4);
   w.kept = take((size_t)g.n_units * g.budget * 4);
-  w.tailq = take((size_t)g.n_units * 4);
   w.total = off;
   return w;
 }
@@ -544,7 +533,7 @@ tria_status tria_score(const tria_stats *stats, const tria_cache_view *cache,
   tp.discard_agg = 0;
   if (launch_coef(make_coef(stats, g, cache, ws, wl, nullptr, false), s) != cudaSuccess)
     return TRIA_ERR_CUDA;
-  if (launch_score(sp, false, s) != cudaSuccess) return TRIA_ERR_CUDA;
+  if (launch_score(sp, s) != cudaSuccess) return TRIA_ERR_CUDA;
   return cuda_status(launch_tail(tp, s));
 }
 
@@ -619,25 +608,18 @@ tria_status tria_compress_pass(const tria_stats *stats, const tria_cache_view *c
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   static thread_local ScoreParams sp;
   if ((st = make_score(g, cache, params, 0, L, ws, wl, sp)) != TRIA_OK) return st;
-  sp.kept = kept;
-  // offset-mean mode: the scoring kernel also runs each unit's
-  // normalize-then-max and selection (its raw scores stay in L2); the
-  // max-over-offsets mode runs them in a separate kernel: one block per unit
-  // when the candidates' keys fit in shared memory, else blocks over
-  // candidate chunks with a histogram in the workspace
-  const bool fused = g.mode == TRIA_OFFSET_MEAN;
   TailParams tp = make_tail(g, cache, ws, wl);
   tp.kept = kept;
+  // one block per unit when its candidates' keys fit in shared memory, else
+  // blocks over candidate chunks with a histogram in the workspace
   const bool per_unit = unit_tail_fits(g);
   if (mark(0, s) != cudaSuccess) return TRIA_ERR_CUDA;
-  if (launch_coef(make_coef(stats, g, cache, ws, wl, kept, !fused && !per_unit), s) != cudaSuccess)
+  if (launch_coef(make_coef(stats, g, cache, ws, wl, kept, !per_unit), s) != cudaSuccess)
     return TRIA_ERR_CUDA;
   if (mark(1, s) != cudaSuccess) return TRIA_ERR_CUDA;
-  if (launch_score(sp, fused, s) != cudaSuccess) return TRIA_ERR_CUDA;
+  if (launch_score(sp, s) != cudaSuccess) return TRIA_ERR_CUDA;
   if (mark(2, s) != cudaSuccess) return TRIA_ERR_CUDA;
-  if (!fused &&
-      (per_unit ? launch_unit_tail(tp, s) : launch_tail(tp, s)) != cudaSuccess)
-    return TRIA_ERR_CUDA;
+  if ((per_unit ? launch_unit_tail(tp, s) : launch_tail(tp, s)) != cudaSuccess) return TRIA_ERR_CUDA;
   if (mark(3, s) != cudaSuccess) return TRIA_ERR_CUDA;
   CompactParams cp{};
   cp.geo = g;

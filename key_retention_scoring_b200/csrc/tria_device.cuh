@@ -520,15 +520,12 @@ struct alignas(16) UnitScalars {  // 16-byte size: the key area after it is read
   float inv[TRIA_MAX_GROUP];
 };
 
-// U: float4 loads in flight per thread.  CG: raw scores read at L2 only
-// (written by other blocks of the same kernel), else as a stream.  keys may
-// be shared or global memory.
-template <int G, int NT, int U = 8, bool CG = false>
+template <int G, int NT>
 __device__ void unit_keys(const float *raw, int C, const float *s_mean, const float *s_inv,
                           uint32_t *keys, uint32_t *hist, int tid) {
   const int lane = tid & 31;
+  constexpr int U = 8;  // float4 loads in flight per thread
   const float4 *src = reinterpret_cast<const float4 *>(raw);
-  auto ld = [&](const float4 *a) { return CG ? __ldcg(a) : __ldcs(a); };
   if constexpr (G >= 4) {
     // LPC lanes per candidate, each with 4 of its G heads
     constexpr int LPC = G / 4;
@@ -545,7 +542,7 @@ __device__ void unit_keys(const float *raw, int C, const float *s_mean, const fl
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int j = j0 + u * NT + tid;
-        x[u] = (j < n4) ? ld(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[u] = (j < n4) ? __ldcs(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -582,7 +579,7 @@ __device__ void unit_keys(const float *raw, int C, const float *s_mean, const fl
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int j = j0 + u * NT + tid;
-        x[u] = (j < n4) ? ld(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[u] = (j < n4) ? __ldcs(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -787,157 +784,6 @@ __device__ void select_keys(const uint32_t *keys, int C, int K, int N, int B, in
   }
 }
 
-
-// ---------------------------------------------------------------------------
-// Selection of one unit over order keys in global memory (the keys of a
-// unit whose candidates do not fit in shared memory, or whose tail runs
-// next to other work).  keys[c] for c < C, readable (as uint4) up to
-// ceil(C / 32) * 32 entries; hist (shared) holds the histogram of bits
-// [31:20] of all C keys on entry.  Digits of 12, 12 and 8 bits:
-//   1. the first digit's bin from hist;
-//   2. one pass over the keys gathers the keys of that bin into the list
-//      (up to kListCap) and histograms their second digit;
-//   3. the third digit from the list (or, when the bin is larger than the
-//      list, from one more pass over the keys) gives the threshold key T and
-//      the number `need` of keys equal to T that are kept (lowest slots);
-//   4. one emission pass in slot order: thread t of round r takes the 32
-//      keys of word r NT + t and keeps those above T and, by a block scan of
-//      the tie counts, the first `need` keys equal to T; a block scan of the
-//      kept counts places them in the ascending kept list.
-// kept receives sinks, the selected candidates and the window (as
-// select_keys).  Runs on a group of NT threads (barrier BAR).
-// ---------------------------------------------------------------------------
-template <int NW>
-struct GroupScalars {
-  int warp_tmp[NW];
-  uint32_t prefix;
-  int remaining;
-  int digit;
-  int above;
-  int bin_count;
-  int list_n;
-  float mean[TRIA_MAX_GROUP];
-  float inv[TRIA_MAX_GROUP];
-};
-
-// the 32 keys of word w (entries past C read as 0 and masked by the caller)
-__device__ __forceinline__ void load_word(const uint32_t *keys, int w, uint32_t (&k)[32]) {
-  const uint4 *src = reinterpret_cast<const uint4 *>(keys + (int64_t)w * 32);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint4 v = __ldcg(src + i);
-    k[4 * i] = v.x;
-    k[4 * i + 1] = v.y;
-    k[4 * i + 2] = v.z;
-    k[4 * i + 3] = v.w;
-  }
-}
-
-template <int BAR, int NT, class Sc>
-__device__ void select_global(const uint32_t *keys, int C, int K, int N, int B, int W, int S,
-                              int32_t *kept, uint32_t *hist, uint2 *list, Sc &sc, int tid) {
-  const int lane = tid & 31;
-  for (int j = tid; j < S; j += NT) kept[j] = j;
-  for (int j = tid; j < W; j += NT) kept[B - W + j] = N - W + j;
-  if (K <= 0) return;
-  if (tid == 0) {
-    sc.prefix = 0u;
-    sc.remaining = K;
-    sc.list_n = 0;
-  }
-  csync<BAR, NT>();
-  pick_bin<BAR, NT>(hist, kHistBins, sc, 20, tid);
-  const uint32_t d1 = sc.prefix >> 20;
-  clear_words<NT>(hist, kHistBins, tid);
-  csync<BAR, NT>();
-  const int nw = (C + 31) / 32;
-  // pass over the keys: the first digit's bin -> list, second-digit histogram
-  for (int w = tid; w - tid < nw; w += NT) {
-    uint32_t k[32];
-    uint32_t inm = 0u;
-    if (w < nw) {
-      load_word(keys, w, k);
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        inm |= (32 * w + i < C && (k[i] >> 20) == d1) ? (1u << i) : 0u;
-    }
-    const int cnt = __popc(inm);
-    const int incl = warp_incl_scan(cnt, lane);
-    int base = 0;
-    if (lane == 31 && incl > 0) base = atomicAdd(&sc.list_n, incl);
-    base = __shfl_sync(kFull, base, 31);
-    if (inm) {
-      int idx = base + incl - cnt;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        if ((inm >> i) & 1u) {
-          atomicAdd(hist + ((k[i] >> 8) & 0xfffu), 1u);
-          if (idx < kListCap) list[idx] = make_uint2(k[i], (uint32_t)(32 * w + i));
-          ++idx;
-        }
-      }
-    }
-  }
-  csync<BAR, NT>();
-  pick_bin<BAR, NT>(hist, kHistBins, sc, 8, tid);
-  const int ln = sc.list_n;
-  clear_words<NT>(hist, 256, tid);
-  csync<BAR, NT>();
-  const uint32_t p24 = sc.prefix >> 8;
-  if (ln <= kListCap) {
-    for (int i = tid; i < ln; i += NT) {
-      const uint32_t k = list[i].x;
-      if ((k >> 8) == p24) atomicAdd(hist + (k & 0xffu), 1u);
-    }
-  } else {
-    for (int w = tid; w < nw; w += NT) {
-      uint32_t k[32];
-      load_word(keys, w, k);
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (32 * w + i < C && (k[i] >> 8) == p24) atomicAdd(hist + (k[i] & 0xffu), 1u);
-    }
-  }
-  csync<BAR, NT>();
-  pick_bin<BAR, NT>(hist, 256, sc, 0, tid);
-  const uint32_t T = sc.prefix;
-  const int need = sc.remaining;  // keys equal to T to keep, lowest slots first (>= 1)
-  // emission in slot order
-  int run_keep = 0, run_eq = 0;
-  for (int w0 = 0; w0 < nw && run_keep < K; w0 += NT) {
-    const int w = w0 + tid;
-    uint32_t gtm = 0u, eqm = 0u;
-    if (w < nw) {
-      uint32_t k[32];
-      load_word(keys, w, k);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const bool valid = 32 * w + i < C;
-        gtm |= (valid && k[i] > T) ? (1u << i) : 0u;
-        eqm |= (valid && k[i] == T) ? (1u << i) : 0u;
-      }
-    }
-    const int ne = __popc(eqm);
-    int tot_e;
-    const int rank = run_eq + block_excl_scan<BAR, NT>(ne, tid, sc.warp_tmp, &tot_e);
-    uint32_t keepm = gtm;
-    for (int take = min(ne, need - rank); take > 0; --take) {
-      keepm |= eqm & (0u - eqm);  // lowest remaining tie of this word
-      eqm &= eqm - 1u;
-    }
-    const int nk = __popc(keepm);
-    int tot_k;
-    int pos = run_keep + block_excl_scan<BAR, NT>(nk, tid, sc.warp_tmp, &tot_k);
-    while (keepm) {
-      const int b = __ffs(keepm) - 1;
-      if (pos < K) kept[S + pos] = S + 32 * w + b;
-      ++pos;
-      keepm &= keepm - 1u;
-    }
-    run_eq += tot_e;
-    run_keep += tot_k;
-  }
-}
 
 }  // namespace dev
 }  // namespace tria

@@ -73,8 +73,7 @@ struct CacheDev {
 
 // Workspace carve-up (byte offsets from the workspace base).
 struct WsLayout {
-  size_t hdr;         // 256 B: u32 item counter, i32 status flags, u32 tail queue
-                      // [put, get, units to compress]
+  size_t hdr;         // 256 B: u32 item counter, i32 status flags
   size_t unit_done;   // n_units x u32: finished normalization chunks per unit
   size_t seq_items;   // (n_seq + 1) x i32 prefix of scheduling items per sequence
   size_t row_items;   // (n_seq x nl + 1) x i32 prefix per (sequence, layer) (per-layer lengths)
@@ -84,7 +83,6 @@ struct WsLayout {
   size_t raw;         // n_units x raw_stride fp32
   size_t agg;         // n_units x agg_stride fp32
   size_t kept;        // n_units x budget i32
-  size_t tailq;       // n_units x i32: units whose tails are due, in completion order
   size_t total;
   int64_t raw_stride; // floats per unit, multiple of 32
   int64_t agg_stride; // floats per unit, multiple of 32
@@ -114,16 +112,6 @@ struct ScoreParams {
   float *raw;           // [unit][raw_stride], per candidate G floats
   int64_t raw_stride;
   uint64_t wait_ns;     // bound of every wait in the kernel (0: 2 s)
-  // the pass with its tail fused (the scoring kernel also runs, per unit,
-  // normalize-then-max and the selection once its last item is scored)
-  uint32_t *unit_done;  // [unit] items scored (zeroed by the coefficient kernel)
-  uint32_t *keys;       // [unit][keys_stride] order keys of agg (scratch)
-  int64_t keys_stride;  // multiple of 32
-  int32_t *kept;        // [unit][budget]
-  int discard;          // raw scores and keys are scratch: drop their L2 lines after use
-  int32_t *tailq;       // [unit] completed units in order (-1: not yet), any block's tail
-                        // warps take the next one
-  uint32_t *tq;         // [0] units queued, [1] units taken, [2] units compressed by the pass
 };
 
 // Normalize-then-max (and selection) kernel parameters.
@@ -157,8 +145,6 @@ struct CoefParams {
   int32_t *status;
   int32_t *kept;      // identity rows for units that are not compressed (may be null)
   uint32_t *hist;     // zeroed per unit (may be null)
-  int32_t *tailq;     // set to -1 per unit
-  uint32_t *tq;       // reset; [2] = units the pass compresses
 };
 
 struct SelectParams {
@@ -192,10 +178,9 @@ struct LensParams {
 // Launchers (tria_kernels.cu).  Return cudaGetLastError() of the launch.
 cudaError_t launch_coef(const CoefParams &p, cudaStream_t st);
 // Scoring (tria_score_tc.cu): raw scores and moment partials of every
-// candidate; with fused != 0 (offset-mean mode) also the selection of every
-// compressed unit into p.kept.  The max-over-offsets mode is launched by
-// launch_score_max (tria_score_max.cu) and is never fused.
-cudaError_t launch_score(const ScoreParams &p, bool fused, cudaStream_t st);
+// candidate; the max-over-offsets mode is launched by launch_score_max
+// (tria_score_max.cu).
+cudaError_t launch_score(const ScoreParams &p, cudaStream_t st);
 cudaError_t launch_score_max(const ScoreParams &p, cudaStream_t st);
 cudaError_t launch_tail(const TailParams &p, cudaStream_t st);
 cudaError_t launch_select(const SelectParams &p, cudaStream_t st);

@@ -59,12 +59,7 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
   __shared__ int s_part[kThreads];
 
   if (u == 0) {
-    if (t == 0) {
-      *p.item_counter = 0u;
-      p.tq[0] = 0u;
-      p.tq[1] = 0u;
-    }
-    int comp_units = 0;  // units the pass compresses (this thread's share)
+    if (t == 0) *p.item_counter = 0u;
     if (!g.per_layer) {
       // one length per sequence: items per sequence, prefix over sequences
       // (n_seq <= 1024: <= 4 per thread)
@@ -74,10 +69,7 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
         const int sq = t * per + i;
         if (sq < g.n_seq) {
           const int n = unit_len(g, sq, 0);
-          if (compresses(g, n, 0)) {
-            local += unit_tiles(n, g.window, g.sinks) * g.nl * g.hkv;
-            comp_units += g.nl * g.hkv;
-          }
+          if (compresses(g, n, 0)) local += unit_tiles(n, g.window, g.sinks) * g.nl * g.hkv;
         }
       }
       int total;
@@ -103,10 +95,7 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
       int local = 0;
       for (int i = 0; i < per; ++i) {
         const int r = t * per + i;
-        if (r < rows) {
-          local += row_n(r);
-          comp_units += row_n(r) > 0 ? g.hkv : 0;
-        }
+        if (r < rows) local += row_n(r);
       }
       int total;
       int run = block_excl_scan<0, kThreads>(local, t, s_part, &total);
@@ -123,13 +112,9 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
         p.seq_items[g.n_seq] = total;
       }
     }
-    int n_comp;
-    block_excl_scan<0, kThreads>(comp_units, t, s_part, &n_comp);
-    if (t == 0) p.tq[2] = (uint32_t)n_comp;
   }
   if (t == 0) {
     p.unit_done[u] = 0u;
-    p.tailq[u] = -1;
     if (bad && h == 0 && (lrel == 0 || g.per_layer)) atomicOr(p.status, 1);
   }
   if (p.hist != nullptr)

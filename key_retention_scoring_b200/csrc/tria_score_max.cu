@@ -64,7 +64,7 @@ struct MaxSmem {
 
 template <int G>
 __device__ void mma_issuer_max(const ScoreParams &p, MaxSmem<G> &sm, uint32_t tmem,
-                               const WaitCtl &wc) {
+                               const WaitCtl wc) {
   using Cfg = MaxCfg<G>;
   constexpr int ST = Cfg::STAGES, NN = Cfg::NN;
   const int NT = p.geo.ncol_t;
@@ -209,7 +209,7 @@ __device__ __forceinline__ void epilogue_max(const ScoreParams &p, uint32_t tmem
 
 template <int G, int PAIR>
 __device__ void compute_max(const ScoreParams &p, MaxSmem<G> &sm, uint32_t tmem, int tid,
-                            const WaitCtl &wc) {
+                            const WaitCtl wc) {
   constexpr int ST = MaxCfg<G>::STAGES, GQ = MaxCfg<G>::GQ, W = kBandsPerThread / 2;
   const int warp = tid >> 5, lane = tid & 31;
   const int q = warp >> 2, rg = warp & 3, r = rg * 32 + lane;

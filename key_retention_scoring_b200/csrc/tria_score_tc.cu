@@ -29,31 +29,11 @@
 //               released), 8 steps with A = the magnitude tile in tensor
 //               memory, and tcgen05.commit.  Consecutive steps accumulate
 //               into NACC different partial accumulators (summed by the
-//               epilogue), so they do not wait on each other's results;
-// and, in the fused pass (academ.us article 2607.13051, sec. 4: the
-// normalize-then-max consumes the per-head scores of the whole unit, so it
-// starts once the unit's last key is scored):
-//   warp 10     item warp: when the compute warps finish an item (all its
-//               raw scores and moment partials written) it counts the item
-//               in the unit's device-wide counter; the block that completes
-//               a unit appends it to a device-wide queue of due tails;
-//   warps 11-14 tail warps: take the next due unit from that queue, whichever
-//               block completed it, and run its tail: the mean and std of
-//               each head from the moment partials, the aggregated order
-//               keys (read from the raw scores, which are still in L2), and
-//               the radix selection over the keys into the ascending kept
-//               list.  They run next to the scoring roles, on the issue
-//               slots those leave free.  Taking units from one queue keeps
-//               the tails spread over the blocks: a block slowed by its
-//               tails would otherwise finish the last items of more units
-//               and draw still more tails.  The tail warps wait on other
-//               blocks, so the kernel is launched cooperatively (every block
-//               resident).
-// The raw scores then never need to reach HBM: the tail reads them back
-// from L2 within microseconds of their writing and drops the lines.
-// Every wait is bounded (ScoreParams::wait_ns); on expiry the kernel flags
-// status bit 1, lets its own loads and MMAs land, frees its tensor memory
-// and returns.
+//               epilogue), so they do not wait on each other's results.
+// Normalize-then-max and the selection run in the next kernel (the unit tail
+// in tria_kernels.cu).  Every wait is bounded (ScoreParams::wait_ns); on
+// expiry the kernel flags status bit 1, lets its own loads and MMAs land,
+// frees its tensor memory and returns.
 #include "tria_tc.cuh"
 
 namespace tria {
@@ -67,17 +47,7 @@ constexpr int kBandsPerThread = kBands / kBandGroups;
 constexpr int kComputeWarps = 4 * kBandGroups;
 constexpr int kProducerWarp = kComputeWarps;
 constexpr int kMmaWarp = kComputeWarps + 1;
-constexpr int kItemWarp = kComputeWarps + 2;
-constexpr int kTailWarp0 = kComputeWarps + 3;
-constexpr int kTailWarps = 4;
-constexpr int kTailThreads = 32 * kTailWarps;
-constexpr int kTailBar = 2;                 // named barrier of the tail warps
-constexpr int kTailLoads = 8;               // float4 raw-score loads in flight per tail thread
-constexpr int kItemRing = 8;                // finished-item records in flight
-template <bool FUSED>
-__host__ __device__ constexpr int tc_threads() {
-  return 32 * (kComputeWarps + 2 + (FUSED ? 1 + kTailWarps : 0));
-}
+constexpr int kTcThreads = 32 * (kComputeWarps + 2);
 // The epilogue of tile i runs after the magnitudes of tile i + 2, so two MMA
 // chains are in flight while the compute warps work; magnitude tiles and
 // accumulators rotate through kNB tensor-memory buffers (tile i uses i % kNB,
@@ -87,69 +57,44 @@ constexpr int kNB = 4;
 constexpr uint32_t kTmemCols = 512;         // [0, 256): accumulators; [256, 512): magnitude tiles
 constexpr uint32_t kTmemMag = 256;
 
-template <int G, bool FUSED>
+template <int G>
 struct TcCfg {
   static constexpr int NCOL = (2 * G < 16) ? 16 : 2 * G;   // MMA N
-  // K ring depth: the fused pass gives shared memory to the tail
-  static constexpr int STAGES = FUSED ? ((G <= 8) ? 5 : 4) : ((G <= 8) ? 6 : 5);
+  static constexpr int STAGES = (G <= 8) ? 6 : 5;
   static constexpr int GQ = (G >= kBandGroups) ? G / kBandGroups : 1;  // heads per band group
   static constexpr int BBLK = NCOL * 128;                  // bytes per 64-wide K block of B
   // Consecutive K-steps of a tile accumulate into NACC partial accumulators
   // (summed by the epilogue): an N = 16 MMA is a few tensor-pipe cycles, far
-  // below the latency of its result, so a single accumulator would chain the
-  // tile's 16 MMAs on that latency
-  static constexpr int NACC = (NCOL <= 16) ? 4 : 2;
+  // below the latency of its result, so one accumulator would chain the
+  // tile's 16 MMAs on that latency; two chains of eight measured faster than
+  // four of four (fewer epilogue additions)
+  static constexpr int NACC = 2;
   static_assert(kNB * NACC * NCOL <= 256, "accumulator columns");
 };
 
-// A finished item, from the compute warps to the item warp.
-struct ItemPost {
-  long long u;
-  int N, end;
-};
-
-struct TailArea {
-  uint32_t hist[kHistBins];
-  uint2 list[kListCap];
-  GroupScalars<kTailWarps> sc;
-  ItemPost irec[kItemRing];
-  int act[2];                               // the unit the tail group takes next (-1: none)
-  alignas(8) uint64_t idone[kItemRing];
-  alignas(8) uint64_t ifree[kItemRing];
-};
-
-template <bool FUSED>
-struct TailPart {};
-template <>
-struct TailPart<true> {
-  TailArea t;
-};
-
-template <int G, bool FUSED>
+template <int G>
 struct TcSmem {
-  alignas(1024) uint8_t k[TcCfg<G, FUSED>::STAGES][2][kHalfBlock];
-  alignas(1024) uint8_t b[2][4][TcCfg<G, FUSED>::BBLK];
-  alignas(8) uint64_t full[TcCfg<G, FUSED>::STAGES];
-  alignas(8) uint64_t kempty[TcCfg<G, FUSED>::STAGES];
+  alignas(1024) uint8_t k[TcCfg<G>::STAGES][2][kHalfBlock];
+  alignas(1024) uint8_t b[2][4][TcCfg<G>::BBLK];
+  alignas(8) uint64_t full[TcCfg<G>::STAGES];
+  alignas(8) uint64_t kempty[TcCfg<G>::STAGES];
   alignas(8) uint64_t aready[kNB];
   alignas(8) uint64_t accfull[kNB];
   alignas(8) uint64_t bempty[2];
-  SubRec rec[TcCfg<G, FUSED>::STAGES];
+  SubRec rec[TcCfg<G>::STAGES];
   alignas(16) int seq_items[kMaxSeqTable];
   int seq_len[kMaxSeqTable];
   uint32_t tmem_base;
   volatile int abort_flag;
-  TailPart<FUSED> tp;
   __device__ __forceinline__ uint8_t *bbuf(int i) { return &b[i][0][0]; }
 };
 
 // ---------------------------------------------------------------------------
 // MMA issuer (one lane)
 // ---------------------------------------------------------------------------
-template <int G, bool FUSED>
-__device__ void mma_issuer(const ScoreParams &p, TcSmem<G, FUSED> &sm, uint32_t tmem,
-                           const WaitCtl &wc) {
-  using Cfg = TcCfg<G, FUSED>;
+template <int G>
+__device__ void mma_issuer(const ScoreParams &p, TcSmem<G> &sm, uint32_t tmem, const WaitCtl wc) {
+  using Cfg = TcCfg<G>;
   constexpr int ST = Cfg::STAGES, NCOL = Cfg::NCOL, BBLK = Cfg::BBLK, NACC = Cfg::NACC;
   constexpr uint32_t idesc = idesc_bf16_m128_n(NCOL);
   // descriptors of stage 0 / coefficient buffer 0; an operand at byte offset
@@ -204,12 +149,12 @@ __device__ __forceinline__ void mags(const uint8_t *kt, uint32_t tcol, int r, in
 
 // Epilogue of tile j (record pr): raw scores of this warp's 32 rows and GQ
 // heads, fp64 moment sums, and the item's moment partials after its last tile.
-template <int G, bool FUSED>
-__device__ __forceinline__ bool epilogue(const ScoreParams &p, TcSmem<G, FUSED> &sm, uint32_t tmem,
-                                         int j, const EpRec &pr, int q, int rg, int lane,
-                                         double (&msum)[TcCfg<G, FUSED>::GQ],
-                                         double (&msq)[TcCfg<G, FUSED>::GQ], const WaitCtl &wc) {
-  constexpr int NCOL = TcCfg<G, FUSED>::NCOL, GQ = TcCfg<G, FUSED>::GQ;
+template <int G>
+__device__ __forceinline__ bool epilogue(const ScoreParams &p, TcSmem<G> &sm, uint32_t tmem, int j,
+                                         const EpRec &pr, int q, int rg, int lane,
+                                         double (&msum)[TcCfg<G>::GQ], double (&msq)[TcCfg<G>::GQ],
+                                         const WaitCtl wc) {
+  constexpr int NCOL = TcCfg<G>::NCOL, GQ = TcCfg<G>::GQ, NACC = TcCfg<G>::NACC;
   const Geom &geo = p.geo;
   const bool active = (G >= kBandGroups) || q < G;  // group q scores heads [q GQ, (q + 1) GQ)
   if (!warp_wait(&sm.accfull[j % kNB], (j / kNB) & 1, wc, lane)) return false;
@@ -221,7 +166,6 @@ __device__ __forceinline__ bool epilogue(const ScoreParams &p, TcSmem<G, FUSED> 
   if (active) {
     // this thread's 2 GQ columns ((hi, lo) per head) of each partial
     // accumulator, summed in a fixed order
-    constexpr int NACC = TcCfg<G, FUSED>::NACC;
     uint32_t pa[NACC][2 * GQ];
     const uint32_t col = tmem + ((uint32_t)(32 * rg) << 16) +
                          (uint32_t)((j % kNB) * NACC * NCOL + q * 2 * GQ);
@@ -280,42 +224,15 @@ __device__ __forceinline__ bool epilogue(const ScoreParams &p, TcSmem<G, FUSED> 
   return true;
 }
 
-template <int G, int PAIR, bool FUSED>
-__device__ void compute(const ScoreParams &p, TcSmem<G, FUSED> &sm, uint32_t tmem, int tid,
-                        const WaitCtl &wc) {
-  constexpr int ST = TcCfg<G, FUSED>::STAGES, GQ = TcCfg<G, FUSED>::GQ;
+template <int G, int PAIR>
+__device__ void compute(const ScoreParams &p, TcSmem<G> &sm, uint32_t tmem, int tid, const WaitCtl wc) {
+  constexpr int ST = TcCfg<G>::STAGES, GQ = TcCfg<G>::GQ;
   const int warp = tid >> 5, lane = tid & 31;
   const int q = warp >> 2, rg = warp & 3, r = rg * 32 + lane;  // band group, quadrant, row
   const uint32_t mag_base = tmem + ((uint32_t)(32 * rg) << 16) + kTmemMag;
   double msum[GQ], msq[GQ];
 #pragma unroll
   for (int g = 0; g < GQ; ++g) msum[g] = msq[g] = 0.0;
-  int posted = 0;
-  // fused pass: hand a finished item (or the end) to the item warp
-  auto post = [&](const EpRec &e, int end) -> bool {
-    if constexpr (FUSED) {
-      TailArea &ta = sm.tp.t;
-      const int slot = posted % kItemRing;
-      if (posted >= kItemRing &&
-          !warp_wait(&ta.ifree[slot], ((posted / kItemRing) - 1) & 1, wc, lane))
-        return false;
-      if (warp == 0 && lane == 0) {
-        ItemPost &ip = ta.irec[slot];
-        ip.u = e.u;
-        ip.N = e.N;
-        ip.end = end;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ta.idone[slot]);
-      ++posted;
-    }
-    return true;
-  };
-  auto ep = [&](int j, const EpRec &e) -> bool {
-    if (!epilogue<G, FUSED>(p, sm, tmem, j, e, q, rg, lane, msum, msq, wc)) return false;
-    if (FUSED && (e.flags & kFlagLast)) return post(e, 0);
-    return true;
-  };
   // Tile i: magnitudes of tile i, then the epilogue of tile i - 2 (record
   // `older`, replaced by tile i's record); after the end marker also the
   // epilogue of tile i - 1 (record `other`).  0: go on, 1: done, -1: abort.
@@ -334,11 +251,10 @@ __device__ void compute(const ScoreParams &p, TcSmem<G, FUSED> &sm, uint32_t tme
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.aready[i % kNB]);
-    if (i >= 2 && !ep(i - 2, older)) return -1;
+    if (i >= 2 && !epilogue<G>(p, sm, tmem, i - 2, older, q, rg, lane, msum, msq, wc)) return -1;
     if (end) {
-      if (i >= 1 && !ep(i - 1, other)) return -1;
-      EpRec none{};
-      return post(none, 1) ? 1 : -1;
+      if (i >= 1 && !epilogue<G>(p, sm, tmem, i - 1, other, q, rg, lane, msum, msq, wc)) return -1;
+      return 1;
     }
     older = cur;
     return 0;
@@ -350,135 +266,17 @@ __device__ void compute(const ScoreParams &p, TcSmem<G, FUSED> &sm, uint32_t tme
   }
 }
 
-// ---------------------------------------------------------------------------
-// fused pass: item warp and tail warps
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ int ld_acquire(const int32_t *a) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void st_release(int32_t *a, int v) {
-  asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
-}
-
-template <int G>
-__device__ void item_warp(const ScoreParams &p, TailArea &ta, int lane, const WaitCtl &wc) {
-  const Geom &geo = p.geo;
-  for (int j = 0;; ++j) {
-    const int slot = j % kItemRing;
-    if (!warp_wait(&ta.idone[slot], (j / kItemRing) & 1, wc, lane)) return;
-    const ItemPost ip = ta.irec[slot];
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&ta.ifree[slot]);  // the record is copied
-    if (ip.end) return;
-    // Count the item in the unit's device-wide counter.  The compute warps'
-    // raw-score and moment writes precede their arrivals on idone (release,
-    // block scope), this warp acquired them by its wait, and the fence
-    // below (cumulative) orders them before the count at device scope; the
-    // block that takes the last count fences again and publishes the unit
-    // with a release store, which the tail warps that take it acquire.
-    if (lane == 0) {
-      const int ntiles = unit_tiles(ip.N, geo.window, geo.sinks);
-      __threadfence();
-      const uint32_t old = atomicAdd(p.unit_done + ip.u, 1u);
-      if (old + 1u == (uint32_t)ntiles) {
-        __threadfence();
-        const uint32_t at = atomicAdd(p.tq, 1u);
-        st_release(p.tailq + at, (int)ip.u);
-      }
-    }
-    __syncwarp();
-  }
-}
-
-// Tail warp 0: the next due unit (device-wide order), or -1 when every unit
-// the pass compresses has been taken, or on abort or expiry.  Lane 0 claims
-// the next queue position and waits (bounded) until a block publishes the
-// unit that completes there.
-__device__ int claim_tail(const ScoreParams &p, int lane, const WaitCtl &wc) {
-  int u = -1;
-  if (lane == 0) {
-    const uint32_t at = atomicAdd(p.tq + 1, 1u);
-    if (at < __ldcg(p.tq + 2)) {
-      const uint64_t t0 = global_timer();
-      for (;;) {
-        u = ld_acquire(p.tailq + at);
-        if (u >= 0) break;
-        if (*wc.abort_flag) break;
-        if (global_timer() - t0 > wc.limit_ns) {
-          flag_expiry(wc);
-          break;
-        }
-        __nanosleep(500);
-      }
-    }
-  }
-  return __shfl_sync(kFull, u, 0);
-}
-
-template <int G>
-__device__ void run_tail(const ScoreParams &p, TailArea &ta, long long u, int tt) {
-  const Geom &geo = p.geo;
-  const int s = (int)(u / ((int64_t)geo.nl * geo.hkv));
-  const int lrel = (int)((u / geo.hkv) % geo.nl);
-  const int N = unit_len(geo, s, lrel);
-  const int C = N - geo.window - geo.sinks;
-  const int B = geo.lbudget[lrel];
-  unit_norm<G, kTailBar, kTailThreads>(p.moments + u * geo.tiles_max * kRowGroups * G * 2,
-                                       unit_tiles(N, geo.window, geo.sinks), C, tt, ta.sc);
-  clear_words<kTailThreads>(ta.hist, kHistBins, tt);
-  csync<kTailBar, kTailThreads>();
-  const float *raw = p.raw + u * p.raw_stride;
-  uint32_t *keys = p.keys + u * p.keys_stride;
-  unit_keys<G, kTailThreads, kTailLoads, true>(raw, C, ta.sc.mean, ta.sc.inv, keys, ta.hist, tt);
-  csync<kTailBar, kTailThreads>();
-  int32_t *kept = p.kept + u * geo.budget;
-  select_global<kTailBar, kTailThreads>(keys, C, B - geo.window - geo.sinks, N, B, geo.window,
-                                        geo.sinks, kept, ta.hist, ta.list, ta.sc, tt);
-  for (int j = B + tt; j < geo.budget; j += kTailThreads) kept[j] = -1;
-  csync<kTailBar, kTailThreads>();
-  if (p.discard) {
-    // the unit's raw scores and keys are dead: drop their lines from L2
-    // without writing them back
-    const int64_t rl = ((int64_t)C * G * 4 + 127) / 128, kl = ((int64_t)C * 4 + 127) / 128;
-    for (int64_t i = tt; i < rl; i += kTailThreads) discard_line(raw + i * 32);
-    for (int64_t i = tt; i < kl; i += kTailThreads) discard_line(keys + i * 32);
-  }
-}
-
-template <int G>
-__device__ void tail_warps(const ScoreParams &p, TailArea &ta, int tt, const WaitCtl &wc) {
-  const int lane = tt & 31;
-  // tail warp 0 takes each due unit and hands it to the group through
-  // shared memory (the other tail warps wait at the group barrier only, so
-  // no tail warp is left waiting for one that stopped)
-  for (int j = 0;; ++j) {
-    if (tt < 32) {
-      const int u = claim_tail(p, lane, wc);
-      if (lane == 0) ta.act[j & 1] = u;
-    }
-    csync<kTailBar, kTailThreads>();
-    const int u = ta.act[j & 1];
-    if (u < 0) return;
-    run_tail<G>(p, ta, u, tt);
-  }
-}
-
-template <int G, int PAIR, int LAYOUT, bool FUSED>
-__global__ void __launch_bounds__(tc_threads<FUSED>(), 1)
-    score_tc_kernel(const __grid_constant__ ScoreParams p) {
-  using Cfg = TcCfg<G, FUSED>;
+template <int G, int PAIR, int LAYOUT>
+__global__ void __launch_bounds__(kTcThreads, 1) score_tc_kernel(const __grid_constant__ ScoreParams p) {
+  using Cfg = TcCfg<G>;
   extern __shared__ uint8_t smem_dyn[];
-  TcSmem<G, FUSED> &sm = *reinterpret_cast<TcSmem<G, FUSED> *>(
+  TcSmem<G> &sm = *reinterpret_cast<TcSmem<G> *>(
       (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
   const Geom &geo = p.geo;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  constexpr int NT = tc_threads<FUSED>();
 
-  for (int i = tid; i <= geo.n_seq; i += NT) sm.seq_items[i] = p.seq_items[i];
-  for (int i = tid; i < geo.n_seq; i += NT) sm.seq_len[i] = unit_len(geo, i, 0);
+  for (int i = tid; i <= geo.n_seq; i += kTcThreads) sm.seq_items[i] = p.seq_items[i];
+  for (int i = tid; i < geo.n_seq; i += kTcThreads) sm.seq_len[i] = unit_len(geo, i, 0);
   if (tid == 0) {
     for (int i = 0; i < Cfg::STAGES; ++i) {
       mbar_init(&sm.full[i], 1);
@@ -489,13 +287,6 @@ __global__ void __launch_bounds__(tc_threads<FUSED>(), 1)
       mbar_init(&sm.accfull[i], 1);
     }
     for (int i = 0; i < 2; ++i) mbar_init(&sm.bempty[i], 1);
-    if constexpr (FUSED) {
-      TailArea &ta = sm.tp.t;
-      for (int i = 0; i < kItemRing; ++i) {
-        mbar_init(&ta.idone[i], kComputeWarps);
-        mbar_init(&ta.ifree[i], 1);
-      }
-    }
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -508,15 +299,12 @@ __global__ void __launch_bounds__(tc_threads<FUSED>(), 1)
   const WaitCtl wc = wait_ctl(&sm.abort_flag, p.status, p.wait_ns);
 
   if (warp < kComputeWarps) {
-    compute<G, PAIR, FUSED>(p, sm, tmem, tid, wc);
+    compute<G, PAIR>(p, sm, tmem, tid, wc);
   } else if (warp == kProducerWarp) {
     producer<Cfg::STAGES, LAYOUT>(p, sm, n_items, lane, wc);
   } else if (warp == kMmaWarp) {
-    if (lane == 0) mma_issuer<G, FUSED>(p, sm, tmem, wc);
+    if (lane == 0) mma_issuer<G>(p, sm, tmem, wc);
     __syncwarp();
-  } else if constexpr (FUSED) {
-    if (warp == kItemWarp) item_warp<G>(p, sm.tp.t, lane, wc);
-    else tail_warps<G>(p, sm.tp.t, tid - 32 * kTailWarp0, wc);
   }
   tc_fence_before();
   __syncthreads();
@@ -526,67 +314,44 @@ __global__ void __launch_bounds__(tc_threads<FUSED>(), 1)
   }
 }
 
-template <int G, int PAIR, int LAYOUT, bool FUSED>
+template <int G, int PAIR, int LAYOUT>
 cudaError_t launch_t(const ScoreParams &p, cudaStream_t st) {
-  auto kern = score_tc_kernel<G, PAIR, LAYOUT, FUSED>;
-  const int smem = (int)sizeof(TcSmem<G, FUSED>) + 1024;
+  auto kern = score_tc_kernel<G, PAIR, LAYOUT>;
+  const int smem = (int)sizeof(TcSmem<G>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  if constexpr (FUSED) {
-    // the tail warps wait on other blocks: every block must be resident
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)sms);
-    cfg.blockDim = dim3((unsigned)tc_threads<FUSED>());
-    cfg.dynamicSmemBytes = (size_t)smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, p);
-  } else {
-    kern<<<sms, tc_threads<FUSED>(), smem, st>>>(p);
-    return cudaGetLastError();
-  }
+  kern<<<sms, kTcThreads, smem, st>>>(p);
+  return cudaGetLastError();
 }
 
-template <int G, bool FUSED>
+template <int G>
 cudaError_t launch_g(const ScoreParams &p, cudaStream_t st) {
   const bool paged = p.cache.layout == TRIA_LAYOUT_PAGED;
   if (p.geo.pairing == TRIA_PAIR_NEOX)
-    return paged ? launch_t<G, TRIA_PAIR_NEOX, TRIA_LAYOUT_PAGED, FUSED>(p, st)
-                 : launch_t<G, TRIA_PAIR_NEOX, TRIA_LAYOUT_CONTIGUOUS, FUSED>(p, st);
-  return paged ? launch_t<G, TRIA_PAIR_INTERLEAVED, TRIA_LAYOUT_PAGED, FUSED>(p, st)
-               : launch_t<G, TRIA_PAIR_INTERLEAVED, TRIA_LAYOUT_CONTIGUOUS, FUSED>(p, st);
+    return paged ? launch_t<G, TRIA_PAIR_NEOX, TRIA_LAYOUT_PAGED>(p, st)
+                 : launch_t<G, TRIA_PAIR_NEOX, TRIA_LAYOUT_CONTIGUOUS>(p, st);
+  return paged ? launch_t<G, TRIA_PAIR_INTERLEAVED, TRIA_LAYOUT_PAGED>(p, st)
+               : launch_t<G, TRIA_PAIR_INTERLEAVED, TRIA_LAYOUT_CONTIGUOUS>(p, st);
 }
 
-template <bool FUSED>
-cudaError_t launch_f(const ScoreParams &p, cudaStream_t st) {
-  switch (p.geo.g) {
-    case 1: return launch_g<1, FUSED>(p, st);
-    case 2: return launch_g<2, FUSED>(p, st);
-    case 4: return launch_g<4, FUSED>(p, st);
-    case 8: return launch_g<8, FUSED>(p, st);
-    case 16: return launch_g<16, FUSED>(p, st);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
-static_assert(sizeof(TcSmem<8, false>) + 1024 <= 232448, "shared memory of the G=8 kernel");
-static_assert(sizeof(TcSmem<16, false>) + 1024 <= 232448, "shared memory of the G=16 kernel");
-static_assert(sizeof(TcSmem<8, true>) + 1024 <= 232448, "shared memory of the G=8 fused kernel");
-static_assert(sizeof(TcSmem<16, true>) + 1024 <= 232448, "shared memory of the G=16 fused kernel");
-static_assert(sizeof(GroupScalars<kTailWarps>) % 8 == 0, "tail scalars");
+static_assert(sizeof(TcSmem<8>) + 1024 <= 232448, "shared memory of the G=8 kernel");
+static_assert(sizeof(TcSmem<16>) + 1024 <= 232448, "shared memory of the G=16 kernel");
 
 }  // namespace
 
-cudaError_t launch_score(const ScoreParams &p, bool fused, cudaStream_t st) {
+cudaError_t launch_score(const ScoreParams &p, cudaStream_t st) {
   if (p.geo.mode == TRIA_OFFSET_MAX) return launch_score_max(p, st);
-  return fused ? launch_f<true>(p, st) : launch_f<false>(p, st);
+  switch (p.geo.g) {
+    case 1: return launch_g<1>(p, st);
+    case 2: return launch_g<2>(p, st);
+    case 4: return launch_g<4>(p, st);
+    case 8: return launch_g<8>(p, st);
+    case 16: return launch_g<16>(p, st);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace tria

@@ -130,7 +130,7 @@ __device__ __forceinline__ void flag_expiry(const WaitCtl &w) {
 }
 
 // Bounded wait (one thread) for the phase of `parity`; false on expiry or abort.
-static __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const WaitCtl &w) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const WaitCtl &w) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try(a, parity)) return true;
   const uint64_t t0 = global_timer();
@@ -146,7 +146,7 @@ static __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, co
 
 // Wait (one thread) on the abort path for work this block started (copies,
 // MMA commits): not cut short by the abort flag; bounded by kDrainNs.
-static __device__ __noinline__ bool mbar_drain(uint64_t *bar, uint32_t parity, int32_t *status) {
+__device__ __forceinline__ bool mbar_drain(uint64_t *bar, uint32_t parity, int32_t *status) {
   const uint32_t a = smem_u32(bar);
   const uint64_t t0 = global_timer();
   for (;;) {
@@ -423,7 +423,7 @@ __device__ __forceinline__ void mags_regs(const uint8_t *kt, int r, int q, uint3
 // bempty[2], rec[ST], seq_items, seq_len, bbuf(i).
 // ---------------------------------------------------------------------------
 template <int ST, int LAYOUT, class Smem>
-__device__ void producer(const ScoreParams &p, Smem &sm, int n_items, int lane, const WaitCtl &wc) {
+__device__ void producer(const ScoreParams &p, Smem &sm, int n_items, int lane, const WaitCtl wc) {
   const uint32_t kBBytes = (uint32_t)p.geo.b_bytes;  // one unit's coefficient image
   const Geom &geo = p.geo;
   const uint64_t pol = evict_first_policy();
@@ -447,19 +447,13 @@ __device__ void producer(const ScoreParams &p, Smem &sm, int n_items, int lane, 
         if (sm.seq_items[mid] <= it) lo = mid; else hi = mid - 1;
       }
       s = lo;
-      // Items of a (sequence, layer) row take the row's KV heads in turn
-      // (item k of the row: tile k / hkv of head k % hkv), so the last items
-      // of the row's units are claimed one after another by different
-      // blocks: the blocks that complete units, and run their tails, rotate
-      // over the whole grid instead of repeating with the item count.
       if (!geo.per_layer) {
         ntiles = (sm.seq_items[s + 1] - sm.seq_items[s]) / units_per_seq;
         const int rem = it - sm.seq_items[s];
-        const int row_n = geo.hkv * ntiles;
-        lrel = rem / row_n;
-        const int idx = rem - lrel * row_n;
-        tile = idx / geo.hkv;
-        h = idx - tile * geo.hkv;
+        const int ul = rem / ntiles;
+        tile = rem % ntiles;
+        lrel = ul / geo.hkv;
+        h = ul % geo.hkv;
         N = sm.seq_len[s];
       } else {
         // a length per (sequence, layer): the layer is the last row of the
@@ -475,8 +469,8 @@ __device__ void producer(const ScoreParams &p, Smem &sm, int n_items, int lane, 
         N = unit_len(geo, s, lrel);
         ntiles = unit_tiles(N, W, S);
         const int rem = it - __ldcg(ri + lrel);
-        tile = rem / geo.hkv;
-        h = rem - tile * geo.hkv;
+        h = rem / ntiles;
+        tile = rem % ntiles;
       }
       u = (long long)s * units_per_seq + lrel * geo.hkv + h;
       tbase = (S / kTileKeys + tile) * kTileKeys;
