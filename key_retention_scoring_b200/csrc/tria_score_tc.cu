@@ -27,9 +27,7 @@
 //   warp 9      one lane issues tcgen05.mma (M=128, N=16|32, K=16): 8 steps
 //               with A = the K tile in shared memory (then the K stage is
 //               released), 8 steps with A = the magnitude tile in tensor
-//               memory, and tcgen05.commit.  Consecutive steps accumulate
-//               into NACC different partial accumulators (summed by the
-//               epilogue), so they do not wait on each other's results.
+//               memory, and tcgen05.commit.
 // Normalize-then-max and the selection run in the next kernel (the unit tail
 // in tria_kernels.cu).  Every wait is bounded (ScoreParams::wait_ns); on
 // expiry the kernel flags status bit 1, lets its own loads and MMAs land,
@@ -63,12 +61,12 @@ struct TcCfg {
   static constexpr int STAGES = (G <= 8) ? 6 : 5;
   static constexpr int GQ = (G >= kBandGroups) ? G / kBandGroups : 1;  // heads per band group
   static constexpr int BBLK = NCOL * 128;                  // bytes per 64-wide K block of B
-  // Consecutive K-steps of a tile accumulate into NACC partial accumulators
-  // (summed by the epilogue): an N = 16 MMA is a few tensor-pipe cycles, far
-  // below the latency of its result, so one accumulator would chain the
-  // tile's 16 MMAs on that latency; two chains of eight measured faster than
-  // four of four (fewer epilogue additions)
-  static constexpr int NACC = 2;
+  // K-steps of a tile may accumulate into NACC partial accumulators (summed
+  // by the epilogue) so that consecutive MMAs do not wait on each other's
+  // results; with two tiles of slack between a tile's MMAs and its epilogue
+  // the single chain of 16 measured fastest (931 us per Qwen3-32B 32K pass,
+  // against 936 with two chains and 960 with four)
+  static constexpr int NACC = 1;
   static_assert(kNB * NACC * NCOL <= 256, "accumulator columns");
 };
 
