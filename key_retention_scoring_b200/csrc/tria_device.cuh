@@ -1,6 +1,6 @@
 // Device helpers shared by the kernels: bf16 unpacking, cache hints, the
 // order-preserving score key, block scans, the radix top-K selection of one
-// unit and the per-unit tail (normalize-then-max, selection).
+// unit over agg in global memory and normalize-then-max.
 //
 // Everything that synchronises takes a barrier id BAR: 0 = __syncthreads of
 // a kSelThreads-thread block, n > 0 = named barrier n over the first
@@ -417,7 +417,19 @@ __device__ void unit_norm(const double *mom_unit, int ntiles, int C, int tid, Sc
   const double2 *m2 = reinterpret_cast<const double2 *>(mom_unit);
   for (int g = w; g < G; g += NW) {
     double s1 = 0.0, s2 = 0.0;
-    for (int i = lane; i < n; i += 32) {
+    int i = lane;
+    // eight loads in flight, added in the same order as one at a time
+    for (; i + 7 * 32 < n; i += 8 * 32) {
+      double2 v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = __ldcg(m2 + (int64_t)(i + 32 * e) * G + g);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        s1 += v[e].x;
+        s2 += v[e].y;
+      }
+    }
+    for (; i < n; i += 32) {
       const double2 v = __ldcg(m2 + (int64_t)i * G + g);
       s1 += v.x;
       s2 += v.y;
@@ -490,124 +502,6 @@ __device__ void agg_range(const float *__restrict__ raw, float *agg, int c0, int
   }
 }
 
-// ---------------------------------------------------------------------------
-// Per-unit tail with the candidates' agg keys in shared memory (one block of
-// NT threads per unit).
-// unit_keys: keys[c] = order_key(agg[c]), agg[c] = max_g (S_g[c] - mean_g)
-// inv_g (NaN when any term is), from one coalesced pass over the unit's raw
-// scores [C][G]; adds the top 12 key bits of every candidate to hist.
-// select_keys: radix top-K over the keys (digits of 12, 12 and 8 bits), then
-// the ascending kept list: sinks, the K candidates above the threshold key T
-// plus the lowest-slot keys equal to T, the window.  After the first digit
-// (histogram of unit_keys), one pass over the keys counts, per warp range,
-// the keys above the chosen bin, histograms the bin's keys on the second
-// digit and gathers them into a list; the third digit and the per-warp
-// counts of keys above / equal to T inside the bin come from the list.  A bin
-// larger than the list falls back to passes over all keys.  The emission is
-// one more pass.
-// ---------------------------------------------------------------------------
-struct alignas(16) UnitScalars {  // 16-byte size: the key area after it is read as uint4
-  int warp_tmp[32];
-  uint32_t prefix;
-  int remaining;
-  int digit;
-  int above;
-  int bin_count;
-  int list_n;
-  int warp_gt[32];
-  int warp_eq[32];
-  float mean[TRIA_MAX_GROUP];
-  float inv[TRIA_MAX_GROUP];
-};
-
-template <int G, int NT>
-__device__ void unit_keys(const float *raw, int C, const float *s_mean, const float *s_inv,
-                          uint32_t *keys, uint32_t *hist, int tid) {
-  const int lane = tid & 31;
-  constexpr int U = 8;  // float4 loads in flight per thread
-  const float4 *src = reinterpret_cast<const float4 *>(raw);
-  if constexpr (G >= 4) {
-    // LPC lanes per candidate, each with 4 of its G heads
-    constexpr int LPC = G / 4;
-    const int h0 = (tid % LPC) * 4;
-    float m[4], iv[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      m[k] = s_mean[h0 + k];
-      iv[k] = s_inv[h0 + k];
-    }
-    const int n4 = C * LPC;
-    for (int j0 = 0; j0 < n4; j0 += NT * U) {
-      float4 x[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int j = j0 + u * NT + tid;
-        x[u] = (j < n4) ? __ldcs(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int j = j0 + u * NT + tid;
-        const float z0 = __fmul_rn(__fsub_rn(x[u].x, m[0]), iv[0]);
-        const float z1 = __fmul_rn(__fsub_rn(x[u].y, m[1]), iv[1]);
-        const float z2 = __fmul_rn(__fsub_rn(x[u].z, m[2]), iv[2]);
-        const float z3 = __fmul_rn(__fsub_rn(x[u].w, m[3]), iv[3]);
-        int nan = (z0 != z0) | (z1 != z1) | (z2 != z2) | (z3 != z3);
-        float a = fmaxf(fmaxf(z0, z1), fmaxf(z2, z3));
-#pragma unroll
-        for (int o = 1; o < LPC; o <<= 1) {
-          a = fmaxf(a, __shfl_xor_sync(kFull, a, o));
-          nan |= __shfl_xor_sync(kFull, nan, o);
-        }
-        const uint32_t k = nan ? 0u : order_key(a);
-        const bool lead = (j < n4) && (tid % LPC) == 0;
-        if (lead) keys[j / LPC] = k;
-        hist_add(hist, k >> 20, lead, lane);
-      }
-    }
-  } else {
-    // a float4 holds CPF = 4 / G candidates
-    constexpr int CPF = 4 / G;
-    float m[G], iv[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      m[g] = s_mean[g];
-      iv[g] = s_inv[g];
-    }
-    const int n4 = (C + CPF - 1) / CPF;
-    for (int j0 = 0; j0 < n4; j0 += NT * U) {
-      float4 x[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int j = j0 + u * NT + tid;
-        x[u] = (j < n4) ? __ldcs(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int j = j0 + u * NT + tid;
-        const float v[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
-#pragma unroll
-        for (int e = 0; e < CPF; ++e) {
-          const int c = j * CPF + e;
-          float a = 0.0f;
-          int nan = 0;
-#pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const float z = __fmul_rn(__fsub_rn(v[e * G + g], m[g]), iv[g]);
-            a = (g == 0) ? z : fmaxf(a, z);
-            nan |= (z != z);
-          }
-          const uint32_t k = nan ? 0u : order_key(a);
-          const bool in = (j < n4) && c < C;
-          if (in) keys[c] = k;
-          hist_add(hist, k >> 20, in, lane);
-        }
-      }
-    }
-  }
-}
-
-static_assert(sizeof(UnitScalars) % 16 == 0, "shared-memory areas after UnitScalars stay 16-byte aligned");
-
 // Warp-wide inclusive scan of v (lane order).
 __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
 #pragma unroll
@@ -617,173 +511,6 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
   }
   return v;
 }
-
-// keys: shared memory, readable (as uint4) up to a multiple of 4 NT entries
-// past C; entries >= C are ignored.  Warp w owns the candidates
-// [w R, (w + 1) R), R = steps * 128; a lane takes 4 consecutive keys per step.
-template <int NT>
-__device__ void select_keys(const uint32_t *keys, int C, int K, int N, int B, int W, int S,
-                            int32_t *kept, uint32_t *hist, uint2 *list, UnitScalars &sc, int tid) {
-  const int lane = tid & 31, warp = tid >> 5;
-  for (int j = tid; j < S; j += NT) kept[j] = j;
-  for (int j = tid; j < W; j += NT) kept[B - W + j] = N - W + j;
-  if (K <= 0) return;
-  if (tid == 0) {
-    sc.prefix = 0u;
-    sc.remaining = K;
-    sc.list_n = 0;
-  }
-  __syncthreads();
-  pick_bin<0, NT>(hist, kHistBins, sc, 20, tid);
-  const int steps = (C + NT * 4 - 1) / (NT * 4);
-  const int R = steps * 128;
-  const int cb = warp * R;
-  clear_words<NT>(hist, kHistBins, tid);
-  __syncthreads();
-  const uint32_t d1 = sc.prefix >> 20;
-  {
-    // keys above the chosen first-digit bin, per warp; the bin's keys go to
-    // the second-digit histogram and the list
-    int above = 0;
-    for (int e = 0; e < steps; ++e) {
-      const int c0 = cb + e * 128 + lane * 4;
-      const uint4 k4 = *reinterpret_cast<const uint4 *>(keys + c0);
-      const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
-      uint32_t inmask = 0u;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const bool valid = c0 + i < C;
-        above += (valid && (kk[i] >> 20) > d1) ? 1 : 0;
-        inmask |= (valid && (kk[i] >> 20) == d1) ? (1u << i) : 0u;
-      }
-      if (__ballot_sync(kFull, inmask != 0u)) {
-        const int cnt = __popc(inmask);
-        const int incl = warp_incl_scan(cnt, lane);
-        int base = 0;
-        if (lane == 31) base = atomicAdd(&sc.list_n, incl);
-        base = __shfl_sync(kFull, base, 31);
-        int idx = base + incl - cnt;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          if ((inmask >> i) & 1u) {
-            atomicAdd(hist + ((kk[i] >> 8) & 0xfffu), 1u);
-            if (idx < kListCap) list[idx] = make_uint2(kk[i], (uint32_t)(c0 + i));
-            ++idx;
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) above += __shfl_xor_sync(kFull, above, o);
-    if (lane == 0) {
-      sc.warp_gt[warp] = above;
-      sc.warp_eq[warp] = 0;
-    }
-  }
-  __syncthreads();
-  pick_bin<0, NT>(hist, kHistBins, sc, 8, tid);
-  const int ln = sc.list_n;
-  const bool use_list = ln <= kListCap;
-  clear_words<NT>(hist, kHistBins, tid);
-  __syncthreads();
-  {
-    const uint32_t d12 = sc.prefix >> 8;
-    if (use_list) {
-      for (int i = tid; i < ln; i += NT) {
-        const uint32_t k = list[i].x;
-        if ((k >> 8) == d12) atomicAdd(hist + (k & 0xffu), 1u);
-      }
-    } else {
-      for (int c = tid; c < C; c += NT) {
-        const uint32_t k = keys[c];
-        if ((k >> 8) == d12) atomicAdd(hist + (k & 0xffu), 1u);
-      }
-    }
-  }
-  __syncthreads();
-  pick_bin<0, NT>(hist, kHistBins, sc, 0, tid);
-  const uint32_t T = sc.prefix;
-  const int need = sc.remaining;  // keys equal to T to take, lowest slots first (>= 1)
-  // per-warp counts of the keys of the first-digit bin above / equal to T
-  if (use_list) {
-    for (int i = tid; i < ln; i += NT) {
-      const uint2 e = list[i];
-      const int w = (int)e.y / R;
-      if (e.x > T) atomicAdd(&sc.warp_gt[w], 1);
-      else if (e.x == T) atomicAdd(&sc.warp_eq[w], 1);
-    }
-  } else {
-    int gt = 0, eq = 0;
-    for (int e = 0; e < steps; ++e) {
-      const int c0 = cb + e * 128 + lane * 4;
-      const uint4 k4 = *reinterpret_cast<const uint4 *>(keys + c0);
-      const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const bool valid = c0 + i < C;
-        gt += (valid && (kk[i] >> 20) == d1 && kk[i] > T) ? 1 : 0;
-        eq += (valid && kk[i] == T) ? 1 : 0;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      gt += __shfl_xor_sync(kFull, gt, o);
-      eq += __shfl_xor_sync(kFull, eq, o);
-    }
-    if (lane == 0) {
-      atomicAdd(&sc.warp_gt[warp], gt);
-      atomicAdd(&sc.warp_eq[warp], eq);
-    }
-  }
-  __syncthreads();
-  int gt_before = 0, eq_before = 0;
-  for (int i = 0; i < warp; ++i) {
-    gt_before += sc.warp_gt[i];
-    eq_before += sc.warp_eq[i];
-  }
-  // emission in slot order
-  int run_keep = gt_before + min(eq_before, need);
-  int run_eq = eq_before;
-  for (int e = 0; e < steps; ++e) {
-    const int c0 = cb + e * 128 + lane * 4;
-    const uint4 k4 = *reinterpret_cast<const uint4 *>(keys + c0);
-    const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
-    uint32_t gtm = 0u, eqm = 0u;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const bool valid = c0 + i < C;
-      gtm |= (valid && kk[i] > T) ? (1u << i) : 0u;
-      eqm |= (valid && kk[i] == T) ? (1u << i) : 0u;
-    }
-    uint32_t keepm = gtm;
-    if (__ballot_sync(kFull, eqm != 0u)) {
-      // ties in slot order: lanes in order, then a lane's keys in order
-      const int ne = __popc(eqm);
-      const int incl = warp_incl_scan(ne, lane);
-      int rank = run_eq + incl - ne;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if ((eqm >> i) & 1u) {
-          if (rank < need) keepm |= 1u << i;
-          ++rank;
-        }
-      }
-      run_eq += __shfl_sync(kFull, incl, 31);
-    }
-    const int nk = __popc(keepm);
-    const int incl = warp_incl_scan(nk, lane);
-    int pos = run_keep + incl - nk;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if ((keepm >> i) & 1u) {
-        if (pos < K) kept[S + pos] = S + c0 + i;
-        ++pos;
-      }
-    }
-    run_keep += __shfl_sync(kFull, incl, 31);
-  }
-}
-
 
 }  // namespace dev
 }  // namespace tria

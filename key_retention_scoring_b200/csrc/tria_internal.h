@@ -90,7 +90,7 @@ struct WsLayout {
 
 constexpr int kAggHistBins = 4096;
 constexpr int kAggChunk = 4096;   // candidates per block of the normalization kernel
-constexpr int kUnitTailMaxC = 45056;       // candidates per unit of the one-block-per-unit tail
+constexpr int kMaxTailCluster = 8;         // blocks per unit of the cluster tail (portable cluster size)
 constexpr size_t kMaxDynSmem = 232448;     // opt-in shared memory per block (227 KB)
 
 WsLayout ws_layout(const Geom &g);
@@ -128,6 +128,8 @@ struct TailParams {
   uint32_t *unit_done;  // [unit]
   int discard_raw;      // raw is workspace scratch: drop its L2 lines after use
   int discard_agg;      // agg is workspace scratch
+  int cluster;          // unit tail: blocks per unit (a thread-block cluster)
+  int slice;            // unit tail: candidates per block (a multiple of 128)
 };
 
 struct CoefParams {
@@ -184,8 +186,9 @@ cudaError_t launch_score(const ScoreParams &p, cudaStream_t st);
 cudaError_t launch_score_max(const ScoreParams &p, cudaStream_t st);
 cudaError_t launch_tail(const TailParams &p, cudaStream_t st);
 cudaError_t launch_select(const SelectParams &p, cudaStream_t st);
-// Normalize-then-max + selection with one block per unit (kept != null);
-// only when unit_tail_fits(geo).
+// Normalize-then-max + selection with one thread-block cluster per unit and
+// the agg keys in shared memory (kept != null; tria_tail.cu); only when
+// unit_tail_fits(geo).
 bool unit_tail_fits(const Geom &g);
 cudaError_t launch_unit_tail(const TailParams &p, cudaStream_t st);
 cudaError_t launch_compact(const CompactParams &p, cudaStream_t st);

@@ -8,6 +8,7 @@
 //   tail_kernel     blocks over (unit, candidate chunk): normalize-then-max,
 //                   histogram of the agg keys, selection by the last block.
 //   select_kernel   one CTA per unit: radix top-K of agg + ascending kept list.
+//   (the cluster unit tail of the pass is in tria_tail.cu)
 //   (the compaction kernel is in tria_compact.cu)
 //
 // Sources: academ.us article 2607.13051 (Eqs. 2, 3, 4, 6, 7 and sec. 4),
@@ -299,58 +300,6 @@ __global__ void __launch_bounds__(kThreads) tail_kernel(const __grid_constant__ 
 }
 
 // ---------------------------------------------------------------------------
-// unit_tail_kernel: normalize-then-max and selection with one block of
-// kUnitThreads per unit (units strided over the grid), for passes whose
-// candidates' keys fit in shared memory.  The unit's raw scores are read
-// once; agg lives only as order keys in shared memory.
-// ---------------------------------------------------------------------------
-constexpr int kUnitThreads = 1024;
-
-// the key area is read 4 NT keys at a time by the selection: padded to that
-size_t unit_tail_smem_bytes(int c_max) {
-  const size_t pad = (size_t)kUnitThreads * 4;
-  return sizeof(UnitScalars) + (size_t)kHistBins * 4 + (size_t)kListCap * 8 +
-         (((size_t)c_max + pad - 1) / pad) * pad * 4;
-}
-
-template <int G>
-__global__ void __launch_bounds__(kUnitThreads, 1) unit_tail_kernel(const __grid_constant__ TailParams p) {
-  extern __shared__ __align__(16) uint8_t smem_ut[];
-  UnitScalars &sc = *reinterpret_cast<UnitScalars *>(smem_ut);
-  uint32_t *hist = reinterpret_cast<uint32_t *>(smem_ut + sizeof(UnitScalars));
-  uint2 *list = reinterpret_cast<uint2 *>(hist + kHistBins);
-  uint32_t *keys = reinterpret_cast<uint32_t *>(list + kListCap);
-  const Geom &geo = p.geo;
-  const int t = threadIdx.x;
-  for (int64_t u = blockIdx.x; u < geo.n_units; u += gridDim.x) {
-    const int s = (int)(u / ((int64_t)geo.nl * geo.hkv));
-    const int lrel = (int)((u / geo.hkv) % geo.nl);
-    const int N = unit_len(geo, s, lrel);
-    // invalid lengths and units left as they are: the coefficient kernel
-    // wrote their kept rows and flagged the former
-    if (!compresses(geo, N, lrel)) continue;
-    const int B = geo.lbudget[lrel];
-    const int C = N - geo.window - geo.sinks;
-    unit_norm<G, 0, kUnitThreads>(p.moments + u * geo.tiles_max * kRowGroups * G * 2,
-                                  unit_tiles(N, geo.window, geo.sinks), C, t, sc);
-    clear_words<kUnitThreads>(hist, kHistBins, t);
-    __syncthreads();
-    const float *raw = p.raw + u * p.raw_stride;
-    unit_keys<G, kUnitThreads>(raw, C, sc.mean, sc.inv, keys, hist, t);
-    __syncthreads();
-    if (p.discard_raw) {
-      const int64_t lines = ((int64_t)C * G * 4 + 127) / 128;
-      for (int64_t i = t; i < lines; i += kUnitThreads) discard_line(raw + i * 32);
-    }
-    int32_t *kept = p.kept + u * geo.budget;
-    select_keys<kUnitThreads>(keys, C, B - geo.window - geo.sinks, N, B, geo.window, geo.sinks,
-                              kept, hist, list, sc, t);
-    for (int j = B + t; j < geo.budget; j += kUnitThreads) kept[j] = -1;
-    __syncthreads();
-  }
-}
-
-// ---------------------------------------------------------------------------
 // select_kernel: one CTA per unit
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads) select_kernel(const __grid_constant__ SelectParams p) {
@@ -394,38 +343,6 @@ cudaError_t launch_tail(const TailParams &p, cudaStream_t st) {
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
-}
-
-template <int G>
-cudaError_t launch_unit_tail_g(const TailParams &p, size_t smem, cudaStream_t st) {
-  auto kern = unit_tail_kernel<G>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  int dev = 0, sms = 0, per_sm = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kUnitThreads, smem)) != cudaSuccess)
-    return e;
-  int64_t grid = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
-  if (grid > p.geo.n_units) grid = p.geo.n_units;
-  kern<<<(unsigned)grid, kUnitThreads, smem, st>>>(p);
-  return cudaGetLastError();
-}
-
-bool unit_tail_fits(const Geom &g) {
-  return g.c_max <= kUnitTailMaxC && unit_tail_smem_bytes(g.c_max) <= kMaxDynSmem;
-}
-
-cudaError_t launch_unit_tail(const TailParams &p, cudaStream_t st) {
-  const size_t smem = unit_tail_smem_bytes(p.geo.c_max);
-  switch (p.geo.g) {
-    case 1: return launch_unit_tail_g<1>(p, smem, st);
-    case 2: return launch_unit_tail_g<2>(p, smem, st);
-    case 4: return launch_unit_tail_g<4>(p, smem, st);
-    case 8: return launch_unit_tail_g<8>(p, smem, st);
-    case 16: return launch_unit_tail_g<16>(p, smem, st);
-    default: return cudaErrorInvalidValue;
-  }
 }
 
 cudaError_t launch_select(const SelectParams &p, cudaStream_t st) {

@@ -211,6 +211,54 @@ def test_offset_sets_and_theta():
 
 
 # ---------------------------------------------------------------------------
+# long units: the pass's unit tail splits a unit's candidates over a cluster of
+# 2, 4 or 8 blocks (more than 45056 candidates per unit)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("seq_len", [60000, 100000, 200000], ids=["2blocks", "4blocks", "8blocks"])
+def test_cluster_tail_long_units(seq_len):
+    cfg = synth.CONFIGS[4].scaled(n_layers=1, n_q_heads=16, n_kv_heads=2, seq_len=seq_len)
+    full_check(cfg)
+
+
+def test_cluster_tail_ragged_lengths_paged():
+    # lengths per sequence from 20000 to 120000: the cluster is sized for the
+    # longest, so the shorter units leave their trailing blocks without candidates
+    cfg = synth.CONFIGS[3].scaled(n_layers=1, n_q_heads=8, n_kv_heads=2, n_seq=3, budget=9000,
+                                  len_range=(20000, 120000))
+    full_check(cfg)
+
+
+def test_cluster_tail_ties_across_blocks():
+    # unit h = 0: every candidate row equal, so every agg is equal and the K
+    # lowest slots are kept; unit h = 1: rows repeat with period 3, so the
+    # threshold falls on a value held by about C / 3 keys in every block of the
+    # cluster (four blocks), and the kept ties run into the second block
+    cfg = synth.CONFIGS[4].scaled(n_layers=1, n_q_heads=16, n_kv_heads=2, seq_len=100000)
+    w = synth.Workload(cfg)
+    st = load_stats(w)
+    try:
+        N, W, S, B = cfg.seq_len, cfg.window, cfg.sinks, cfg.budget
+        k = w.k[0]
+        k[0, 0, S:N - W] = k[0, 0, S:S + 1]
+        base = k[0, 1, S:S + 3].clone()
+        C = N - W - S
+        k[0, 1, S:N - W] = base.repeat((C + 2) // 3, 1)[:C]
+        agg, _, kept_sep = score_layers(w, st, 0, 1, want_scores=False)
+        for h in range(2):
+            PH.check_kept_same_precision(kept_sep[0, 0, h], agg[0, 0, h, :C], N, cfg, f"h{h}")
+        K = B - W - S
+        want0 = np.concatenate([np.arange(S), np.arange(S, S + K), np.arange(N - W, N)])
+        assert np.array_equal(kept_sep[0, 0, 0], want0)
+        kept_all, _, _ = compress(w, st)
+        for h in range(2):
+            assert np.array_equal(kept_all[0, 0, h], kept_sep[0, 0, h]), f"h{h}"
+    finally:
+        st.free()
+        del w
+        torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------
 # multi-pass: positions are no longer slot indices after compaction
 # ---------------------------------------------------------------------------
 def test_multi_pass_with_appends():
