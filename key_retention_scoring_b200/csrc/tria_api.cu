@@ -132,11 +132,12 @@ tria_status make_geom(const tria_stats *stats, const tria_cache_view *cache,
   g.mode = params->offset_reduce;
   if (g.mode != TRIA_OFFSET_MEAN && g.mode != TRIA_OFFSET_MAX) return TRIA_ERR_INVALID_ARG;
   g.n_off = d.offset_log2_max + 1;
-  g.ncol_t = ((2 * g.n_off * g.g + 15) / 16) * 16;
+  g.ncol_t = ((g.n_off * g.g + 15) / 16) * 16;
   g.ncol_n = g.ncol;
   if (g.mode == TRIA_OFFSET_MAX) {
     if (g.n_off > 17 || 2 * g.n_off * g.g > kMaxOffCols) return TRIA_ERR_UNSUPPORTED;
-    g.b_bytes = (g.ncol_t + g.ncol_n) * 256;  // two 64-wide K blocks of 128-byte rows each
+    // trig hi and lo parts (two 64-wide K blocks of 128-byte rows each), norm
+    g.b_bytes = (2 * g.ncol_t + g.ncol_n) * 256;
   } else {
     g.b_bytes = g.ncol * kCoefK * 2;
   }

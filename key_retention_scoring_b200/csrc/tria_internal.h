@@ -51,7 +51,7 @@ struct Geom {
   int64_t n_units;  // n_seq * nl * hkv
   int mode;      // TRIA_OFFSET_MEAN / TRIA_OFFSET_MAX
   int n_off;     // |D| = offset_log2_max + 1
-  int ncol_t;    // max mode: trig operand rows, 2 |D| G rounded up to 16
+  int ncol_t;    // max mode: trig operand rows, |D| G rounded up to 16
   int ncol_n;    // max mode: norm operand rows, max(16, 2G)
   int b_bytes;   // bytes of one unit's coefficient image
 };

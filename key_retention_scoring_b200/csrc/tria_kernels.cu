@@ -139,10 +139,12 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
     }
     __syncthreads();
     unsigned char *dst = reinterpret_cast<unsigned char *>(p.btile) + u * (int64_t)g.b_bytes;
-    // trig rows n = 2 (gg nd + j) + part over the 128 key dims (two 64-wide blocks)
-    for (int i = t; i < g.ncol_t * 16; i += kThreads) {
-      const int n = i >> 4, ch = i & 15, kb = ch >> 3, c8 = ch & 7;
-      const int col = n >> 1, part = n & 1, gg = col / nd, j = col % nd;
+    // trig rows n = gg nd + j over the 128 key dims: the hi parts in two
+    // 64-wide blocks, then the lo parts in two more
+    for (int i = t; i < 2 * g.ncol_t * 16; i += kThreads) {
+      const int part = i / (g.ncol_t * 16), i2 = i % (g.ncol_t * 16);
+      const int n = i2 >> 4, ch = i2 & 15, kb = ch >> 3, c8 = ch & 7;
+      const int gg = n / nd, j = n % nd;
       uint32_t w[4];
       for (int e = 0; e < 8; e += 2) {
         uint16_t b2[2];
@@ -162,12 +164,12 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
         }
         w[e >> 1] = (uint32_t)b2[0] | ((uint32_t)b2[1] << 16);
       }
-      *reinterpret_cast<uint4 *>(dst + kb * (g.ncol_t * 128) + n * 128 + ((c8 ^ (n & 7)) << 4)) =
-          make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4 *>(dst + (2 * part + kb) * (g.ncol_t * 128) + n * 128 +
+                                 ((c8 ^ (n & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     // norm rows n = 2 gg + part over the magnitude dims: block 0 multiplies
     // |k_f| hi (w_f split hi/lo over the rows), block 1 |k_f| lo (w_f hi, 0)
-    unsigned char *dn = dst + 2 * g.ncol_t * 128;
+    unsigned char *dn = dst + 4 * g.ncol_t * 128;
     for (int i = t; i < g.ncol_n * 16; i += kThreads) {
       const int n = i >> 4, ch = i & 15, kb = ch >> 3, c8 = ch & 7;
       const int gg = n >> 1, part = n & 1;

@@ -5,20 +5,23 @@
 //
 // S_g(k) = max_j S_trig,g(k, Delta + delta_j) + S_norm,g(k).  The maximum is
 // not linear, so nothing folds: per (head g, offset delta_j) the coefficient
-// vector c_gj = E[q_g] mask e^{i omega (p_q + delta_j)} is its own bf16 hi/lo
-// column pair (2 |D| G columns, written by the coefficient kernel) and the
-// norm weights a separate 2G-column operand.  Per tile two contractions,
-// [k] (128 x 128) . Btrig (128 x 2 |D| G) into a trig accumulator (one or two
-// MMAs per K-step, N <= 256 each) and [m_hi | m_lo] . Bnorm (128 x 2G) into
-// a norm accumulator, then a max over the offset pairs in the epilogue.
-// Tensor memory holds one buffer of each (trig 0..271, norm 288.., magnitudes
-// 320..383), so a tile's epilogue runs before the next tile's MMAs; the
-// compute warps hide it behind the next tile's magnitude math (computed into
-// registers first, stored to tensor memory after the epilogue).
+// vector c_gj = E[q_g] mask e^{i omega (p_q + delta_j)} is its own column of
+// the trig operand (|D| G columns, padded to a multiple of 16: NTH), split
+// into bf16 hi and lo parts that sit in two K halves, and the norm weights
+// a separate 2G-column operand.  Per tile two contractions:
+//   [k | k] (128 x 256) . [Bhi ; Blo] (256 x NTH)  -> trig accumulator
+//   [m_hi | m_lo] (128 x 128) . Bnorm (128 x 2G)   -> norm accumulator
+// (the K tile is read twice from shared memory, once per part), then a max
+// over the |D| offset columns of each head in the epilogue.  With one column
+// per (head, offset) a tile needs NTH <= 144 trig columns, so tensor memory
+// holds two buffers of everything (trig 0..143 | 144..287, norm 288.. |
+// 304.., magnitudes 320.. | 384..): the epilogue of tile i - 1 runs while
+// the MMAs of tile i do.
 //
 // Roles as in the offset-mean kernel (tria_score_tc.cu): warps 0-7 compute
-// (magnitudes, epilogue), warp 8 producer (TMA), warp 9 MMA issuer.  Bounded
-// waits and the abort path as described in tria_tc.cuh.
+// (magnitudes of tile i, then the epilogue of tile i - 1), warp 8 producer
+// (TMA), warp 9 MMA issuer.  Bounded waits and the abort path as described
+// in tria_tc.cuh.
 #include "tria_tc.cuh"
 
 namespace tria {
@@ -34,15 +37,20 @@ constexpr int kProducerWarp = kComputeWarps;
 constexpr int kMmaWarp = kComputeWarps + 1;
 constexpr int kThreads = 32 * (kComputeWarps + 2);
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kMaxNormCol = 288, kMaxMagCol = 320;
+constexpr uint32_t kTrigCols = 144;                 // one trig buffer: |D| G <= 136, padded
+constexpr uint32_t kMaxNormCol = 2 * kTrigCols;     // norm buffers: 288.., 304..
+constexpr uint32_t kNormCols = 16;
+constexpr uint32_t kMaxMagCol = kMaxNormCol + 2 * kNormCols;  // magnitude buffers: 320.., 384..
+static_assert(kMaxMagCol + 2 * 64 <= kTmemCols, "tensor memory columns of the max-mode kernel");
 
 template <int G>
 struct MaxCfg {
   static constexpr int NN = (2 * G < 16) ? 16 : 2 * G;                  // norm columns
-  static constexpr int NT_MAX = ((2 * 17 * G + 15) / 16) * 16;          // trig columns at |D| = 17
+  static constexpr int NTH_MAX = ((17 * G + 15) / 16) * 16;             // trig columns at |D| = 17
   static constexpr int STAGES = (G >= 8) ? 2 : 4;
-  static constexpr int BMAX = (NT_MAX + NN) * 256;                       // coefficient image bytes
+  static constexpr int BMAX = (2 * NTH_MAX + NN) * 256;                  // coefficient image bytes
   static constexpr int GQ = (G >= kBandGroups) ? G / kBandGroups : 1;
+  static_assert(NN == (int)kNormCols && NTH_MAX <= (int)kTrigCols, "max-mode operand columns");
 };
 
 template <int G>
@@ -51,8 +59,8 @@ struct MaxSmem {
   alignas(1024) uint8_t b[2][MaxCfg<G>::BMAX];
   alignas(8) uint64_t full[MaxCfg<G>::STAGES];
   alignas(8) uint64_t kempty[MaxCfg<G>::STAGES];
-  alignas(8) uint64_t aready;
-  alignas(8) uint64_t accfull;
+  alignas(8) uint64_t aready[2];
+  alignas(8) uint64_t accfull[2];
   alignas(8) uint64_t bempty[2];
   SubRec rec[MaxCfg<G>::STAGES];
   alignas(16) int seq_items[kMaxSeqTable];
@@ -67,17 +75,18 @@ __device__ void mma_issuer_max(const ScoreParams &p, MaxSmem<G> &sm, uint32_t tm
                                const WaitCtl wc) {
   using Cfg = MaxCfg<G>;
   constexpr int ST = Cfg::STAGES, NN = Cfg::NN;
-  const int NT = p.geo.ncol_t;
-  const int N1 = NT < 256 ? NT : 256, N2 = NT - N1;
-  const uint32_t id1 = idesc_bf16_m128_n(N1), id2 = idesc_bf16_m128_n(N2 > 0 ? N2 : 16);
+  const int NTH = p.geo.ncol_t;
+  const uint32_t idt = idesc_bf16_m128_n(NTH);
   constexpr uint32_t idn = idesc_bf16_m128_n(NN);
   const uint64_t da0 = sw128_desc(smem_u32(&sm.k[0][0][0]));
   const uint64_t db0 = sw128_desc(smem_u32(&sm.b[0][0]));
   constexpr uint32_t kStageBytes = 2 * kHalfBlock;
-  const uint32_t nbase = 2u * NT * 128u;  // norm image after the trig image
+  const uint32_t tblk = (uint32_t)NTH * 128u;  // one 64-wide K block of the trig image
+  const uint32_t nbase = 4u * tblk;            // norm image after the trig hi and lo parts
   int i = 0;
   for (;; ++i) {
-    if (!mbar_wait(&sm.aready, i & 1, wc)) break;
+    const int ab = i & 1;
+    if (!mbar_wait(&sm.aready[ab], (i >> 1) & 1, wc)) break;
     tc_fence_after();
     const int stage = i % ST;
     const SubRec &rec = sm.rec[stage];
@@ -85,26 +94,27 @@ __device__ void mma_issuer_max(const ScoreParams &p, MaxSmem<G> &sm, uint32_t tm
     if (flags & kFlagEnd) break;
     const uint64_t da = da0 + (uint64_t)((stage * kStageBytes) >> 4);
     const uint64_t db = db0 + (uint64_t)(((uint32_t)bpar * (uint32_t)Cfg::BMAX) >> 4);
+    const uint32_t dt = tmem + (uint32_t)ab * kTrigCols;
+    // trig: K = 128 key dims against the hi part, then again against the lo part
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      const uint32_t ao = (s >> 2) * kHalfBlock + (s & 3) * 32;
-      const uint32_t bo = (uint32_t)(s >> 2) * (uint32_t)NT * 128u + (s & 3) * 32;
-      mma_bf16(tmem, da + (ao >> 4), db + (bo >> 4), id1, s > 0 ? 1u : 0u);
-      if (N2 > 0)
-        mma_bf16(tmem + (uint32_t)N1, da + (ao >> 4), db + ((bo + (uint32_t)N1 * 128u) >> 4), id2,
-                 s > 0 ? 1u : 0u);
+    for (int s = 0; s < 16; ++s) {
+      const int k = s & 7;
+      const uint32_t ao = (k >> 2) * kHalfBlock + (k & 3) * 32;
+      const uint32_t bo = (uint32_t)(s >> 2) * tblk + (k & 3) * 32;
+      mma_bf16(dt, da + (ao >> 4), db + (bo >> 4), idt, s > 0 ? 1u : 0u);
     }
     mma_commit(&sm.kempty[stage]);  // the K tile is consumed
+    const uint32_t dn = tmem + kMaxNormCol + (uint32_t)ab * kNormCols;
+    const uint32_t ta = tmem + kMaxMagCol + (uint32_t)ab * 64u;
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
       const uint32_t bo = nbase + (uint32_t)(s >> 2) * NN * 128u + (s & 3) * 32;
-      mma_bf16_ta(tmem + kMaxNormCol, tmem + kMaxMagCol + (uint32_t)(s * 8), db + (bo >> 4), idn,
-                  s > 0 ? 1u : 0u);
+      mma_bf16_ta(dn, ta + (uint32_t)(s * 8), db + (bo >> 4), idn, s > 0 ? 1u : 0u);
     }
     if (flags & kFlagLast) mma_commit(&sm.bempty[bpar]);
-    mma_commit(&sm.accfull);
+    mma_commit(&sm.accfull[ab]);  // issued last: it covers every MMA before it
   }
-  if (i > 0) mbar_drain(&sm.accfull, (i - 1) & 1, wc.status);
+  if (i > 0) mbar_drain(&sm.accfull[(i - 1) & 1], ((i - 1) >> 1) & 1, wc.status);
 }
 
 // Raw scores, fp64 moment sums and the item's moment partials of one tile.
@@ -159,11 +169,12 @@ __device__ __forceinline__ float max_nan(float a, float b) {
   return d;
 }
 
-// Epilogue of the previous tile: per head of this thread's band group,
-// S = max_j (hi_j + lo_j) + (norm hi + norm lo).
+// Epilogue of tile j (buffer j & 1): per head of this thread's band group,
+// S = max_j trig_j + (norm hi + norm lo).
 template <int G>
-__device__ __forceinline__ void epilogue_max(const ScoreParams &p, uint32_t tmem, const EpRec &pr,
-                                             int q, int rg, int lane, double (&msum)[MaxCfg<G>::GQ],
+__device__ __forceinline__ void epilogue_max(const ScoreParams &p, uint32_t tmem, int buf,
+                                             const EpRec &pr, int q, int rg, int lane,
+                                             double (&msum)[MaxCfg<G>::GQ],
                                              double (&msq)[MaxCfg<G>::GQ]) {
   constexpr int GQ = MaxCfg<G>::GQ;
   const bool active = (G >= kBandGroups) || q < G;
@@ -171,31 +182,31 @@ __device__ __forceinline__ void epilogue_max(const ScoreParams &p, uint32_t tmem
   float sc[GQ];
   if (active) {
     const uint32_t lb = tmem + ((uint32_t)(32 * rg) << 16);
+    const uint32_t tb = lb + (uint32_t)buf * kTrigCols;
+    const uint32_t nb = lb + kMaxNormCol + (uint32_t)buf * kNormCols;
 #pragma unroll
     for (int gi = 0; gi < GQ; ++gi) {
       const int g = q * GQ + gi;
-      // the head's 2 nd columns: one 32-column load (offsets 0..15; beyond
-      // 2 nd it reads the next head's columns, unused) and one 2-column load
-      // for offset 16
-      uint32_t t[32], t16[2], nv[2];
-      const uint32_t c0 = lb + (uint32_t)(g * nd * 2);
-      tmem_ld_nowait<32>(c0, t);
-      if (nd == 17) tmem_ld_nowait<2>(c0 + 32, t16);
-      tmem_ld_nowait<2>(lb + kMaxNormCol + (uint32_t)(2 * g), nv);
+      // the head's nd columns: one 16-column load (offsets 0..15; past nd it
+      // reads the next head's columns, unused) and, at nd = 17, a 2-column
+      // load for offset 16 (its second column is unused)
+      uint32_t t[16], t16[2], nv[2];
+      const uint32_t c0 = tb + (uint32_t)(g * nd);
+      tmem_ld_nowait<16>(c0, t);
+      if (nd == 17) tmem_ld_nowait<2>(c0 + 16, t16);
+      tmem_ld_nowait<2>(nb + (uint32_t)(2 * g), nv);
       tmem_wait_ld();
-      // offsets past |D| read as -inf; a pairwise tree of NaN-propagating
-      // maxes, built in place over the loaded words
+      // offsets past |D| read as -inf; a pairwise tree of NaN-propagating maxes
 #pragma unroll
       for (int j = 0; j < 16; ++j)
-        t[j] = __float_as_uint((j < nd) ? __uint_as_float(t[2 * j]) + __uint_as_float(t[2 * j + 1])
-                                        : -INFINITY);
-      const float v16 = (nd == 17) ? __uint_as_float(t16[0]) + __uint_as_float(t16[1]) : -INFINITY;
+        if (j >= nd) t[j] = __float_as_uint(-INFINITY);
 #pragma unroll
       for (int w = 1; w < 16; w *= 2) {
 #pragma unroll
         for (int j = 0; j + w < 16; j += 2 * w)
           t[j] = __float_as_uint(max_nan(__uint_as_float(t[j]), __uint_as_float(t[j + w])));
       }
+      const float v16 = (nd == 17) ? __uint_as_float(t16[0]) : -INFINITY;
       const float m = max_nan(__uint_as_float(t[0]), v16);
       sc[gi] = m + (__uint_as_float(nv[0]) + __uint_as_float(nv[1]));
     }
@@ -207,6 +218,9 @@ __device__ __forceinline__ void epilogue_max(const ScoreParams &p, uint32_t tmem
   emit_scores<G>(p, pr, sc, active, q, rg, lane, msum, msq);
 }
 
+// Tile i: magnitudes of tile i into buffer i & 1 (its previous reader, the
+// MMAs of tile i - 2, finished before this warp's epilogue of tile i - 2),
+// then the epilogue of tile i - 1 while the MMAs of tile i run.
 template <int G, int PAIR>
 __device__ void compute_max(const ScoreParams &p, MaxSmem<G> &sm, uint32_t tmem, int tid,
                             const WaitCtl wc) {
@@ -225,26 +239,24 @@ __device__ void compute_max(const ScoreParams &p, MaxSmem<G> &sm, uint32_t tmem,
     const int flags = rc.flags;
     const bool end = (flags & kFlagEnd) != 0;
     EpRec cur{};
-    uint32_t hi[W], lo[W];
     if (!end) {
       cur = ep_of(rc);
+      uint32_t hi[W], lo[W];
       mags_regs<PAIR, kBandsPerThread>(&sm.k[stage][0][0], r, q, hi, lo);
-    }
-    if (i >= 1) {
-      // the previous tile's MMAs are done: its scores, and its magnitude
-      // buffer may be overwritten
-      if (!warp_wait(&sm.accfull, (i - 1) & 1, wc, lane)) return;
-      tc_fence_after();
-      epilogue_max<G>(p, tmem, prev, q, rg, lane, msum, msq);
-    }
-    if (!end) {
-      tmem_st<W>(mag + (uint32_t)(W * q), hi);
-      tmem_st<W>(mag + (uint32_t)(32 + W * q), lo);
+      const uint32_t mb = mag + (uint32_t)((i & 1) * 64);
+      tmem_st<W>(mb + (uint32_t)(W * q), hi);
+      tmem_st<W>(mb + (uint32_t)(32 + W * q), lo);
       tmem_wait_st();
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.aready);
+    if (lane == 0) mbar_arrive(&sm.aready[i & 1]);
+    if (i >= 1) {
+      const int j = i - 1;
+      if (!warp_wait(&sm.accfull[j & 1], (j >> 1) & 1, wc, lane)) return;
+      tc_fence_after();
+      epilogue_max<G>(p, tmem, j & 1, prev, q, rg, lane, msum, msq);
+    }
     if (end) return;
     prev = cur;
   }
@@ -266,8 +278,10 @@ __global__ void __launch_bounds__(kThreads, 1) score_max_kernel(const __grid_con
       mbar_init(&sm.full[i], 1);
       mbar_init(&sm.kempty[i], 1);
     }
-    mbar_init(&sm.aready, kComputeWarps);
-    mbar_init(&sm.accfull, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.aready[i], kComputeWarps);
+      mbar_init(&sm.accfull[i], 1);
+    }
     for (int i = 0; i < 2; ++i) mbar_init(&sm.bempty[i], 1);
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -321,7 +335,7 @@ cudaError_t launch_max_g(const ScoreParams &p, cudaStream_t st) {
 
 static_assert(sizeof(MaxSmem<8>) + 1024 <= 232448, "shared memory of the G=8 max-mode kernel");
 static_assert(sizeof(MaxSmem<4>) + 1024 <= 232448, "shared memory of the G=4 max-mode kernel");
-static_assert(MaxCfg<8>::NT_MAX <= 288 - 16, "max-mode trig columns");
+
 
 }  // namespace
 
