@@ -12,6 +12,8 @@ after every other GPU test in the same process.
 """
 from __future__ import annotations
 
+import gc
+
 import pytest
 
 import synth
@@ -84,11 +86,18 @@ class _Pair:
         T.tria_compress_pass(self.st, self.ca, self.prm, self.kept_a, self.ws, self.freed_a,
                              self.nf_a)
         torch.cuda.synchronize()
-        free0 = torch.cuda.mem_get_info()[0]
-        alloc0 = torch.cuda.memory_allocated()
-        T.tria_compress_pass_static(self.st, self.cb, self.prm, self.kept_b, self.freed_b,
-                                    self.nf_b, self.status_b)
-        torch.cuda.synchronize()
+        # no garbage collection inside the measured window: a collection could
+        # free unrelated tensors and change the allocator's tally
+        gc.collect()
+        gc.disable()
+        try:
+            free0 = torch.cuda.mem_get_info()[0]
+            alloc0 = torch.cuda.memory_allocated()
+            T.tria_compress_pass_static(self.st, self.cb, self.prm, self.kept_b, self.freed_b,
+                                        self.nf_b, self.status_b)
+            torch.cuda.synchronize()
+        finally:
+            gc.enable()
         if check_no_alloc:
             assert torch.cuda.mem_get_info()[0] == free0, f"{what}: device memory changed"
             assert torch.cuda.memory_allocated() == alloc0
