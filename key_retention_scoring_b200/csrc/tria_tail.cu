@@ -73,7 +73,6 @@ template <int G, int KPT>
 __device__ void slice_keys(const float *raw, int P, const float *s_mean, const float *s_inv,
                            uint32_t *keys, uint32_t *hist, int tid) {
   constexpr int NT = kTailThreads;
-  const int lane = tid & 31;
   constexpr int U = 8;  // float4 loads in flight per thread
   const float4 *src = reinterpret_cast<const float4 *>(raw);
   if constexpr (G >= 4) {
@@ -111,7 +110,7 @@ __device__ void slice_keys(const float *raw, int P, const float *s_mean, const f
         const uint32_t k = nan ? 0u : order_key(a);
         const bool lead = (j < n4) && (tid % LPC) == 0;
         if (lead) keys[key_word<KPT>(j / LPC)] = k;
-        hist_add(hist, k >> 20, lead, lane);
+        hist_add(hist, k >> 20, lead);
       }
     }
   } else {
@@ -149,7 +148,7 @@ __device__ void slice_keys(const float *raw, int P, const float *s_mean, const f
           const uint32_t k = nan ? 0u : order_key(a);
           const bool in = (j < n4) && c < P;
           if (in) keys[key_word<KPT>(c)] = k;
-          hist_add(hist, k >> 20, in, lane);
+          hist_add(hist, k >> 20, in);
         }
       }
     }
