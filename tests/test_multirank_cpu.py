@@ -76,8 +76,9 @@ def test_reference_arm_rank_gating(capsys, monkeypatch):
 
 
 def test_reference_arm_line_on_rank0(capsys):
-    """Rank 0 times the oracle on one unit per step and prints the contract's
-    JSON line (the tiny configuration keeps this to a second)."""
+    """Rank 0 times the oracle (one process per host core, one unit each per
+    step) and prints the contract's JSON line with the GPU arm's config (the
+    tiny configuration keeps this to seconds)."""
     import json
 
     import bench
@@ -90,6 +91,9 @@ def test_reference_arm_line_on_rank0(capsys):
     assert line["impl"] == "reference" and line["value"] > 0 and line["steps"] == 2
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+    import synth
+    assert line["config"] == bench.config_desc(synth.CONFIGS[0])
+    assert line["cpu_baseline"]["cores"] == bench.host_cores()
 
 
 def test_recorded_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
