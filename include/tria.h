@@ -149,8 +149,8 @@ typedef enum {
                            published default; computed folded (Eq. 7)               */
   TRIA_OFFSET_MAX = 1   /* the maximum over D instead (the non-default variant named
                            at the end of sec. 4 of the same article); not foldable:
-                           |D| scores per head per key.  Needs |D| <= 17 and
-                           G * |D| <= 136 (G <= 8 at |D| = 17), else UNSUPPORTED    */
+                           |D| scores per head per key.  Needs G <= 8, |D| <= 17
+                           and G * |D| <= 136, else UNSUPPORTED                    */
 } tria_offset_reduce;
 
 /* Retention parameters (one set for all units of a call).  Zero-initialise

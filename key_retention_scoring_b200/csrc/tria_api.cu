@@ -135,7 +135,8 @@ tria_status make_geom(const tria_stats *stats, const tria_cache_view *cache,
   g.ncol_t = ((g.n_off * g.g + 15) / 16) * 16;
   g.ncol_n = g.ncol;
   if (g.mode == TRIA_OFFSET_MAX) {
-    if (g.n_off > 17 || 2 * g.n_off * g.g > kMaxOffCols) return TRIA_ERR_UNSUPPORTED;
+    // the max-over-offsets kernel is built for G <= 8
+    if (g.g > 8 || g.n_off > 17 || 2 * g.n_off * g.g > kMaxOffCols) return TRIA_ERR_UNSUPPORTED;
     // trig hi and lo parts (two 64-wide K blocks of 128-byte rows each), norm
     g.b_bytes = (2 * g.ncol_t + g.ncol_n) * 256;
   } else {

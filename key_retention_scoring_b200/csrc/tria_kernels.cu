@@ -139,33 +139,40 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
     }
     __syncthreads();
     unsigned char *dst = reinterpret_cast<unsigned char *>(p.btile) + u * (int64_t)g.b_bytes;
+    // the unit's E[q_g] mask per head and band (read 17 x 2 times per value below)
+    __shared__ double2 mu_s[TRIA_MAX_GROUP][kBands];
+    for (int i = t; i < g.g * kBands; i += kThreads)
+      mu_s[i / kBands][i % kBands] = p.mu_raw[((int64_t)l * g.hq + h * g.g) * kBands + i];
+    __syncthreads();
     // trig rows n = gg nd + j over the 128 key dims: the hi parts in two
-    // 64-wide blocks, then the lo parts in two more
-    for (int i = t; i < 2 * g.ncol_t * 16; i += kThreads) {
-      const int part = i / (g.ncol_t * 16), i2 = i % (g.ncol_t * 16);
-      const int n = i2 >> 4, ch = i2 & 15, kb = ch >> 3, c8 = ch & 7;
+    // 64-wide blocks, then the lo parts in two more (each value computed once)
+    for (int i = t; i < g.ncol_t * 16; i += kThreads) {
+      const int n = i >> 4, ch = i & 15, kb = ch >> 3, c8 = ch & 7;
       const int gg = n / nd, j = n % nd;
-      uint32_t w[4];
+      uint32_t whi[4], wlo[4];
       for (int e = 0; e < 8; e += 2) {
-        uint16_t b2[2];
+        uint16_t h2[2], l2[2];
         for (int q2 = 0; q2 < 2; ++q2) {
           const int k = ch * 8 + e + q2;  // key dim
           float x = 0.0f;
           if (gg < g.g) {
             const int f = (g.pairing == TRIA_PAIR_NEOX) ? (k & 63) : (k >> 1);
             const bool im = (g.pairing == TRIA_PAIR_NEOX) ? (k >= 64) : (k & 1);
-            const double2 mu = p.mu_raw[((int64_t)l * g.hq + h * g.g + gg) * kBands + f];
+            const double2 mu = mu_s[gg][f];
             const double2 r = rotj[f][j];
             x = im ? (float)(mu.x * r.y + mu.y * r.x) : (float)(mu.x * r.x - mu.y * r.y);
           }
-          const uint16_t hi = bf16_rn_bits(x);
-          const uint16_t lo = bf16_rn_bits(x - __uint_as_float((uint32_t)hi << 16));
-          b2[q2] = (part == 0) ? hi : lo;
+          h2[q2] = bf16_rn_bits(x);
+          l2[q2] = bf16_rn_bits(x - __uint_as_float((uint32_t)h2[q2] << 16));
         }
-        w[e >> 1] = (uint32_t)b2[0] | ((uint32_t)b2[1] << 16);
+        whi[e >> 1] = (uint32_t)h2[0] | ((uint32_t)h2[1] << 16);
+        wlo[e >> 1] = (uint32_t)l2[0] | ((uint32_t)l2[1] << 16);
       }
-      *reinterpret_cast<uint4 *>(dst + (2 * part + kb) * (g.ncol_t * 128) + n * 128 +
-                                 ((c8 ^ (n & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      const int64_t off = (int64_t)n * 128 + ((c8 ^ (n & 7)) << 4);
+      *reinterpret_cast<uint4 *>(dst + kb * (g.ncol_t * 128) + off) =
+          make_uint4(whi[0], whi[1], whi[2], whi[3]);
+      *reinterpret_cast<uint4 *>(dst + (2 + kb) * (g.ncol_t * 128) + off) =
+          make_uint4(wlo[0], wlo[1], wlo[2], wlo[3]);
     }
     // norm rows n = 2 gg + part over the magnitude dims: block 0 multiplies
     // |k_f| hi (w_f split hi/lo over the rows), block 1 |k_f| lo (w_f hi, 0)

@@ -481,6 +481,16 @@ def test_offset_max_unsupported_shapes():
         with pytest.raises(T.TriaError) as ei:
             T.tria_workspace_size(st, cache, prm)
         assert ei.value.status == 2
+        # G = 16 with few offsets (2 |D| G <= 272) is unsupported as well: the
+        # max-over-offsets kernel is built for G <= 8
+        st.free()
+        cfg4 = cfg.scaled(offset_log2_max=3)
+        w4 = synth.Workload(cfg4, with_values=False, with_positions=False)
+        st = load_stats(w4)
+        cache = T.Cache.from_workload(w4)
+        with pytest.raises(T.TriaError) as ei:
+            T.tria_workspace_size(st, cache, prm)
+        assert ei.value.status == 2
         # the mean mode of the same shape is fine
         T.tria_workspace_size(st, cache, T.params(cfg.budget, cfg.window, cfg.sinks))
         with pytest.raises(T.TriaError) as ei:
