@@ -205,6 +205,14 @@ def test_no_window_no_sinks_gqa1_and_gqa2():
                                        pairing=synth.PAIR_INTERLEAVED))
 
 
+def test_gqa16():
+    # G = 16: the scoring kernel's 32-column instance (5-stage ring) and the
+    # tail's four-lanes-per-candidate path, with a ragged last tile
+    full_check(synth.CONFIGS[0].scaled(n_q_heads=32, n_kv_heads=2, seq_len=3000))
+    # and a unit long enough for a cluster of two tail blocks
+    full_check(synth.CONFIGS[4].scaled(n_layers=1, n_q_heads=16, n_kv_heads=1, seq_len=50000))
+
+
 def test_offset_sets_and_theta():
     for m in (0, 7, 12):
         full_check(synth.CONFIGS[0].scaled(offset_log2_max=m, seq_len=1800, theta=5e5))
