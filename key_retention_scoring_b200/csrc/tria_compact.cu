@@ -33,10 +33,12 @@ constexpr int kPieces = kRowBytes / 16;                   // 16-byte pieces per 
 constexpr int kRowStep = kCpThreads / kPieces;            // rows covered by one pass of the block
 constexpr int kRowsPerThread = kCpRows / kRowStep;        // 8
 
+constexpr int kMinBlock = 8;                              // smallest paged block size
 struct CpSmem {
   alignas(16) uint8_t buf[kCpDepth][kCpRows][kRowBytes];
   int32_t pos[kCpDepth][kCpRows];
   int32_t src[kCpDepth][kCpRows];   // source of each destination row (-1: stays)
+  int32_t dblk[kCpDepth][kCpRows / kMinBlock];  // paged: the chunk's destination blocks
 };
 
 struct ItemGeo {
@@ -117,6 +119,7 @@ __device__ void update_len(const CompactParams &p, const ItemGeo &g) {
   }
 }
 
+template <bool PAGED>
 __global__ void __launch_bounds__(kCpThreads, 1) compact_kernel(const __grid_constant__ CompactParams p) {
   extern __shared__ __align__(16) uint8_t smem_cp[];
   CpSmem &sm = *reinterpret_cast<CpSmem *>(smem_cp);
@@ -153,22 +156,47 @@ __global__ void __launch_bounds__(kCpThreads, 1) compact_kernel(const __grid_con
     }
   };
 
-  // kept entries (raw) of this thread's rows of chunk q
-  auto fetch = [&](const Cur &q, int (&kv)[kRowsPerThread]) {
+  constexpr bool paged = PAGED;
+  const int bs = p.cache.block_size;  // a power of two (8 .. 128)
+  const int bsh = __ffs(bs) - 1, bsm = bs - 1;
+  // kept entries (raw) of this thread's rows of chunk q and, paged, the
+  // block-table entries of their sources (both used one iteration later, so
+  // the dependent table load is off the copy path)
+  auto fetch = [&](const Cur &q, int (&kv)[kRowsPerThread], int (&kb)[kRowsPerThread]) {
     if (q.i < my_items) {
-      const int32_t *kept = p.kept + (item_of(q.i) >> 1) * geo.budget;
+      const int64_t u = item_of(q.i) >> 1;
+      const int32_t *kept = p.kept + u * geo.budget;
 #pragma unroll
       for (int e = 0; e < kRowsPerThread; ++e) {
         const int j = q.c * kCpRows + rr + e * kRowStep;
         kv[e] = (j < geo.budget) ? __ldg(kept + j) : -1;
       }
+      if constexpr (paged) {
+        const int32_t *bt = p.cache.block_table +
+                            (int64_t)(u / ((int64_t)geo.nl * geo.hkv)) * p.cache.max_blocks;
+#pragma unroll
+        for (int e = 0; e < kRowsPerThread; ++e) {
+          const int j = q.c * kCpRows + rr + e * kRowStep, v = kv[e];
+          const bool moves = j < geo.budget && v != j && v >= 0 && v < cap && j < cap;
+          kb[e] = moves ? __ldg(bt + (v >> bsh)) : 0;
+        }
+      }
     }
   };
   // copies of this thread's pieces of chunk q into buffer b (one commit
   // group per chunk, empty past the end)
-  auto issue = [&](const Cur &q, int b, const int (&kv)[kRowsPerThread]) {
+  auto issue = [&](const Cur &q, int b, const int (&kv)[kRowsPerThread],
+                   const int (&kb)[kRowsPerThread]) {
     if (q.i < my_items) {
       const ItemGeo g = item_geo(p, item_of(q.i));
+      if constexpr (paged) {
+        // the chunk's destination blocks, for its write-back two iterations on
+        const int nb = kCpRows >> bsh, b0 = (q.c * kCpRows) >> bsh;
+        if (t < nb)
+          sm.dblk[b][t] = (b0 + t < p.cache.max_blocks)
+                              ? __ldg(p.cache.block_table + (int64_t)g.s * p.cache.max_blocks + b0 + t)
+                              : 0;
+      }
 #pragma unroll
       for (int e = 0; e < kRowsPerThread; ++e) {
         const int r = rr + e * kRowStep, j = q.c * kCpRows + r;
@@ -176,7 +204,10 @@ __global__ void __launch_bounds__(kCpThreads, 1) compact_kernel(const __grid_con
         const int src = (j >= geo.budget || v == j || v < 0 || v >= cap || j >= cap) ? -1 : v;
         if (piece == 0) sm.src[b][r] = src;
         if (src >= 0) {
-          cp16(&sm.buf[b][r][piece * 16], g.base + row_off(p.cache, g.s, g.h, src) * 2 + piece * 16);
+          const int64_t off = paged ? (int64_t)kb[e] * p.cache.s_blk + (int64_t)(src & bsm) * p.cache.s_tok +
+                                          (int64_t)g.h * p.cache.s_head
+                                    : row_off(p.cache, g.s, g.h, src);
+          cp16(&sm.buf[b][r][piece * 16], g.base + off * 2 + piece * 16);
           if (g.pos != nullptr && piece == 0) cp4(&sm.pos[b][r], g.pos + src);
         }
       }
@@ -184,21 +215,21 @@ __global__ void __launch_bounds__(kCpThreads, 1) compact_kernel(const __grid_con
     cp_commit();
   };
 
-  int kv[kRowsPerThread];
+  int kv[kRowsPerThread], kb[kRowsPerThread];
   Cur fc = start();  // next chunk to fetch
   for (int k = 0; k < kCpAhead; ++k) {
-    fetch(fc, kv);
-    issue(fc, k % kCpDepth, kv);
+    fetch(fc, kv, kb);
+    issue(fc, k % kCpDepth, kv, kb);
     advance(fc);
   }
   Cur pend = fc;  // fetched, to be issued at the next iteration
-  fetch(pend, kv);
+  fetch(pend, kv, kb);
   advance(fc);
   Cur wc = start();  // chunk to write back
   for (int64_t k = 0; wc.i < my_items; ++k) {
-    issue(pend, (int)((k + kCpAhead) % kCpDepth), kv);
+    issue(pend, (int)((k + kCpAhead) % kCpDepth), kv, kb);
     pend = fc;
-    fetch(pend, kv);  // used at the next iteration
+    fetch(pend, kv, kb);  // used at the next iteration
     advance(fc);
     cp_wait<kCpAhead>();  // this thread's copies of chunk k have landed
     __syncthreads();      // ... and every other thread's
@@ -212,7 +243,10 @@ __global__ void __launch_bounds__(kCpThreads, 1) compact_kernel(const __grid_con
       const int src = __shfl_sync(kFull, mine, (threadIdx.x & 31) & ~(kPieces - 1));
       if (src >= 0) {
         const uint4 v = *reinterpret_cast<const uint4 *>(&sm.buf[b][r][piece * 16]);
-        *reinterpret_cast<uint4 *>(g.base + row_off(p.cache, g.s, g.h, j) * 2 + piece * 16) = v;
+        const int64_t off = paged ? (int64_t)sm.dblk[b][r >> bsh] * p.cache.s_blk +
+                                        (int64_t)(j & bsm) * p.cache.s_tok + (int64_t)g.h * p.cache.s_head
+                                  : row_off(p.cache, g.s, g.h, j);
+        *reinterpret_cast<uint4 *>(g.base + off * 2 + piece * 16) = v;
         if (g.pos != nullptr && piece == 0) g.pos[j] = sm.pos[b][r];
       }
     }
@@ -283,14 +317,16 @@ cudaError_t launch_layer_lens(const LensParams &p, cudaStream_t st) {
 
 cudaError_t launch_compact(const CompactParams &p, cudaStream_t st) {
   const int smem = (int)sizeof(CpSmem);
-  cudaError_t e = cudaFuncSetAttribute(compact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const bool paged = p.cache.layout == TRIA_LAYOUT_PAGED;
+  auto kern = paged ? compact_kernel<true> : compact_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   int64_t grid = p.geo.n_units * 2;
   if (grid > sms) grid = sms;
-  compact_kernel<<<(unsigned)grid, kCpThreads, smem, st>>>(p);
+  kern<<<(unsigned)grid, kCpThreads, smem, st>>>(p);
   return cudaGetLastError();
 }
 
