@@ -245,7 +245,10 @@ __global__ void __launch_bounds__(kTailThreads, 1) cluster_tail_kernel(const __g
   const Geom &geo = p.geo;
   const int t = threadIdx.x;
   const int cs = p.cluster;
-  const int64_t u = blockIdx.x / cs;
+  // the last units first: the scoring kernel claims units in ascending
+  // order, so the raw scores it wrote last may still be in L2 (154.4 against
+  // 156.8 us per Qwen3-32B 32K pass)
+  const int64_t u = p.geo.n_units - 1 - blockIdx.x / cs;
   const int rank = (int)(blockIdx.x % cs);  // clusters are cs consecutive blocks along x
   const int s = (int)(u / ((int64_t)geo.nl * geo.hkv));
   const int lrel = (int)((u / geo.hkv) % geo.nl);
