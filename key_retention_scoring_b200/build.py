@@ -10,7 +10,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(os.path.dirname(PKG), "include")
 LIB = os.path.join(PKG, "libtria.so")
-SOURCES = ["tria_api.cu", "tria_kernels.cu", "tria_score_tc.cu", "tria_score_max.cu", "tria_tail.cu",
+SOURCES = ["tria_api.cu", "tria_kernels.cu", "tria_score_tc.cu", "tria_score_max.cu",
+           "tria_score_grouped.cu", "tria_tail.cu",
            "tria_compact.cu",
            "tria_calib.cu", "tria_static.cu", "tria_decode.cu", "tria_stats_io.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -143,6 +143,11 @@ tria_status make_geom(const tria_stats *stats, const tria_cache_view *cache,
     g.b_bytes = g.ncol * kCoefK * 2;
   }
   if (g.n_units * (int64_t)g.tiles_max > INT32_MAX) return TRIA_ERR_UNSUPPORTED;
+  // paged offset-mean scoring reads whole blocks when one block of every KV
+  // head is a 128-row tile and the heads' coefficient columns fit N <= 128
+  g.grouped = (cache->layout == TRIA_LAYOUT_PAGED && g.mode == TRIA_OFFSET_MEAN &&
+               (g.hkv == 2 || g.hkv == 4 || g.hkv == 8) && cache->block_size * g.hkv == 128 &&
+               g.g <= 8 && g.hkv * g.ncol <= 128) ? 1 : 0;
   *geo = g;
   return TRIA_OK;
 }
@@ -173,7 +178,8 @@ struct MapKey {
   bool operator<(const MapKey &o) const { return std::memcmp(this, &o, sizeof(MapKey)) < 0; }
 };
 
-tria_status k_tensor_map(const tria_cache_view *c, int hkv, const void *base, CUtensorMap *out) {
+tria_status k_tensor_map(const tria_cache_view *c, int hkv, bool all_heads, const void *base,
+                        CUtensorMap *out) {
   MapKey key;
   std::memset(&key, 0, sizeof(key));
   key.ptr = base;
@@ -188,8 +194,21 @@ tria_status k_tensor_map(const tria_cache_view *c, int hkv, const void *base, CU
     key.strides[1] = (uint64_t)c->stride_head * 2;
     key.strides[2] = (uint64_t)c->stride_seq * 2;
     key.box[0] = 64; key.box[1] = 128; key.box[2] = 1; key.box[3] = 1;
+  } else if (all_heads) {
+    // [num_blocks][block_size][hkv][128] by strides, dimensions ordered (dim,
+    // token, head, block): box = one block of every head x 64 dims, rows
+    // head-major (head block_size + token)
+    key.dims[0] = 128;
+    key.dims[1] = (uint64_t)c->block_size;
+    key.dims[2] = (uint64_t)hkv;
+    key.dims[3] = (uint64_t)c->num_blocks;
+    key.strides[0] = (uint64_t)c->stride_token * 2;
+    key.strides[1] = (uint64_t)c->stride_head * 2;
+    key.strides[2] = (uint64_t)c->stride_block * 2;
+    key.box[0] = 64; key.box[1] = (uint32_t)c->block_size; key.box[2] = (uint32_t)hkv; key.box[3] = 1;
   } else {
-    // [num_blocks][block_size][hkv][128] by strides; box = one block of one head x 64 dims
+    // [num_blocks][block_size][hkv][128] by strides; box = one block of one
+    // head x 64 dims
     key.dims[0] = 128;
     key.dims[1] = (uint64_t)hkv;
     key.dims[2] = (uint64_t)c->block_size;
@@ -283,7 +302,7 @@ tria_status make_score(const Geom &g, const tria_cache_view *c, const tria_param
                        int layer1, void *ws, const WsLayout &wl, ScoreParams &sp) {
   std::memset(&sp, 0, sizeof(sp));
   for (int l = layer0; l < layer1; ++l) {
-    const tria_status st = k_tensor_map(c, g.hkv, c->k_layers[l], &sp.kmap[l - layer0]);
+    const tria_status st = k_tensor_map(c, g.hkv, g.grouped != 0, c->k_layers[l], &sp.kmap[l - layer0]);
     if (st != TRIA_OK) return st;
   }
   sp.geo = g;

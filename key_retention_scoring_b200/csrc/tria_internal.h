@@ -54,6 +54,7 @@ struct Geom {
   int ncol_t;    // max mode: trig operand rows, |D| G rounded up to 16
   int ncol_n;    // max mode: norm operand rows, max(16, 2G)
   int b_bytes;   // bytes of one unit's coefficient image
+  int grouped;   // paged scoring tiles of one block x all KV heads (tria_score_grouped.cu)
 };
 
 // Cache addressing (pointers indexed by layer - layer0).
@@ -184,6 +185,7 @@ cudaError_t launch_coef(const CoefParams &p, cudaStream_t st);
 // (tria_score_max.cu).
 cudaError_t launch_score(const ScoreParams &p, cudaStream_t st);
 cudaError_t launch_score_max(const ScoreParams &p, cudaStream_t st);
+cudaError_t launch_score_grouped(const ScoreParams &p, cudaStream_t st);
 cudaError_t launch_tail(const TailParams &p, cudaStream_t st);
 cudaError_t launch_select(const SelectParams &p, cudaStream_t st);
 // Normalize-then-max + selection with one thread-block cluster per unit and

@@ -59,6 +59,9 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
   __shared__ float cf[TRIA_MAX_GROUP][3 * kBands];
   __shared__ int s_part[kThreads];
 
+  // scheduling items per 1024-slot range of a (sequence, layer): one per KV
+  // head, or one for all heads when the paged tiles hold every head
+  const int ipu = g.grouped ? 1 : g.hkv;
   if (u == 0) {
     if (t == 0) *p.item_counter = 0u;
     if (!g.per_layer) {
@@ -70,7 +73,7 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
         const int sq = t * per + i;
         if (sq < g.n_seq) {
           const int n = unit_len(g, sq, 0);
-          if (compresses(g, n, 0)) local += unit_tiles(n, g.window, g.sinks) * g.nl * g.hkv;
+          if (compresses(g, n, 0)) local += unit_tiles(n, g.window, g.sinks) * g.nl * ipu;
         }
       }
       int total;
@@ -80,7 +83,7 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
         if (sq < g.n_seq) {
           p.seq_items[sq] = run;
           const int n = unit_len(g, sq, 0);
-          if (compresses(g, n, 0)) run += unit_tiles(n, g.window, g.sinks) * g.nl * g.hkv;
+          if (compresses(g, n, 0)) run += unit_tiles(n, g.window, g.sinks) * g.nl * ipu;
         }
       }
       if (t == 0) p.seq_items[g.n_seq] = total;
@@ -91,7 +94,7 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
       const int per = (rows + kThreads - 1) / kThreads;
       auto row_n = [&](int r) {
         const int n = unit_len(g, r / g.nl, r % g.nl);
-        return compresses(g, n, r % g.nl) ? unit_tiles(n, g.window, g.sinks) * g.hkv : 0;
+        return compresses(g, n, r % g.nl) ? unit_tiles(n, g.window, g.sinks) * ipu : 0;
       };
       int local = 0;
       for (int i = 0; i < per; ++i) {
@@ -215,7 +218,12 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
     cf[gg][2 * kBands + f] = (float)p.w_norm[qi];
   }
   __syncthreads();
-  unsigned char *dst = reinterpret_cast<unsigned char *>(p.btile) + u * (int64_t)g.b_bytes;
+  // grouped paged tiles: the hkv units of a (sequence, layer) share one image
+  // with their columns side by side (unit h at rows h ncol .. h ncol + ncol - 1
+  // of every K block)
+  const int64_t gu = g.grouped ? u - h : u;
+  const int rows = g.grouped ? g.hkv * g.ncol : g.ncol, row0 = g.grouped ? h * g.ncol : 0;
+  unsigned char *dst = reinterpret_cast<unsigned char *>(p.btile) + gu * (int64_t)g.b_bytes;
   for (int i = t; i < g.ncol * (kCoefK / 8); i += kThreads) {
     const int n = i / (kCoefK / 8), ch = i % (kCoefK / 8), k0 = ch * 8;
     const int gg = n >> 1, part = n & 1;
@@ -242,7 +250,7 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
       w[e >> 1] = (uint32_t)b2[0] | ((uint32_t)b2[1] << 16);
     }
     const int kb = ch >> 3, c8 = ch & 7;
-    *reinterpret_cast<uint4 *>(dst + kb * (g.ncol * 128) + n * 128 + ((c8 ^ (n & 7)) << 4)) =
+    *reinterpret_cast<uint4 *>(dst + kb * (rows * 128) + (row0 + n) * 128 + ((c8 ^ (n & 7)) << 4)) =
         make_uint4(w[0], w[1], w[2], w[3]);
   }
 }

@@ -342,6 +342,7 @@ static_assert(sizeof(TcSmem<16>) + 1024 <= 232448, "shared memory of the G=16 ke
 
 cudaError_t launch_score(const ScoreParams &p, cudaStream_t st) {
   if (p.geo.mode == TRIA_OFFSET_MAX) return launch_score_max(p, st);
+  if (p.geo.grouped) return launch_score_grouped(p, st);
   switch (p.geo.g) {
     case 1: return launch_g<1>(p, st);
     case 2: return launch_g<2>(p, st);

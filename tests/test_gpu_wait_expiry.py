@@ -78,6 +78,14 @@ def test_wait_expiry_sets_status_and_returns(offset_reduce, use_score):
     full_check(synth.CONFIGS[0], offset_reduce=offset_reduce)
 
 
+def test_wait_expiry_paged_whole_block_scoring():
+    # a paged batch with 8 KV heads and 16-token blocks: the scoring kernel
+    # that reads whole blocks (all heads per tile)
+    cfg = synth.CONFIGS[3].scaled(n_layers=1, n_seq=2, len_range=(3000, 5000))
+    _expire(cfg, 0, False)
+    full_check(cfg)
+
+
 def test_default_limit_is_not_hit():
     cfg = synth.CONFIGS[2].scaled(n_layers=2, seq_len=4096)
     w = synth.Workload(cfg)
