@@ -401,9 +401,12 @@ def main():
     ap.add_argument("--layers", type=int, default=0,
                     help="override the workload's layer count (small profiling cases)")
     ap.add_argument("--only-extra", default="",
-                    choices=["", "decode_attention", "offset_max", "layer_budgets", "calibration"],
+                    choices=["", "decode_attention", "offset_max", "layer_budgets", "calibration",
+                             "workload"],
                     help="after the warm-up passes run just this extra and print its result "
                          "(profiling of one kernel on a small case)")
+    ap.add_argument("--seqs", type=int, default=0,
+                    help="with --only-extra workload: override the workload's sequence count")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -421,6 +424,21 @@ def main():
     from key_retention_scoring_b200 import build as tria_build
 
     torch.cuda.set_device(local)
+    if args.only_extra == "workload":
+        # one pass of a workload shape (any layout), optionally cut to fewer
+        # layers / sequences: the `workloads` measurement on a small case
+        tria_build.build()
+        synth.build()
+        wcfg = synth.CONFIGS[args.config]
+        if args.layers:
+            wcfg = wcfg.scaled(n_layers=args.layers)
+        if args.seqs:
+            wcfg = wcfg.scaled(n_seq=args.seqs)
+        hbm, _ = peaks()
+        res = workload_pass(T, torch, args.config, hbm, cfg=wcfg)
+        if rank == 0:
+            print(json.dumps({"extra": "workload", "config": config_desc(wcfg), **res}), flush=True)
+        return 0
     if world > 1:
         from datetime import timedelta
 
@@ -611,16 +629,17 @@ def pass_roofline(k_bytes, compact_bytes, ms, hbm):
             "compact_bytes": compact_bytes, "us": ms * 1e3}
 
 
-def workload_pass(T, torch, ci, hbm, passes=None):
+def workload_pass(T, torch, ci, hbm, passes=None, cfg=None):
     """One full compression pass of workload `ci` (the other shapes of the
-    pages' workloads), timed with the pass's own CUDA events.  Contiguous
+    pages' workloads; `cfg`, when given, a cut-down instance of it), timed
+    with the pass's own CUDA events.  Contiguous
     caches restore the rows compaction overwrites between passes; the paged
     batch (157.5 GB of K + V, no room for backups) is generated afresh
     before each pass, after a warm-up pass of the same kernels on a small
     instance of it."""
     import synth
 
-    cfg = synth.CONFIGS[ci]
+    cfg = synth.CONFIGS[ci] if cfg is None else cfg
     paged = cfg.layout == synth.LAYOUT_PAGED
     passes = passes or (2 if paged else 5)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
@@ -697,7 +716,9 @@ def workload_pass(T, torch, ci, hbm, passes=None):
                "kernels_us": {"coef": 1e3 * seg["coef"], "score": 1e3 * seg["score"],
                               "normalize_select": 1e3 * seg["select"],
                               "compact": 1e3 * seg["compact"]},
-               "roofline": {"bound": "hbm", "kernel": "score_tc_kernel",
+               "roofline": {"bound": "hbm",
+                            "kernel": "scoring (score_tc_kernel; score_grp_kernel for paged blocks "
+                                      "of 128 rows over all KV heads)",
                             "achieved": k_bytes / (seg["score"] * 1e-3) / 1e9, "peak": hbm,
                             "unit": "GB/s",
                             "frac": k_bytes / (seg["score"] * 1e-3) / 1e9 / hbm,
