@@ -144,10 +144,11 @@ tria_status make_geom(const tria_stats *stats, const tria_cache_view *cache,
   }
   if (g.n_units * (int64_t)g.tiles_max > INT32_MAX) return TRIA_ERR_UNSUPPORTED;
   // paged offset-mean scoring reads whole blocks when one block of every KV
-  // head is a 128-row tile and the heads' coefficient columns fit N <= 128
+  // head is a 128-row tile; the heads' 2G coefficient columns each, side by
+  // side, are the MMA's N (16 <= N <= 128)
   g.grouped = (cache->layout == TRIA_LAYOUT_PAGED && g.mode == TRIA_OFFSET_MEAN &&
                (g.hkv == 2 || g.hkv == 4 || g.hkv == 8) && cache->block_size * g.hkv == 128 &&
-               g.g <= 8 && g.hkv * g.ncol <= 128) ? 1 : 0;
+               g.g <= 8 && g.hkv * 2 * g.g >= 16) ? 1 : 0;
   *geo = g;
   return TRIA_OK;
 }

@@ -54,7 +54,8 @@ struct Geom {
   int ncol_t;    // max mode: trig operand rows, |D| G rounded up to 16
   int ncol_n;    // max mode: norm operand rows, max(16, 2G)
   int b_bytes;   // bytes of one unit's coefficient image
-  int grouped;   // paged scoring tiles of one block x all KV heads (tria_score_grouped.cu)
+  int grouped;   // paged scoring tiles of one block x all KV heads (tria_score_grouped.cu):
+                 // the units of a (sequence, layer) share one image of 2G columns each
 };
 
 // Cache addressing (pointers indexed by layer - layer0).

@@ -219,12 +219,13 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
   }
   __syncthreads();
   // grouped paged tiles: the hkv units of a (sequence, layer) share one image
-  // with their columns side by side (unit h at rows h ncol .. h ncol + ncol - 1
-  // of every K block)
+  // with their 2G columns side by side (unit h at rows 2G h .. 2G h + 2G - 1
+  // of every K block; no padding columns)
   const int64_t gu = g.grouped ? u - h : u;
-  const int rows = g.grouped ? g.hkv * g.ncol : g.ncol, row0 = g.grouped ? h * g.ncol : 0;
+  const int ucols = g.grouped ? 2 * g.g : g.ncol;
+  const int rows = g.grouped ? g.hkv * ucols : g.ncol, row0 = g.grouped ? h * ucols : 0;
   unsigned char *dst = reinterpret_cast<unsigned char *>(p.btile) + gu * (int64_t)g.b_bytes;
-  for (int i = t; i < g.ncol * (kCoefK / 8); i += kThreads) {
+  for (int i = t; i < ucols * (kCoefK / 8); i += kThreads) {
     const int n = i / (kCoefK / 8), ch = i % (kCoefK / 8), k0 = ch * 8;
     const int gg = n >> 1, part = n & 1;
     uint32_t w[4];
@@ -249,8 +250,8 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
       }
       w[e >> 1] = (uint32_t)b2[0] | ((uint32_t)b2[1] << 16);
     }
-    const int kb = ch >> 3, c8 = ch & 7;
-    *reinterpret_cast<uint4 *>(dst + kb * (rows * 128) + (row0 + n) * 128 + ((c8 ^ (n & 7)) << 4)) =
+    const int kb = ch >> 3, c8 = ch & 7, row = row0 + n;
+    *reinterpret_cast<uint4 *>(dst + kb * (rows * 128) + row * 128 + ((c8 ^ (row & 7)) << 4)) =
         make_uint4(w[0], w[1], w[2], w[3]);
   }
 }

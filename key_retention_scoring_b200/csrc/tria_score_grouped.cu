@@ -8,7 +8,8 @@
 // bytes, two TMA boxes of {64 dims, BS tokens, HKV heads}.  Rows are
 // head-major (row = head BS + token).  Each row must meet its own head's
 // coefficients, so the B operand holds the HKV units' coefficient columns
-// side by side (N = HKV NCOL <= 128, written so by the coefficient kernel):
+// side by side (2G each, no padding: N = 2 G HKV, 16 <= N <= 128, written so
+// by the coefficient kernel):
 //   D[128 x N] = [ktilde | m_hi | m_lo] (128 x 256) . [B_0 | ... | B_{HKV-1}]
 // and row r keeps the block of columns of head r / BS (the other blocks
 // are computed and ignored: the tensor pipe has the room).  The score of a
@@ -41,14 +42,14 @@ constexpr uint32_t kTmemCols = 512;
 
 template <int G, int HKV>
 struct GrpCfg {
-  static constexpr int NCOL = (2 * G < 16) ? 16 : 2 * G;  // one unit's columns
+  static constexpr int NCOL = 2 * G;                        // one unit's columns (hi, lo per head)
   static constexpr int N = HKV * NCOL;                      // MMA N
   static constexpr int BS = kRows / HKV;                    // tokens per tile (the block size)
-  static constexpr int STAGES = 4;
+  static constexpr int STAGES = (N <= 64) ? 5 : 4;
   static constexpr int GQ = (G >= kBandGroups) ? G / kBandGroups : 1;
   static constexpr int BBLK = N * 128;                      // bytes per 64-wide K block of B
   static constexpr uint32_t MAG0 = 2 * N;                   // magnitude buffers after two accumulators
-  static_assert(N % 16 == 0 && N <= 128, "MMA N of the grouped kernel");
+  static_assert(N % 16 == 0 && N >= 16 && N <= 128, "MMA N of the grouped kernel");
   static_assert(MAG0 + 2 * 64 <= kTmemCols, "tensor memory of the grouped kernel");
 };
 
@@ -81,7 +82,7 @@ __device__ void producer_grp(const ScoreParams &p, GrpSmem<G, HKV> &sm, int n_it
                              const WaitCtl wc) {
   using Cfg = GrpCfg<G, HKV>;
   constexpr int ST = Cfg::STAGES, BS = Cfg::BS;
-  const uint32_t kImg = (uint32_t)(HKV * p.geo.b_bytes);  // the (sequence, layer)'s image
+  constexpr uint32_t kImg = (uint32_t)Cfg::N * 512u;  // the (sequence, layer)'s image: N x 256 bf16
   const Geom &geo = p.geo;
   const uint64_t pol = evict_first_policy();
   const int W = geo.window, S = geo.sinks;
@@ -432,8 +433,12 @@ cudaError_t launch_grp_t(const ScoreParams &p, cudaStream_t st) {
 
 template <int G, int HKV>
 cudaError_t launch_grp_h(const ScoreParams &p, cudaStream_t st) {
-  if (p.geo.pairing == TRIA_PAIR_NEOX) return launch_grp_t<G, HKV, TRIA_PAIR_NEOX>(p, st);
-  return launch_grp_t<G, HKV, TRIA_PAIR_INTERLEAVED>(p, st);
+  if constexpr (2 * G * HKV < 16) {
+    return cudaErrorInvalidValue;  // N < 16: not selected by the geometry
+  } else {
+    if (p.geo.pairing == TRIA_PAIR_NEOX) return launch_grp_t<G, HKV, TRIA_PAIR_NEOX>(p, st);
+    return launch_grp_t<G, HKV, TRIA_PAIR_INTERLEAVED>(p, st);
+  }
 }
 
 template <int HKV>
