@@ -136,7 +136,7 @@ tria_status make_geom(const tria_stats *stats, const tria_cache_view *cache,
   g.ncol_n = g.ncol;
   if (g.mode == TRIA_OFFSET_MAX) {
     // the max-over-offsets kernel is built for G <= 8
-    if (g.g > 8 || g.n_off > 17 || 2 * g.n_off * g.g > kMaxOffCols) return TRIA_ERR_UNSUPPORTED;
+    if (g.g > 8 || g.n_off > kMaxOffsets || 2 * g.n_off * g.g > kMaxOffCols) return TRIA_ERR_UNSUPPORTED;
     // trig hi and lo parts (two 64-wide K blocks of 128-byte rows each), norm
     g.b_bytes = (2 * g.ncol_t + g.ncol_n) * 256;
   } else {
@@ -287,6 +287,7 @@ CoefParams make_coef(const tria_stats *st, const Geom &g, const tria_cache_view 
   cp.mu_raw = st->dev.mu_raw;
   cp.w_norm = st->dev.w_norm;
   cp.omega = st->dev.omega;
+  cp.rot_off = st->dev.rot_off;
   cp.query_pos = c->query_pos;
   cp.btile = at<uint16_t>(ws, wl.btile);
   cp.item_counter = at<uint32_t>(ws, wl.hdr);
@@ -424,14 +425,17 @@ tria_status tria_load_stats(const tria_model_desc *desc, const float *q_mean_re,
   const size_t n = (size_t)d.n_layers * d.n_q_heads * F;
   std::vector<double> omega(F);
   std::vector<double> wre(F), wim(F);
+  std::vector<double2> rot_off((size_t)F * kMaxOffsets, double2{0.0, 0.0});
   const int nd = d.offset_log2_max + 1;
   for (int f = 0; f < F; ++f) {
     omega[f] = std::pow(d.rope_theta, -2.0 * f / (double)d.head_dim);
     double sr = 0.0, si = 0.0;
     double delta = 1.0;
     for (int j = 0; j < nd; ++j) {
-      sr += std::cos(omega[f] * delta);
-      si += std::sin(omega[f] * delta);
+      const double c = std::cos(omega[f] * delta), sn = std::sin(omega[f] * delta);
+      sr += c;
+      si += sn;
+      if (j < kMaxOffsets) rot_off[(size_t)f * kMaxOffsets + j] = double2{c, sn};
       delta *= 2.0;
     }
     wre[f] = sr / nd;
@@ -462,11 +466,13 @@ tria_status tria_load_stats(const tria_model_desc *desc, const float *q_mean_re,
   if (cudaMalloc(&st->dev.mu_fold, n * sizeof(double2)) != cudaSuccess ||
       cudaMalloc(&st->dev.mu_raw, n * sizeof(double2)) != cudaSuccess ||
       cudaMalloc(&st->dev.w_norm, n * sizeof(double)) != cudaSuccess ||
-      cudaMalloc(&st->dev.omega, F * sizeof(double)) != cudaSuccess) {
+      cudaMalloc(&st->dev.omega, F * sizeof(double)) != cudaSuccess ||
+      cudaMalloc(&st->dev.rot_off, rot_off.size() * sizeof(double2)) != cudaSuccess) {
     cudaFree(st->dev.mu_fold);
     cudaFree(st->dev.mu_raw);
     cudaFree(st->dev.w_norm);
     cudaFree(st->dev.omega);
+    cudaFree(st->dev.rot_off);
     delete st;
     cudaGetLastError();
     return TRIA_ERR_OOM;
@@ -479,6 +485,9 @@ tria_status tria_load_stats(const tria_model_desc *desc, const float *q_mean_re,
     e = cudaMemcpyAsync(st->dev.w_norm, wn.data(), n * sizeof(double), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(st->dev.omega, omega.data(), F * sizeof(double), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(st->dev.rot_off, rot_off.data(), rot_off.size() * sizeof(double2),
+                        cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {
     tria_free_stats(st);
@@ -495,6 +504,7 @@ tria_status tria_free_stats(tria_stats *st) {
   cudaFree(st->dev.mu_raw);
   cudaFree(st->dev.w_norm);
   cudaFree(st->dev.omega);
+  cudaFree(st->dev.rot_off);
   delete st;
   return cuda_status(e);
 }

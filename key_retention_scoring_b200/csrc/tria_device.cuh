@@ -51,6 +51,13 @@ __device__ __forceinline__ void discard_line(const void *ptr) {
   asm volatile("discard.global.L2 [%0], 128;" ::"l"(ptr) : "memory");
 }
 
+// Maximum that returns NaN when either operand is NaN.
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
 // Order-preserving unsigned key of an fp32 score: larger score -> larger
 // key; -0.0 and +0.0 share a key; NaN gets the smallest key of all.
 __device__ __forceinline__ uint32_t order_key(float a) {

@@ -17,6 +17,7 @@ constexpr int kCoefK = 256;         // K extent of the coefficient tile: 128 key
 constexpr int kTileKeys = 1024;     // keys per scheduling item of the score kernel
 constexpr int kRowGroups = 4;       // moment partials per item: one per 32-row group of a tile
 constexpr int kMaxSeqTable = TRIA_MAX_SEQS + 1;
+constexpr int kMaxOffsets = 17;     // |D| bound of the max-over-offsets form
 
 // Device copy of the folded statistics.
 struct StatsDev {
@@ -25,6 +26,7 @@ struct StatsDev {
   double2 *mu_raw;    // [L][Hq][F]  E[q_f] mask_f (unfolded: the max-over-offsets form)
   double *w_norm;     // [L][Hq][F]  E|q_f| - |E q_f|            (fp64)
   double *omega;      // [F]         theta^(-2f/d)               (fp64)
+  double2 *rot_off;   // [F][kMaxOffsets] e^{i omega_f 2^j}, j < min(|D|, kMaxOffsets) (fp64)
 };
 
 // Per-call geometry.
@@ -140,6 +142,7 @@ struct CoefParams {
   const double2 *mu_raw;
   const double *w_norm;
   const double *omega;
+  const double2 *rot_off;
   const int64_t *query_pos;
   uint16_t *btile;
   uint32_t *item_counter;

@@ -44,6 +44,13 @@ __device__ __forceinline__ uint16_t bf16_rn_bits(float x) {
   return (uint16_t)(u >> 16);
 }
 
+// e^{i omega_f p} for a query position p (fp64).
+__device__ __forceinline__ double2 rot_at(const CoefParams &p, int f, int64_t pos) {
+  double sn, cs;
+  sincos(p.omega[f] * (double)pos, &sn, &cs);
+  return make_double2(cs, sn);
+}
+
 __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ CoefParams p) {
   const Geom &g = p.geo;
   const int t = threadIdx.x;
@@ -131,22 +138,28 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
 
   if (g.mode == TRIA_OFFSET_MAX) {
     // max over the offsets: one coefficient vector per (head, offset delta_j)
-    // with the unfolded center, c_gfj = E[q_gf] mask_f e^{i omega_f (p_q + delta_j)}
-    __shared__ double2 rotj[kBands][17];
+    // with the unfolded center, c_gfj = E[q_gf] mask_f e^{i omega_f (p_q + delta_j)};
+    // e^{i omega_f (p_q + 2^j)} = e^{i omega_f p_q} e^{i omega_f 2^j}, the
+    // second factor from the table built with the statistics.  Band f sits
+    // at f + f/8 in the shared tables so that the eight bands 8 apart that a
+    // warp reads together fall in different banks.
+    __shared__ double2 rotj[kMaxOffsets][kBands + kBands / 8];
+    __shared__ double2 mu_s[8][kBands + kBands / 8];  // the form takes G <= 8
     const int nd = g.n_off;
+    if (t < kBands) rot[t] = rot_at(p, t, p.query_pos[s]);
+    // the unit's E[q_g] mask per head and band (read 17 x 2 times per value below)
+    for (int i = t; i < g.g * kBands; i += kThreads) {
+      const int f = i % kBands;
+      mu_s[i / kBands][f + (f >> 3)] = p.mu_raw[((int64_t)l * g.hq + h * g.g) * kBands + i];
+    }
+    __syncthreads();
     for (int i = t; i < kBands * nd; i += kThreads) {
-      const int f = i / nd, j = i % nd;
-      double sn, cs;
-      sincos(p.omega[f] * ((double)p.query_pos[s] + (double)(1ll << j)), &sn, &cs);
-      rotj[f][j] = make_double2(cs, sn);
+      const int f = i % kBands, j = i / kBands;
+      const double2 a = rot[f], b = p.rot_off[f * kMaxOffsets + j];
+      rotj[j][f + (f >> 3)] = make_double2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
     }
     __syncthreads();
     unsigned char *dst = reinterpret_cast<unsigned char *>(p.btile) + u * (int64_t)g.b_bytes;
-    // the unit's E[q_g] mask per head and band (read 17 x 2 times per value below)
-    __shared__ double2 mu_s[TRIA_MAX_GROUP][kBands];
-    for (int i = t; i < g.g * kBands; i += kThreads)
-      mu_s[i / kBands][i % kBands] = p.mu_raw[((int64_t)l * g.hq + h * g.g) * kBands + i];
-    __syncthreads();
     // trig rows n = gg nd + j over the 128 key dims: the hi parts in two
     // 64-wide blocks, then the lo parts in two more (each value computed once)
     for (int i = t; i < g.ncol_t * 16; i += kThreads) {
@@ -161,8 +174,8 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
           if (gg < g.g) {
             const int f = (g.pairing == TRIA_PAIR_NEOX) ? (k & 63) : (k >> 1);
             const bool im = (g.pairing == TRIA_PAIR_NEOX) ? (k >= 64) : (k & 1);
-            const double2 mu = mu_s[gg][f];
-            const double2 r = rotj[f][j];
+            const double2 mu = mu_s[gg][f + (f >> 3)];
+            const double2 r = rotj[j][f + (f >> 3)];
             x = im ? (float)(mu.x * r.y + mu.y * r.x) : (float)(mu.x * r.x - mu.y * r.y);
           }
           h2[q2] = bf16_rn_bits(x);
@@ -202,11 +215,7 @@ __global__ void __launch_bounds__(kThreads) coef_kernel(const __grid_constant__ 
     return;
   }
 
-  if (t < kBands) {
-    double sn, cs;
-    sincos(p.omega[t] * (double)p.query_pos[s], &sn, &cs);
-    rot[t] = make_double2(cs, sn);
-  }
+  if (t < kBands) rot[t] = rot_at(p, t, p.query_pos[s]);
   __syncthreads();
   for (int i = t; i < g.g * kBands; i += kThreads) {
     const int gg = i / kBands, f = i % kBands;

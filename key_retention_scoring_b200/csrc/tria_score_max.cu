@@ -168,13 +168,6 @@ __device__ __forceinline__ void emit_scores(const ScoreParams &p, const EpRec &p
   }
 }
 
-// Maximum that returns NaN when either operand is NaN.
-__device__ __forceinline__ float max_nan(float a, float b) {
-  float d;
-  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
-  return d;
-}
-
 // Epilogue of tile j (buffer j & 1): per head of this thread's band group,
 // S = max_j trig_j + (norm hi + norm lo).
 template <int G>

@@ -100,14 +100,11 @@ __device__ void slice_keys(const float *raw, int P, const float *s_mean, const f
         const float z1 = __fmul_rn(__fsub_rn(x[u].y, m[1]), iv[1]);
         const float z2 = __fmul_rn(__fsub_rn(x[u].z, m[2]), iv[2]);
         const float z3 = __fmul_rn(__fsub_rn(x[u].w, m[3]), iv[3]);
-        int nan = (z0 != z0) | (z1 != z1) | (z2 != z2) | (z3 != z3);
-        float a = fmaxf(fmaxf(z0, z1), fmaxf(z2, z3));
+        // NaN in any head makes agg NaN, whose key is 0
+        float a = max_nan(max_nan(z0, z1), max_nan(z2, z3));
 #pragma unroll
-        for (int o = 1; o < LPC; o <<= 1) {
-          a = fmaxf(a, __shfl_xor_sync(kFull, a, o));
-          nan |= __shfl_xor_sync(kFull, nan, o);
-        }
-        const uint32_t k = nan ? 0u : order_key(a);
+        for (int o = 1; o < LPC; o <<= 1) a = max_nan(a, __shfl_xor_sync(kFull, a, o));
+        const uint32_t k = order_key(a);
         const bool lead = (j < n4) && (tid % LPC) == 0;
         if (lead) keys[key_word<KPT>(j / LPC)] = k;
         hist_add(hist, k >> 20, lead);
@@ -138,14 +135,12 @@ __device__ void slice_keys(const float *raw, int P, const float *s_mean, const f
         for (int e = 0; e < CPF; ++e) {
           const int c = j * CPF + e;
           float a = 0.0f;
-          int nan = 0;
 #pragma unroll
           for (int g = 0; g < G; ++g) {
             const float z = __fmul_rn(__fsub_rn(v[e * G + g], m[g]), iv[g]);
-            a = (g == 0) ? z : fmaxf(a, z);
-            nan |= (z != z);
+            a = (g == 0) ? z : max_nan(a, z);
           }
-          const uint32_t k = nan ? 0u : order_key(a);
+          const uint32_t k = order_key(a);
           const bool in = (j < n4) && c < P;
           if (in) keys[key_word<KPT>(c)] = k;
           hist_add(hist, k >> 20, in);
