@@ -67,6 +67,15 @@ __device__ __forceinline__ int key_word(int c) {
   return chunk_word<KPT>(c / KPT, (c % KPT) >> 2) + (c & 3);
 }
 
+// Eight consecutive floats from a 32-byte-aligned address with one 256-bit
+// streaming load (read once: evict first).
+__device__ __forceinline__ void ld_cs_v8(const float *p, float (&x)[8]) {
+  asm volatile("ld.global.cs.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=f"(x[0]), "=f"(x[1]), "=f"(x[2]), "=f"(x[3]), "=f"(x[4]), "=f"(x[5]),
+                 "=f"(x[6]), "=f"(x[7])
+               : "l"(p));
+}
+
 // Raw-score pass over a slice of P candidates: keys (order keys of agg) into
 // the rotated layout and the histogram of their top 12 bits.
 template <int G, int KPT>
@@ -75,7 +84,48 @@ __device__ void slice_keys(const float *raw, int P, const float *s_mean, const f
   constexpr int NT = kTailThreads;
   constexpr int U = 8;  // float4 loads in flight per thread
   const float4 *src = reinterpret_cast<const float4 *>(raw);
-  if constexpr (G >= 4) {
+  if constexpr (G >= 8) {
+    // LPC lanes per candidate, each loading 8 of its G heads with one
+    // 256-bit load (the slice starts on a 32-byte boundary: checked at launch)
+    constexpr int LPC = G / 8, U8 = 4;
+    const int h0 = (tid % LPC) * 8;
+    float m[8], iv[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      m[k] = s_mean[h0 + k];
+      iv[k] = s_inv[h0 + k];
+    }
+    const int n8 = P * LPC;
+    for (int j0 = 0; j0 < n8; j0 += NT * U8) {
+      float x[U8][8];
+#pragma unroll
+      for (int u = 0; u < U8; ++u) {
+        const int j = j0 + u * NT + tid;
+        if (j < n8) {
+          ld_cs_v8(raw + (int64_t)j * 8, x[u]);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) x[u][k] = 0.0f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U8; ++u) {
+        const int j = j0 + u * NT + tid;
+        float z[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) z[k] = __fmul_rn(__fsub_rn(x[u][k], m[k]), iv[k]);
+        // NaN in any head makes agg NaN, whose key is 0
+        float a = max_nan(max_nan(max_nan(z[0], z[1]), max_nan(z[2], z[3])),
+                          max_nan(max_nan(z[4], z[5]), max_nan(z[6], z[7])));
+#pragma unroll
+        for (int o = 1; o < LPC; o <<= 1) a = max_nan(a, __shfl_xor_sync(kFull, a, o));
+        const uint32_t k = order_key(a);
+        const bool lead = (j < n8) && (tid % LPC) == 0;
+        if (lead) keys[key_word<KPT>(j / LPC)] = k;
+        hist_add(hist, k >> 20, lead);
+      }
+    }
+  } else if constexpr (G >= 4) {
     // LPC lanes per candidate, each with 4 of its G heads
     constexpr int LPC = G / 4;
     const int h0 = (tid % LPC) * 4;
@@ -449,6 +499,10 @@ bool unit_tail_fits(const Geom &g) {
 
 cudaError_t launch_unit_tail(const TailParams &p0, cudaStream_t st) {
   TailParams p = p0;
+  // G >= 8 reads a candidate's heads in 32-byte pieces: the raw scores of
+  // every unit start on a 32-byte boundary (workspace layout)
+  if (p.geo.g >= 8 && ((reinterpret_cast<uintptr_t>(p.raw) & 31u) != 0 || (p.raw_stride & 7) != 0))
+    return cudaErrorInvalidValue;
   int kpt = 0;
   if (!tail_shape(p.geo, &p.cluster, &p.slice, &kpt)) return cudaErrorInvalidValue;
   const size_t smem = tail_smem_bytes(kpt);
