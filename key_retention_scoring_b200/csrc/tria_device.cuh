@@ -58,6 +58,13 @@ __device__ __forceinline__ float max_nan(float a, float b) {
   return d;
 }
 
+// Maximum of three that returns NaN when any operand is NaN (one instruction).
+__device__ __forceinline__ float max3_nan(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Order-preserving unsigned key of an fp32 score: larger score -> larger
 // key; -0.0 and +0.0 share a key; NaN gets the smallest key of all.
 __device__ __forceinline__ uint32_t order_key(float a) {

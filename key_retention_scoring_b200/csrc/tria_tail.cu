@@ -115,8 +115,7 @@ __device__ void slice_keys(const float *raw, int P, const float *s_mean, const f
 #pragma unroll
         for (int k = 0; k < 8; ++k) z[k] = __fmul_rn(__fsub_rn(x[u][k], m[k]), iv[k]);
         // NaN in any head makes agg NaN, whose key is 0
-        float a = max_nan(max_nan(max_nan(z[0], z[1]), max_nan(z[2], z[3])),
-                          max_nan(max_nan(z[4], z[5]), max_nan(z[6], z[7])));
+        float a = max3_nan(max3_nan(z[0], z[1], z[2]), max3_nan(z[3], z[4], z[5]), max_nan(z[6], z[7]));
 #pragma unroll
         for (int o = 1; o < LPC; o <<= 1) a = max_nan(a, __shfl_xor_sync(kFull, a, o));
         const uint32_t k = order_key(a);

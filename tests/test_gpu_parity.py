@@ -266,6 +266,43 @@ def test_cluster_tail_ties_across_blocks():
         torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("shape", ["gqa8", "gqa16"])
+def test_nan_key_row_poisons_its_unit(shape):
+    # one candidate row holding NaN (every dim in unit h = 0, one dim in unit
+    # h = 1) scores NaN for every head; the unit's moments, and so every agg
+    # of the unit, are NaN (the oracle's mean propagates it too).  All keys tie
+    # at the lowest rank: both the fused pass (raw scores -> unit tail) and
+    # score + select keep the K lowest candidate slots; other units are as usual
+    if shape == "gqa8":
+        cfg = synth.CONFIGS[2].scaled(n_layers=1, seq_len=5133)
+    else:
+        cfg = synth.CONFIGS[0].scaled(n_q_heads=32, n_kv_heads=2, seq_len=3000)
+    w = synth.Workload(cfg)
+    st = load_stats(w)
+    try:
+        N, W, S, B = cfg.seq_len, cfg.window, cfg.sinks, cfg.budget
+        C, K = N - W - S, B - W - S
+        k = w.k[0]
+        k[0, 0, S + C // 3] = float("nan")
+        k[0, 1, S + 2 * C // 3, 37] = float("nan")
+        oras = [PH.unit_oracle(w, 0, 0, h) for h in range(2)]
+        agg, _, kept_sep = score_layers(w, st, 0, 1, want_scores=False)
+        want = np.concatenate([np.arange(S), np.arange(S, S + K), np.arange(N - W, N)])
+        for h in range(2):
+            assert np.all(np.isnan(agg[0, 0, h, :C])), f"h{h}: agg not NaN"
+            assert np.array_equal(kept_sep[0, 0, h], want), f"h{h}"
+            PH.check_kept_vs_oracle(kept_sep[0, 0, h], oras[h], cfg, f"h{h} oracle")
+        for h in range(2, cfg.n_kv_heads):
+            PH.check_kept_same_precision(kept_sep[0, 0, h], agg[0, 0, h, :C], N, cfg, f"h{h}")
+        kept_all, _, _ = compress(w, st)
+        for h in range(cfg.n_kv_heads):
+            assert np.array_equal(kept_all[0, 0, h], kept_sep[0, 0, h]), f"h{h}"
+    finally:
+        st.free()
+        del w
+        torch.cuda.empty_cache()
+
+
 # ---------------------------------------------------------------------------
 # multi-pass: positions are no longer slot indices after compaction
 # ---------------------------------------------------------------------------
