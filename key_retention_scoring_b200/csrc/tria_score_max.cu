@@ -189,6 +189,28 @@ __device__ __forceinline__ void epilogue_max(const ScoreParams &p, uint32_t tmem
     // load (offsets 0..15; past nd it reads the next head's columns, unused)
     // and, at nd = 17, a 2-column load for offset 16 (its second column unused)
     constexpr int HP = (GQ >= 2) ? 2 : 1;
+    if (GQ >= 2 && nd == kMaxOffsets) {
+      // |D| = 17: a head pair's 34 trig columns are adjacent (one 32-column
+      // and one 2-column load) and so are its 4 norm columns (one load)
+#pragma unroll
+      for (int g0 = 0; g0 < GQ; g0 += 2) {
+        uint32_t t[32], t2[2], nv[4];
+        const int g = q * GQ + g0;
+        const uint32_t c0 = tb + (uint32_t)(g * kMaxOffsets);
+        tmem_ld_nowait<32>(c0, t);
+        tmem_ld_nowait<2>(c0 + 32, t2);
+        tmem_ld_nowait<4>(nb + (uint32_t)(2 * g), nv);
+        tmem_wait_ld();
+        float m0 = __uint_as_float(t[0]), m1 = __uint_as_float(t[17]);
+#pragma unroll
+        for (int j = 1; j < 17; ++j) m0 = max_nan(m0, __uint_as_float(t[j]));
+#pragma unroll
+        for (int j = 18; j < 32; ++j) m1 = max_nan(m1, __uint_as_float(t[j]));
+        m1 = max_nan(m1, max_nan(__uint_as_float(t2[0]), __uint_as_float(t2[1])));
+        sc[g0] = m0 + (__uint_as_float(nv[0]) + __uint_as_float(nv[1]));
+        sc[g0 + 1] = m1 + (__uint_as_float(nv[2]) + __uint_as_float(nv[3]));
+      }
+    } else {
 #pragma unroll
     for (int g0 = 0; g0 < GQ; g0 += HP) {
       uint32_t t[HP][16], t16[HP][2], nv[HP][2];
@@ -217,6 +239,7 @@ __device__ __forceinline__ void epilogue_max(const ScoreParams &p, uint32_t tmem
         const float m = max_nan(__uint_as_float(t[a][0]), v16);
         sc[g0 + a] = m + (__uint_as_float(nv[a][0]) + __uint_as_float(nv[a][1]));
       }
+    }
     }
   } else {
 #pragma unroll
