@@ -63,7 +63,7 @@ typedef enum {
   TRIA_OK = 0,
   TRIA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or range */
   TRIA_ERR_UNSUPPORTED = 2, /* valid but not built: head_dim != 128, G > 16 */
-  TRIA_ERR_WORKSPACE = 3,   /* workspace null or smaller than required */
+  TRIA_ERR_WORKSPACE = 3,   /* workspace null, not 256-byte aligned, or smaller than required */
   TRIA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
   TRIA_ERR_OOM = 5,         /* device allocation failed (tria_load_stats) */
   TRIA_ERR_IO = 6           /* a stats file could not be opened, read or written,
@@ -274,7 +274,9 @@ tria_status tria_layer_budgets(const tria_stats *stats, const tria_cache_view *c
  * tria_workspace_size - device workspace bytes that tria_score, tria_select
  * and tria_compress_pass need for this cache view, these parameters and the
  * layer range [layer0, layer1).  The workspace is scratch: no state is kept
- * between calls, and concurrent calls need separate workspaces.
+ * between calls, and concurrent calls need separate workspaces.  Its base
+ * must be 256-byte aligned (cudaMalloc's are); the entry points that take it
+ * return TRIA_ERR_WORKSPACE otherwise.
  * Errors: INVALID_ARG.
  */
 tria_status tria_workspace_size(const tria_stats *stats, const tria_cache_view *cache,
