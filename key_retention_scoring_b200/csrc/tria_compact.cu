@@ -32,16 +32,16 @@ constexpr int kPieces = kRowBytes / 16;                   // 16-byte pieces per 
 constexpr int kMinBlock = 8;                              // smallest paged block size
 
 // Block shape per layout.  Contiguous: one block of 512 threads per SM with
-// 256-row chunks.  Paged: two blocks of 256 threads per SM with 128-row
+// 256-row chunks.  Paged: four blocks of 128 threads per SM with 64-row
 // chunks (the same bytes in flight per SM; its row addresses need block-table
-// entries, and two independent blocks hide that better: 2044 -> 1901 us per
-// 8-layer paged batch, while the contiguous pass measured 215 -> 234 us with
-// that shape).
+// entries, and independent blocks hide that better: per 8-layer paged batch
+// 2041 us with one block, 1903 with two of 256 threads and 128-row chunks,
+// 1820 with four; the contiguous pass measured 215 -> 234 us with two).
 template <bool PAGED>
 struct CpCfg {
-  static constexpr int THREADS = PAGED ? 256 : 512;
-  static constexpr int ROWS = PAGED ? 128 : 256;          // destination rows per chunk
-  static constexpr int BPS = PAGED ? 2 : 1;               // blocks per SM
+  static constexpr int THREADS = PAGED ? 128 : 512;
+  static constexpr int ROWS = PAGED ? 64 : 256;           // destination rows per chunk
+  static constexpr int BPS = PAGED ? 4 : 1;               // blocks per SM
   static constexpr int ROW_STEP = THREADS / kPieces;      // rows covered by one pass of the block
   static constexpr int ROWS_PER_THREAD = ROWS / ROW_STEP;  // 8
 };
@@ -207,7 +207,9 @@ __global__ void __launch_bounds__(CpCfg<PAGED>::THREADS, CpCfg<PAGED>::BPS)
       const ItemGeo g = item_geo(p, item_of(q.i));
       if constexpr (paged) {
         // the chunk's destination blocks, for its write-back two iterations on
-        const int nb = kCpRows >> bsh, b0 = (q.c * kCpRows) >> bsh;
+        // destination blocks of the chunk: one when a block holds more rows
+        // than a chunk (the chunk's rows are then all in block b0)
+        const int nb = max(1, kCpRows >> bsh), b0 = (q.c * kCpRows) >> bsh;
         if (t < nb)
           sm.dblk[b][t] = (b0 + t < p.cache.max_blocks)
                               ? __ldg(p.cache.block_table + (int64_t)g.s * p.cache.max_blocks + b0 + t)

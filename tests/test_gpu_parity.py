@@ -194,6 +194,15 @@ def test_paged_noop_and_minimal_units():
     full_check(base.scaled(budget=260))
 
 
+@pytest.mark.parametrize("block_size", [8, 64, 128])
+def test_paged_block_sizes(block_size):
+    # paged blocks smaller and larger than the scoring tile's slot groups and
+    # the compaction's chunks (a 128-token block spans two 64-row chunks)
+    cfg = synth.CONFIGS[3].scaled(n_layers=1, n_seq=3, len_range=(2300, 5000),
+                                  block_size=block_size)
+    full_check(cfg)
+
+
 def test_long_context_small_nearzero_heads():
     cfg = synth.CONFIGS[4].scaled(n_layers=2, seq_len=14000, near_zero_frac=0.5)
     full_check(cfg)
