@@ -1,6 +1,6 @@
 // Unit tail of the compression pass: normalize-then-max and top-K selection
 // with the candidates' agg keys in shared memory, one thread-block cluster of
-// 1, 2, 4 or 8 blocks per unit (sequence, layer, KV head).
+// 1 to 8 blocks per unit (sequence, layer, KV head).
 //
 // Per unit (academ.us article 2607.13051, Eq. 8 and sec. 4; ghidav.me
 // "TriAttention, or: what a rotating query already knows", "The Method"):
@@ -43,13 +43,13 @@ constexpr int kTailWarps = kTailThreads / 32;
 struct alignas(16) TailShared {
   float mean[TRIA_MAX_GROUP];
   float inv[TRIA_MAX_GROUP];
-  int wsum[kTailWarps];  // per-warp totals / exclusive prefixes of the block scans
+  uint32_t wsum[kTailWarps];  // per-warp totals / exclusive prefixes of the block scans
   uint32_t prefix;       // digits of T fixed so far
   int remaining;         // rank of T among the keys matching prefix
   int digit, above;
   int cta_gt, cta_eq;    // this block's keys > T and == T (read by the cluster)
   int pre_gt, pre_eq;    // the same summed over the cluster's lower blocks
-  int total;             // block sum of the last scan
+  uint32_t total;        // block sum of the last scan
   int pad[3];
 };
 static_assert(sizeof(TailShared) % 16 == 0, "the histogram after TailShared stays 16-byte aligned");
@@ -199,22 +199,38 @@ __device__ void slice_keys(const float *raw, int P, const float *s_mean, const f
   }
 }
 
-// Block-wide exclusive scan (warp scans, then warp 0 over the warp totals);
-// returns this thread's exclusive prefix, sc.total the block's sum.  Starts
-// and ends with a barrier-separated use of sc.wsum.
-__device__ __forceinline__ int tail_excl_scan(int v, TailShared &sc, int tid) {
+// Block-wide exclusive scan (warp scans, then warp 0 over the warp totals) of
+// non-negative counts, in unsigned 32-bit arithmetic; returns this thread's
+// exclusive prefix, sc.total the block's sum.  Starts and ends with a
+// barrier-separated use of sc.wsum.
+__device__ __forceinline__ uint32_t tail_excl_scan_u(uint32_t v, TailShared &sc, int tid) {
   const int lane = tid & 31, warp = tid >> 5;
-  const int incl = warp_incl_scan(v, lane);
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += y;
+  }
   if (lane == 31) sc.wsum[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const int x = sc.wsum[lane];
-    const int xi = warp_incl_scan(x, lane);
+    const uint32_t x = sc.wsum[lane];
+    uint32_t xi = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(kFull, xi, o);
+      if (lane >= o) xi += y;
+    }
     sc.wsum[lane] = xi - x;  // each lane reads and writes its own entry
     if (lane == 31) sc.total = xi;
   }
   __syncthreads();
   return sc.wsum[warp] + incl - v;
+}
+
+// The same for int counts (a block's sum stays below 2^31).
+__device__ __forceinline__ int tail_excl_scan(int v, TailShared &sc, int tid) {
+  return (int)tail_excl_scan_u((uint32_t)v, sc, tid);
 }
 
 // The bin holding the sc.remaining-th largest key among hist[0, nbins)
@@ -380,10 +396,14 @@ __global__ void __launch_bounds__(kTailThreads, 1) cluster_tail_kernel(const __g
       eq += (valid && kk[i] == T) ? 1 : 0;
     }
   }
-  const int ex = tail_excl_scan(gt | (eq << 16), sc, t);
+  // gt and eq packed in the low and high halves of one unsigned word: a
+  // block holds at most kTailThreads x 44 = 45056 < 2^16 candidates, so
+  // neither half overflows (a signed word would, past 32767 ties)
+  static_assert(kTailThreads * 44 < (1 << 16), "packed block counts");
+  const uint32_t ex = tail_excl_scan_u((uint32_t)gt | ((uint32_t)eq << 16), sc, t);
   if (t == 0) {
-    sc.cta_gt = sc.total & 0xffff;
-    sc.cta_eq = sc.total >> 16;
+    sc.cta_gt = (int)(sc.total & 0xffffu);
+    sc.cta_eq = (int)(sc.total >> 16);
     sc.pre_gt = 0;
     sc.pre_eq = 0;
   }
@@ -405,8 +425,8 @@ __global__ void __launch_bounds__(kTailThreads, 1) cluster_tail_kernel(const __g
     __syncthreads();
   }
   // emission in slot order
-  int eqr = sc.pre_eq + (ex >> 16);
-  int pos = sc.pre_gt + (ex & 0xffff) + min(eqr, need);
+  int eqr = sc.pre_eq + (int)(ex >> 16);
+  int pos = sc.pre_gt + (int)(ex & 0xffffu) + min(eqr, need);
   const int slot0 = S + c0 + cb;
   for (int q = 0; q < NQ; ++q) {
     const uint4 k4 = *reinterpret_cast<const uint4 *>(keys + chunk_word<KPT>(t, q));
@@ -475,10 +495,10 @@ cudaError_t launch_ct_g(const TailParams &p, int kpt, size_t smem, cudaStream_t 
 
 }  // namespace
 
-// The smallest cluster (1, 2, 4 or 8 blocks) whose slices of at most
+// The smallest cluster (1 to 8 blocks) whose slices of at most
 // ceil(c_max / cs) candidates, rounded up to 128, fit a block's key area.
 bool tail_shape(const Geom &g, int *cs, int *slice, int *kpt) {
-  for (int c = 1; c <= kMaxTailCluster; c *= 2) {
+  for (int c = 1; c <= kMaxTailCluster; ++c) {
     const int sl = ((g.c_max + c - 1) / c + 127) / 128 * 128;
     const int k = tail_kpt(sl);
     if (k != 0 && tail_smem_bytes(k) <= kMaxDynSmem) {

@@ -229,9 +229,10 @@ def test_offset_sets_and_theta():
 
 # ---------------------------------------------------------------------------
 # long units: the pass's unit tail splits a unit's candidates over a cluster of
-# 2, 4 or 8 blocks (more than 45056 candidates per unit)
+# up to 8 blocks (more than 32768 candidates per unit take 2 blocks or more;
+# a block holds at most 45056)
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("seq_len", [60000, 100000, 200000], ids=["2blocks", "4blocks", "8blocks"])
+@pytest.mark.parametrize("seq_len", [60000, 100000, 200000], ids=["2blocks", "3blocks", "5blocks"])
 def test_cluster_tail_long_units(seq_len):
     cfg = synth.CONFIGS[4].scaled(n_layers=1, n_q_heads=16, n_kv_heads=2, seq_len=seq_len)
     full_check(cfg)
@@ -245,11 +246,39 @@ def test_cluster_tail_ragged_lengths_paged():
     full_check(cfg)
 
 
+def test_ties_past_32767_in_one_block():
+    # one block of 44 keys per thread (32768 < C <= 45056) with every candidate
+    # of unit h = 1 equal: all C keys tie at T, more than 2^15 of them in the
+    # block (its tie count is packed in 16 bits of an unsigned word), and the
+    # K lowest slots are kept.  Unit h = 0, whose kept row lies just before,
+    # must come out as its own selection: no write strays outside a unit's row
+    cfg = synth.CONFIGS[2].scaled(n_layers=1, n_q_heads=16, n_kv_heads=2, seq_len=40000)
+    w = synth.Workload(cfg)
+    st = load_stats(w)
+    try:
+        N, W, S, B = cfg.seq_len, cfg.window, cfg.sinks, cfg.budget
+        C, K = N - W - S, B - W - S
+        assert 32768 < C <= 45056
+        k = w.k[0]
+        k[0, 1, S:N - W] = k[0, 1, S:S + 1]
+        agg, _, kept_sep = score_layers(w, st, 0, 1, want_scores=False)
+        want1 = np.concatenate([np.arange(S), np.arange(S, S + K), np.arange(N - W, N)])
+        assert np.array_equal(kept_sep[0, 0, 1], want1)
+        PH.check_kept_same_precision(kept_sep[0, 0, 0], agg[0, 0, 0, :C], N, cfg, "h0")
+        kept_all, _, _ = compress(w, st)
+        for h in range(2):
+            assert np.array_equal(kept_all[0, 0, h], kept_sep[0, 0, h]), f"h{h}"
+    finally:
+        st.free()
+        del w
+        torch.cuda.empty_cache()
+
+
 def test_cluster_tail_ties_across_blocks():
     # unit h = 0: every candidate row equal, so every agg is equal and the K
     # lowest slots are kept; unit h = 1: rows repeat with period 3, so the
     # threshold falls on a value held by about C / 3 keys in every block of the
-    # cluster (four blocks), and the kept ties run into the second block
+    # cluster (three blocks), and the kept ties run into the second block
     cfg = synth.CONFIGS[4].scaled(n_layers=1, n_q_heads=16, n_kv_heads=2, seq_len=100000)
     w = synth.Workload(cfg)
     st = load_stats(w)
