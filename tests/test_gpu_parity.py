@@ -246,6 +246,16 @@ def test_cluster_tail_ragged_lengths_paged():
     full_check(cfg)
 
 
+@pytest.mark.parametrize("C", [32768, 32769, 45056, 45057])
+def test_tail_sizing_boundaries(C):
+    # candidate counts at the unit tail's sizing limits: 32 keys per thread
+    # exactly full (32768), the first 44-keys-per-thread unit (32769), one
+    # block exactly full (45056), and the first cluster of 2 (45057: slices
+    # of 22656 and 22401 candidates)
+    cfg = synth.CONFIGS[2].scaled(n_layers=1, n_q_heads=16, n_kv_heads=2, seq_len=C + 256)
+    full_check(cfg)
+
+
 def test_ties_past_32767_in_one_block():
     # one block of 44 keys per thread (32768 < C <= 45056) with every candidate
     # of unit h = 1 equal: all C keys tie at T, more than 2^15 of them in the
