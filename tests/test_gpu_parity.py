@@ -222,6 +222,22 @@ def test_gqa16():
     full_check(synth.CONFIGS[4].scaled(n_layers=1, n_q_heads=16, n_kv_heads=1, seq_len=50000))
 
 
+def test_units_of_one_partial_tile():
+    # fewer than 128 candidates (one ragged scoring tile), K close to C, with
+    # and without sinks, both pairings
+    full_check(synth.CONFIGS[0].scaled(seq_len=300, budget=290, window=256))
+    full_check(synth.CONFIGS[0].scaled(seq_len=200, budget=190, window=64, sinks=5,
+                                       pairing=synth.PAIR_INTERLEAVED))
+    full_check(synth.CONFIGS[0].scaled(seq_len=130, budget=2, window=1, sinks=0))
+
+
+def test_paged_gqa16():
+    # G = 16 on a paged cache (Hkv x block size = 32 rows: the one-head scoring
+    # kernel; four lanes per candidate in the unit tail)
+    full_check(synth.CONFIGS[3].scaled(n_layers=1, n_q_heads=32, n_kv_heads=2, n_seq=3,
+                                       len_range=(2300, 4000)))
+
+
 def test_offset_sets_and_theta():
     for m in (0, 7, 12):
         full_check(synth.CONFIGS[0].scaled(offset_log2_max=m, seq_len=1800, theta=5e5))
