@@ -580,6 +580,15 @@ def test_offset_max_eight_offsets():
     full_check(cfg, units=units, offset_reduce=T.OFFSET_MAX)
 
 
+@pytest.mark.parametrize("m", [0, 15], ids=["one_offset", "sixteen_offsets"])
+def test_offset_max_offset_count_limits(m):
+    # |D| = 1 (every offset column past the first masked) and |D| = 16 (none
+    # masked, no 17th column)
+    cfg = synth.CONFIGS[2].scaled(n_layers=1, seq_len=3000, offset_log2_max=m)
+    units = [(0, 0, h) for h in (0, 5)]
+    full_check(cfg, units=units, offset_reduce=T.OFFSET_MAX)
+
+
 def test_offset_max_unsupported_shapes():
     cfg = synth.CONFIGS[0].scaled(n_q_heads=32, n_kv_heads=2)  # G = 16
     w = synth.Workload(cfg, with_values=False, with_positions=False)
