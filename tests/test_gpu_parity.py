@@ -231,6 +231,17 @@ def test_units_of_one_partial_tile():
     full_check(synth.CONFIGS[0].scaled(seq_len=130, budget=2, window=1, sinks=0))
 
 
+@pytest.mark.parametrize("hkv,bs,hq", [(4, 32, 32), (2, 64, 8), (2, 64, 16), (8, 16, 16)],
+                         ids=["hkv4_bs32_g8", "hkv2_bs64_g4", "hkv2_bs64_g8", "hkv8_bs16_g2"])
+def test_paged_whole_block_shapes(hkv, bs, hq):
+    # whole-block paged scoring (Hkv x block size = 128 rows per tile): a head
+    # fills one warp (32-token blocks), two warps (64), or shares a warp with
+    # another head (16), with 2G columns per head
+    cfg = synth.CONFIGS[3].scaled(n_layers=1, n_q_heads=hq, n_kv_heads=hkv, block_size=bs,
+                                  n_seq=3, len_range=(2300, 4500))
+    full_check(cfg)
+
+
 def test_paged_gqa16():
     # G = 16 on a paged cache (Hkv x block size = 32 rows: the one-head scoring
     # kernel; four lanes per candidate in the unit tail)
