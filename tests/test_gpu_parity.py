@@ -187,6 +187,14 @@ def test_llama3_paged_small_interleaved_sinks():
     full_check(cfg)
 
 
+def test_contiguous_batch_of_mixed_lengths():
+    # a contiguous cache of several sequences of different lengths, some at or
+    # below the budget (left as they are) and some compressed
+    cfg = synth.CONFIGS[2].scaled(n_layers=2, n_q_heads=32, n_seq=5, seq_len=0,
+                                  len_range=(1200, 7000))
+    full_check(cfg)
+
+
 def test_paged_noop_and_minimal_units():
     # N <= budget (no-op), N = budget + 1, budget = window + sinks (K = 0)
     base = synth.CONFIGS[3].scaled(n_layers=1, n_seq=3, len_range=(2040, 2060))
