@@ -273,6 +273,14 @@ def test_cluster_tail_long_units(seq_len):
     full_check(cfg)
 
 
+def test_pass_units_past_the_cluster_tail():
+    # more than 8 x 45056 candidates per unit: the pass selects with the
+    # chunked tail over global agg (workspace histogram) instead of a cluster
+    cfg = synth.CONFIGS[4].scaled(n_layers=1, n_q_heads=16, n_kv_heads=2, seq_len=370000)
+    assert cfg.seq_len - cfg.window - cfg.sinks > 8 * 45056
+    full_check(cfg)
+
+
 def test_cluster_tail_ragged_lengths_paged():
     # lengths per sequence from 20000 to 120000: the cluster is sized for the
     # longest, so the shorter units leave their trailing blocks without candidates
