@@ -46,11 +46,10 @@ struct alignas(16) TailShared {
   uint32_t wsum[kTailWarps];  // per-warp totals / exclusive prefixes of the block scans
   uint32_t prefix;       // digits of T fixed so far
   int remaining;         // rank of T among the keys matching prefix
-  int digit, above;
   int cta_gt, cta_eq;    // this block's keys > T and == T (read by the cluster)
   int pre_gt, pre_eq;    // the same summed over the cluster's lower blocks
   uint32_t total;        // block sum of the last scan
-  int pad[3];
+  int pad[1];
 };
 static_assert(sizeof(TailShared) % 16 == 0, "the histogram after TailShared stays 16-byte aligned");
 
@@ -244,23 +243,19 @@ __device__ void pick_bin_desc(const uint32_t *hist, int nbins, TailShared &sc, i
   int v = 0;
   if (first < nbins)
     for (int e = 0; e < per; ++e) v += (int)hist[nbins - 1 - (first + e)];
-  const int rem = sc.remaining;
+  const int rem = sc.remaining;  // read by every thread before the scan's barriers
   int cum = tail_excl_scan(v, sc, tid);
   if (v > 0 && cum < rem && rem <= cum + v) {
+    // the one thread whose bins hold the rank: it alone updates the state
     for (int e = 0; e < per; ++e) {
       const int d = nbins - 1 - (first + e);
       const int c = (int)hist[d];
       if (cum < rem && rem <= cum + c) {
-        sc.digit = d;
-        sc.above = cum;
+        sc.prefix |= (uint32_t)d << shift;
+        sc.remaining = rem - cum;
       }
       cum += c;
     }
-  }
-  __syncthreads();
-  if (tid == 0) {
-    sc.prefix |= (uint32_t)sc.digit << shift;
-    sc.remaining = rem - sc.above;
   }
   __syncthreads();
 }
@@ -357,12 +352,18 @@ __global__ void __launch_bounds__(kTailThreads, 1) cluster_tail_kernel(const __g
   __syncthreads();
   {
     const uint32_t d1 = sc.prefix >> 20;
-    for (int q = 0; q < NQ; ++q) {
+    auto keys_q1 = [&](int q) {
       const uint4 k4 = *reinterpret_cast<const uint4 *>(keys + chunk_word<KPT>(t, q));
       const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         if (4 * q + i < nmine && (kk[i] >> 20) == d1) atomicAdd(hist + ((kk[i] >> 8) & 0xfffu), 1u);
+    };
+    if (nmine == KPT) {
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) keys_q1(q);
+    } else {
+      for (int q = 0; 4 * q < nmine; ++q) keys_q1(q);
     }
   }
   cluster_sum_hist(hist, kHistBins, cs, t);
@@ -372,12 +373,18 @@ __global__ void __launch_bounds__(kTailThreads, 1) cluster_tail_kernel(const __g
   __syncthreads();
   {
     const uint32_t d12 = sc.prefix >> 8;
-    for (int q = 0; q < NQ; ++q) {
+    auto keys_q2 = [&](int q) {
       const uint4 k4 = *reinterpret_cast<const uint4 *>(keys + chunk_word<KPT>(t, q));
       const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         if (4 * q + i < nmine && (kk[i] >> 8) == d12) atomicAdd(hist + (kk[i] & 0xffu), 1u);
+    };
+    if (nmine == KPT) {
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) keys_q2(q);
+    } else {
+      for (int q = 0; 4 * q < nmine; ++q) keys_q2(q);
     }
   }
   cluster_sum_hist(hist, 256, cs, t);
@@ -386,7 +393,7 @@ __global__ void __launch_bounds__(kTailThreads, 1) cluster_tail_kernel(const __g
   const int need = sc.remaining;  // keys equal to T to keep, lowest slots first (>= 1)
   // this thread's keys above / equal to T; block prefixes (counts < 2^16 per block)
   int gt = 0, eq = 0;
-  for (int q = 0; q < NQ; ++q) {
+  auto keys_q3 = [&](int q) {
     const uint4 k4 = *reinterpret_cast<const uint4 *>(keys + chunk_word<KPT>(t, q));
     const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
@@ -395,6 +402,12 @@ __global__ void __launch_bounds__(kTailThreads, 1) cluster_tail_kernel(const __g
       gt += (valid && kk[i] > T) ? 1 : 0;
       eq += (valid && kk[i] == T) ? 1 : 0;
     }
+  };
+  if (nmine == KPT) {
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) keys_q3(q);
+  } else {
+    for (int q = 0; 4 * q < nmine; ++q) keys_q3(q);
   }
   // gt and eq packed in the low and high halves of one unsigned word: a
   // block holds at most kTailThreads x 44 = 45056 < 2^16 candidates, so
@@ -428,7 +441,7 @@ __global__ void __launch_bounds__(kTailThreads, 1) cluster_tail_kernel(const __g
   int eqr = sc.pre_eq + (int)(ex >> 16);
   int pos = sc.pre_gt + (int)(ex & 0xffffu) + min(eqr, need);
   const int slot0 = S + c0 + cb;
-  for (int q = 0; q < NQ; ++q) {
+  auto keys_q4 = [&](int q) {
     const uint4 k4 = *reinterpret_cast<const uint4 *>(keys + chunk_word<KPT>(t, q));
     const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
@@ -446,6 +459,12 @@ __global__ void __launch_bounds__(kTailThreads, 1) cluster_tail_kernel(const __g
         }
       }
     }
+  };
+  if (nmine == KPT) {
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) keys_q4(q);
+  } else {
+    for (int q = 0; 4 * q < nmine; ++q) keys_q4(q);
   }
 }
 
